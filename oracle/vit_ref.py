@@ -1,0 +1,307 @@
+"""Plain float64 CPU oracle of the ViT vision tower and its 2x2-merge projector.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this module.  The CUDA library never calls it, and it
+shares no code with the CUDA library: it imports numpy and nothing else.
+
+Every function is the plain definition of one step, in float64, in raster token order
+(token (t, h, w) at index t*gh*gw + h*gw + w), written to be checked by eye against
+the passage it cites.  Inputs are the same seeded numbers the GPU receives: bf16
+weights and activations converted exactly to float64, fp32 pixels converted to float64.
+The oracle rounds nothing itself.
+
+Sources (web pages on the MiniMax-M3 vision tower):
+  * "MiniMax-M3 Vision" model card, Architecture table: CLIP-style ViT, 32 layers,
+    hidden 1280, 16 heads, intermediate 5120, patch 14, Conv3d patch embed, 3D RoPE,
+    GELU; 2x2 spatial merge with temporal patch 2; projector Linear(1280,6144), GELU,
+    Linear(6144,6144), flatten four 6144-wide patches, Linear(24576,6144), GELU,
+    Linear(6144,6144).  Same card, Architecture notes: 1280-wide tower tokens,
+    5120-wide merged tokens (2x2 of 1280), 6144-wide projected tokens at 448.
+  * "v2_loaders - Differentiable Vision Tower Loaders (spark2)", section 3 (MiniMax-M3
+    vision tower): the frame is repeated to temporal depth 2, grid_thw = [t, h, w],
+    3D RoPE with rope_theta 10000.
+  * "spark_model/layers/vision_encoder/enc_impl/init.rs" (VisionEncoder::new): per-axis
+    RoPE inverse frequencies inv_freq[k] = theta^(-2k/dim), k < dim/2; ViT attention
+    over a full [seq, seq] score matrix per head, i.e. the dense, non-causal softmax.
+  * "metrale_model_arch/weight_loader/qwen3_vl.rs" (load_vision_encoder): a ViT block
+    holds norm1, qkv, proj, norm2, fc1, fc2, each with weight and bias (pre-LN block).
+
+Readings where the pages are silent (each is also checked by a pin in
+tests/test_oracle_pins.py):
+  * 3D RoPE: head channels split into contiguous blocks [t | h | w] of sizes
+    ``rope_sections``; inside a block of size s, channel pair (j, j + s/2) is rotated
+    by angle pos_axis * theta^(-2j/s) (rotate-half pairing).  Image positions are
+    (t=0, h=row, w=col).
+  * LayerNorm eps 1e-6, GELU in its tanh form, no CLS token, no absolute position
+    embedding, no LayerNorm before or after the tower.
+  * 2x2 merge: merged token (i, j) concatenates tokens (2i,2j), (2i,2j+1), (2i+1,2j),
+    (2i+1,2j+1) in that order; merged tokens are in raster (i, j) order.
+  * Images of a batch are independent (attention never crosses images).
+
+Parity with the real MiniMax-M3 weights is not checked here (no trained weights or
+reference outputs exist on the pages); every function below is pinned against
+mathematics, library routines or brute force in the pin tests.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "token_grid", "patch_unfold", "patch_embed", "layer_norm", "gelu",
+    "rope_inv_freq", "positions_raster", "apply_rope_3d", "attention",
+    "attention_probs", "tower_layer", "merge_2x2", "projector", "forward",
+    "block_order", "merge_source_map",
+]
+
+
+# ----------------------------------------------------------------------- shapes
+
+def token_grid(image_hw: tuple[int, int], patch: int = 14, merge: int = 2,
+               frames: int = 1, temporal_patch: int = 2) -> dict:
+    """Token counts of one image (model card, Architecture: patch 14, 2x2 merge).
+
+    A single frame is repeated up to ``temporal_patch`` frames (v2_loaders FINDINGS,
+    section 3), so one image gives t = 1.
+    """
+    H, W = image_hw
+    if H % (patch * merge) or W % (patch * merge):
+        raise ValueError("image side must be a multiple of patch * merge")
+    t = max(1, -(-frames // temporal_patch))
+    gh, gw = H // patch, W // patch
+    n = t * gh * gw
+    return dict(t=t, h=gh, w=gw, tokens=n, merged=n // (merge * merge))
+
+
+# ----------------------------------------------------------- patch embedding
+
+def patch_unfold(image: np.ndarray, patch: int = 14, temporal_patch: int = 2) -> np.ndarray:
+    """One image [3, H, W] -> patch vectors [gh*gw, 3*tp*patch*patch] in raster order.
+
+    v2_loaders FINDINGS, section 3: the temporal dimension is padded to 2 by repeating
+    the frame.  Model card, Architecture: Conv3d patch embedding with patch 14 and
+    temporal patch 2.  The vector of patch (h, w) lists the pixels in (c, t, kh, kw)
+    order, the order of a Conv3d weight [hidden, 3, tp, patch, patch] flattened.
+    """
+    C, H, W = image.shape
+    gh, gw = H // patch, W // patch
+    out = np.empty((gh * gw, C * temporal_patch * patch * patch), dtype=np.float64)
+    for h in range(gh):
+        for w in range(gw):
+            block = image[:, h * patch:(h + 1) * patch, w * patch:(w + 1) * patch]
+            clip = np.stack([block] * temporal_patch, axis=1)  # [C, tp, p, p]
+            out[h * gw + w] = clip.reshape(-1)
+    return out
+
+
+def patch_embed(patches: np.ndarray, weight: np.ndarray, bias: np.ndarray) -> np.ndarray:
+    """Conv3d with kernel = stride = (tp, p, p) as a matrix product (model card,
+    Architecture: Conv3d patch embed).  weight is [hidden, 3, tp, p, p]."""
+    return patches @ weight.reshape(weight.shape[0], -1).T + bias
+
+
+# ------------------------------------------------------- normalisation, GELU
+
+def layer_norm(x: np.ndarray, gamma: np.ndarray, beta: np.ndarray, eps: float) -> np.ndarray:
+    """Affine LayerNorm over the last axis (pre-LN CLIP-style block: norm1 / norm2 in
+    the qwen3_vl.rs ViTBlock; model card: CLIP-style ViT)."""
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * gamma + beta
+
+
+def gelu(x: np.ndarray, tanh_form: bool = True) -> np.ndarray:
+    """GELU (model card, Architecture).  tanh form:
+    0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))); exact form: x Phi(x)."""
+    if tanh_form:
+        return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+    from math import erf, sqrt
+    return x * 0.5 * (1.0 + np.vectorize(erf)(x / sqrt(2.0)))
+
+
+# ---------------------------------------------------------------------- RoPE
+
+def rope_inv_freq(dim: int, theta: float) -> np.ndarray:
+    """inv_freq[k] = theta^(-2k/dim) for k < dim/2 (init.rs, VisionEncoder::new,
+    RoPE inverse-frequency table), applied per axis section."""
+    k = np.arange(dim // 2, dtype=np.float64)
+    return theta ** (-2.0 * k / dim)
+
+
+def positions_raster(t: int, h: int, w: int) -> np.ndarray:
+    """(t, h, w) position of every token in raster order, shape [t*h*w, 3]."""
+    tt, hh, ww = np.meshgrid(np.arange(t), np.arange(h), np.arange(w), indexing="ij")
+    return np.stack([tt.ravel(), hh.ravel(), ww.ravel()], axis=1).astype(np.int64)
+
+
+def apply_rope_3d(x: np.ndarray, pos: np.ndarray, sections, theta: float) -> np.ndarray:
+    """3D rotary embedding (v2_loaders FINDINGS section 3: rope_mode 3d, theta 10000).
+
+    x: [N, H, D]; pos: [N, 3] integer (t, h, w).  Channels [0, s_t) follow t,
+    [s_t, s_t+s_h) follow h, the rest follow w.  In a block of size s starting at
+    ``off``, the pair (off+j, off+j+s/2) is the 2-vector (a, b) rotated by the angle
+    phi = pos_axis * theta^(-2j/s):  a' = a cos phi - b sin phi,  b' = b cos phi + a sin phi.
+    """
+    assert sum(sections) == x.shape[-1]
+    out = x.copy()
+    off = 0
+    for axis, s in enumerate(sections):
+        half = s // 2
+        phi = pos[:, axis:axis + 1].astype(np.float64) * rope_inv_freq(s, theta)[None, :]
+        c = np.cos(phi)[:, None, :]
+        sn = np.sin(phi)[:, None, :]
+        a = x[:, :, off:off + half]
+        b = x[:, :, off + half:off + s]
+        out[:, :, off:off + half] = a * c - b * sn
+        out[:, :, off + half:off + s] = b * c + a * sn
+        off += s
+    return out
+
+
+# ----------------------------------------------------------------- attention
+
+def attention_probs(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """softmax(q k^T * scale) over keys for one head; q [n, D], k [N, D] -> [n, N]."""
+    s = (q @ k.T) * scale
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+              rows=None, row_block: int = 512) -> np.ndarray:
+    """Bidirectional multi-head attention: O_h = softmax(q_h k_h^T * scale) v_h.
+
+    init.rs (VisionScratch): the ViT attention is a full [seq, seq] score matrix per
+    head followed by a row softmax, i.e. the dense non-causal definition.
+    q, k, v: [H, N, D].  Returns [n, H, D] for the query rows ``rows`` (all rows by
+    default).  Rows are processed ``row_block`` at a time only to bound memory; each
+    row's arithmetic is the definition itself.
+    """
+    H, N, D = q.shape
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.empty((len(rows), H, v.shape[-1]), dtype=np.float64)
+    for h in range(H):
+        for s0 in range(0, len(rows), row_block):
+            r = rows[s0:s0 + row_block]
+            out[s0:s0 + len(r), h] = attention_probs(q[h, r], k[h], scale) @ v[h]
+    return out
+
+
+# --------------------------------------------------------------- tower layer
+
+def tower_layer(x: np.ndarray, w: dict, i: int, cfg: dict, pos: np.ndarray | None) -> np.ndarray:
+    """One pre-LN ViT block on one image's tokens x [N, hidden] (qwen3_vl.rs ViTBlock:
+    norm1, qkv, proj, norm2, fc1, fc2; model card: CLIP-style, GELU, 3D RoPE).
+
+        x = x + O( MHA( RoPE(q), RoPE(k), v ) ),  [q|k|v] = LN1(x) Wqkv^T + bqkv
+        x = x + fc2( GELU( fc1( LN2(x) ) ) )
+
+    q, k, v are the three consecutive ``hidden``-wide column blocks of the qkv output;
+    head h is columns [h*D, (h+1)*D) of each.  ``pos`` None means no rotary embedding.
+    """
+    p = f"layers.{i}."
+    N, d = x.shape
+    H, D = cfg["heads"], cfg["head_dim"]
+    xn = layer_norm(x, w[p + "ln1.weight"], w[p + "ln1.bias"], cfg["ln_eps"])
+    qkv = xn @ w[p + "attn.qkv.weight"].T + w[p + "attn.qkv.bias"]
+    q = qkv[:, 0 * d:1 * d].reshape(N, H, D)
+    k = qkv[:, 1 * d:2 * d].reshape(N, H, D)
+    v = qkv[:, 2 * d:3 * d].reshape(N, H, D)
+    if pos is not None:
+        q = apply_rope_3d(q, pos, cfg["rope_sections"], cfg["rope_theta"])
+        k = apply_rope_3d(k, pos, cfg["rope_sections"], cfg["rope_theta"])
+    o = attention(q.transpose(1, 0, 2), k.transpose(1, 0, 2), v.transpose(1, 0, 2),
+                  1.0 / np.sqrt(D)).reshape(N, d)
+    x = x + o @ w[p + "attn.o.weight"].T + w[p + "attn.o.bias"]
+    xn = layer_norm(x, w[p + "ln2.weight"], w[p + "ln2.bias"], cfg["ln_eps"])
+    hmid = gelu(xn @ w[p + "mlp.fc1.weight"].T + w[p + "mlp.fc1.bias"], cfg["gelu_tanh"])
+    return x + hmid @ w[p + "mlp.fc2.weight"].T + w[p + "mlp.fc2.bias"]
+
+
+# ------------------------------------------------------- merge and projector
+
+def merge_2x2(x: np.ndarray, t: int, h: int, w: int) -> np.ndarray:
+    """2x2 spatial merge (model card: "2x2 spatial merge"; 5120-wide merged tokens are
+    2x2 of 1280).  x [t*h*w, C] raster -> [t*(h/2)*(w/2), 4C]; merged (i, j)
+    concatenates tokens (2i,2j), (2i,2j+1), (2i+1,2j), (2i+1,2j+1)."""
+    C = x.shape[1]
+    g = x.reshape(t, h, w, C)
+    out = np.empty((t, h // 2, w // 2, 4 * C), dtype=x.dtype)
+    for i in range(h // 2):
+        for j in range(w // 2):
+            out[:, i, j] = np.concatenate(
+                [g[:, 2 * i, 2 * j], g[:, 2 * i, 2 * j + 1],
+                 g[:, 2 * i + 1, 2 * j], g[:, 2 * i + 1, 2 * j + 1]], axis=-1)
+    return out.reshape(t * (h // 2) * (w // 2), 4 * C)
+
+
+def projector(x: np.ndarray, w: dict, cfg: dict, t: int, h: int, w_: int) -> np.ndarray:
+    """Projector (model card, Architecture): Linear(d, P), GELU, Linear(P, P) on every
+    tower token; flatten the four P-wide tokens of each 2x2 group (4P wide);
+    Linear(4P, P), GELU, Linear(P, P_out)."""
+    g = cfg["proj_gelu_tanh"]
+    y = gelu(x @ w["proj.patch_fc1.weight"].T + w["proj.patch_fc1.bias"], g)
+    y = y @ w["proj.patch_fc2.weight"].T + w["proj.patch_fc2.bias"]
+    ym = merge_2x2(y, t, h, w_)
+    z = gelu(ym @ w["proj.merge_fc1.weight"].T + w["proj.merge_fc1.bias"], g)
+    return z @ w["proj.merge_fc2.weight"].T + w["proj.merge_fc2.bias"]
+
+
+# ------------------------------------------------------------------- forward
+
+def forward(pixels: np.ndarray, w: dict, cfg: dict, keep_layers: bool = False,
+            layers: int | None = None) -> dict:
+    """Tower + merge + projector for a batch of images pixels [B, 3, H, W].
+
+    Returns dict(tower=[B, N, d], merged=[B, N/4, 4d], out=[B, N/4, P_out]) and, with
+    ``keep_layers``, ``layer_in`` / ``layer_out`` lists of [B, N, d] per layer.
+    ``layers`` runs only the first layers (used for bounded CPU timing).
+    """
+    B = pixels.shape[0]
+    p, tp = cfg["patch"], cfg["temporal_patch"]
+    L = cfg["layers"] if layers is None else layers
+    tows, merged, outs = [], [], []
+    lin = [[] for _ in range(L)]
+    lout = [[] for _ in range(L)]
+    for b in range(B):
+        img = pixels[b].astype(np.float64)
+        gh, gw = img.shape[1] // p, img.shape[2] // p
+        pos = positions_raster(1, gh, gw) if cfg.get("use_rope", True) else None
+        x = patch_embed(patch_unfold(img, p, tp), w["embeddings.proj.weight"],
+                        w["embeddings.proj.bias"])
+        for i in range(L):
+            if keep_layers:
+                lin[i].append(x)
+            x = tower_layer(x, w, i, cfg, pos)
+            if keep_layers:
+                lout[i].append(x)
+        tows.append(x)
+        merged.append(merge_2x2(x, 1, gh, gw))
+        outs.append(projector(x, w, cfg, 1, gh, gw))
+    res = dict(tower=np.stack(tows), merged=np.stack(merged), out=np.stack(outs))
+    if keep_layers:
+        res["layer_in"] = [np.stack(a) for a in lin]
+        res["layer_out"] = [np.stack(a) for a in lout]
+    return res
+
+
+# ----------------------------------------------------------------- index maps
+
+def block_order(t: int, h: int, w: int) -> np.ndarray:
+    """Raster index of the token at each position of 2x2-block order: the four tokens
+    of merged group (i, j) are consecutive, in the merge's member order, and the groups
+    follow raster (i, j) order.  Used only to compare index maps exactly."""
+    out = []
+    for tt in range(t):
+        for i in range(h // 2):
+            for j in range(w // 2):
+                for di in (0, 1):
+                    for dj in (0, 1):
+                        out.append(tt * h * w + (2 * i + di) * w + (2 * j + dj))
+    return np.asarray(out, dtype=np.int64)
+
+
+def merge_source_map(t: int, h: int, w: int) -> np.ndarray:
+    """[t*(h/2)*(w/2), 4] raster indices of the four tokens each merged token gathers."""
+    idx = np.arange(t * h * w, dtype=np.int64)[:, None]
+    return merge_2x2(idx, t, h, w).astype(np.int64)

@@ -1,0 +1,380 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Each test checks one oracle function against brute force, a library routine, a closed
+form, an invariant of the mathematics, or a shape fact the pages print
+(tests/golden/shape_facts.json).  The set is chosen so that a dropped term, a wrong
+sign or index, or a transposed operand in the oracle fails at least one test.
+CPU only.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import vit_ref as R
+from vision_transformer_encoder_vit_b200 import synthetic as S
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "shape_facts.json")
+torch.set_default_dtype(torch.float64)
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ------------------------------------------------------------------ attention
+
+def _attention_brute(q, k, v, scale):
+    """Scalar loops over (query i, key j, channel c) with math.exp; no numpy algebra."""
+    H, N, D = q.shape
+    Dv = v.shape[2]
+    out = np.zeros((N, H, Dv))
+    for h in range(H):
+        for i in range(N):
+            s = []
+            for j in range(N):
+                acc = 0.0
+                for c in range(D):
+                    acc += q[h, i, c] * k[h, j, c]
+                s.append(acc * scale)
+            mx = max(s)
+            e = [math.exp(x - mx) for x in s]
+            tot = sum(e)
+            for c in range(Dv):
+                acc = 0.0
+                for j in range(N):
+                    acc += e[j] / tot * v[h, j, c]
+                out[i, h, c] = acc
+    return out
+
+
+@pytest.mark.parametrize("H,N,D", [(1, 1, 4), (2, 7, 5), (3, 17, 8), (1, 64, 6)])
+def test_attention_matches_brute_force(H, N, D):
+    r = _rng(N * 31 + D)
+    q, k, v = (r.standard_normal((H, N, D)) for _ in range(3))
+    scale = 1 / math.sqrt(D)
+    np.testing.assert_allclose(R.attention(q, k, v, scale), _attention_brute(q, k, v, scale),
+                               rtol=0, atol=1e-12)
+
+
+def test_attention_brute_force_tiny_config_shape():
+    # The tiny tower's attention shape: 4 heads of 32 over 64 tokens.
+    r = _rng(5)
+    q, k, v = (r.standard_normal((4, 64, 32)) * 0.5 for _ in range(3))
+    np.testing.assert_allclose(R.attention(q, k, v, 32 ** -0.5),
+                               _attention_brute(q, k, v, 32 ** -0.5), atol=1e-12, rtol=0)
+
+
+def test_attention_matches_torch_sdpa():
+    r = _rng(1)
+    q, k, v = (r.standard_normal((4, 300, 80)) for _ in range(3))
+    ref = F.scaled_dot_product_attention(torch.tensor(q), torch.tensor(k), torch.tensor(v))
+    got = R.attention(q, k, v, 80 ** -0.5, row_block=37)
+    np.testing.assert_allclose(got.transpose(1, 0, 2), ref.numpy(), atol=1e-12, rtol=0)
+
+
+def test_attention_row_sample_equals_full():
+    r = _rng(2)
+    q, k, v = (r.standard_normal((2, 200, 16)) for _ in range(3))
+    rows = np.array([0, 5, 199, 77])
+    np.testing.assert_allclose(R.attention(q, k, v, 0.25, rows=rows),
+                               R.attention(q, k, v, 0.25)[rows], atol=1e-14, rtol=0)
+
+
+def test_softmax_rows_sum_to_one_and_nonnegative():
+    r = _rng(3)
+    p = R.attention_probs(r.standard_normal((50, 8)) * 4, r.standard_normal((90, 8)) * 4, 0.3)
+    assert (p >= 0).all()
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-12, rtol=0)
+
+
+def test_attention_special_cases():
+    r = _rng(4)
+    H, N, D = 2, 33, 8
+    q, k, v = (r.standard_normal((H, N, D)) for _ in range(3))
+    # a single key: every output row is that key's value
+    o = R.attention(q, k[:, :1], v[:, :1], 0.5)
+    np.testing.assert_allclose(o, np.broadcast_to(v[:, :1].transpose(1, 0, 2), o.shape), atol=1e-12)
+    # all keys equal: uniform weights, output is the mean of the values
+    keq = np.broadcast_to(k[:, :1], k.shape)
+    o = R.attention(q, keq, v, 0.5)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=1)[None], o.shape), atol=1e-12)
+    # V = 1 gives 1; a one-hot value column j reveals the probabilities of key j
+    np.testing.assert_allclose(R.attention(q, k, np.ones_like(v), 0.5), 1.0, atol=1e-12)
+    j = 11
+    vj = np.zeros((H, N, 1))
+    vj[:, j, 0] = 1.0
+    o = R.attention(q, k, vj, 0.5)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h, 0], R.attention_probs(q[h], k[h], 0.5)[:, j], atol=1e-14)
+
+
+def test_attention_is_noncausal():
+    # The last key must influence the first query (no causal mask).
+    r = _rng(6)
+    q, k, v = (r.standard_normal((1, 10, 4)) for _ in range(3))
+    v2 = v.copy()
+    v2[0, -1] += 1.0
+    assert abs(R.attention(q, k, v2, 0.5)[0] - R.attention(q, k, v, 0.5)[0]).max() > 1e-6
+
+
+# ----------------------------------------------------------------------- RoPE
+
+def test_rope_hand_values():
+    # sections (8, 12, 12) of head_dim 32: channel 8 starts the h block (half 6),
+    # channel 20 starts the w block (half 6), channel 0 the t block (half 4).
+    sec, th = (8, 12, 12), 10000.0
+    pos = np.array([[3, 1, 2]])
+    cases = [  # (input channel, axis position, freq index j, block half, block offset)
+        (8, 1, 0, 6, 8), (9, 1, 1, 6, 8), (20, 2, 0, 6, 20), (23, 2, 3, 6, 20), (1, 3, 1, 4, 0)]
+    for ch, p, j, half, off in cases:
+        x = np.zeros((1, 1, 32))
+        x[0, 0, ch] = 1.0
+        y = R.apply_rope_3d(x, pos, sec, th)[0, 0]
+        block = 2 * half
+        phi = p * th ** (-2.0 * j / block)
+        exp = np.zeros(32)
+        exp[ch] = math.cos(phi)
+        exp[ch + half] = math.sin(phi)
+        np.testing.assert_allclose(y, exp, atol=1e-15)
+        # the second member of a pair turns the other way: e_b -> (-sin, cos)
+        x = np.zeros((1, 1, 32))
+        x[0, 0, ch + half] = 1.0
+        y = R.apply_rope_3d(x, pos, sec, th)[0, 0]
+        exp = np.zeros(32)
+        exp[ch] = -math.sin(phi)
+        exp[ch + half] = math.cos(phi)
+        np.testing.assert_allclose(y, exp, atol=1e-15)
+
+
+def test_rope_inv_freq_closed_form():
+    np.testing.assert_allclose(R.rope_inv_freq(32, 10000.0)[[0, 1, 15]],
+                               [1.0, 10000.0 ** (-1 / 16), 10000.0 ** (-15 / 16)], rtol=1e-15)
+
+
+@pytest.mark.parametrize("sec,D", [((16, 32, 32), 80), ((8, 12, 12), 32)])
+def test_rope_invariants(sec, D):
+    r = _rng(D)
+    N, H = 40, 3
+    x = r.standard_normal((N, H, D))
+    pos = np.stack([np.zeros(N, int), r.integers(0, 150, N), r.integers(0, 150, N)], 1)
+    y = R.apply_rope_3d(x, pos, sec, 10000.0)
+    # norm preserved per head vector
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+    # position (0,0,0) is the identity
+    np.testing.assert_array_equal(R.apply_rope_3d(x, np.zeros_like(pos), sec, 10000.0), x)
+    # t = 0 leaves the t block unchanged
+    np.testing.assert_array_equal(y[..., :sec[0]], x[..., :sec[0]])
+    # q.k depends only on the position offset: shift all positions by (0, dh, dw)
+    k = r.standard_normal((N, H, D))
+    d1 = np.einsum("nhd,mhd->hnm", y, R.apply_rope_3d(k, pos, sec, 10000.0))
+    shift = pos + np.array([0, 7, 13])
+    d2 = np.einsum("nhd,mhd->hnm", R.apply_rope_3d(x, shift, sec, 10000.0),
+                   R.apply_rope_3d(k, shift, sec, 10000.0))
+    np.testing.assert_allclose(d1, d2, atol=1e-10)
+
+
+def test_rope_positions_raster():
+    p = R.positions_raster(1, 3, 4)
+    assert p.shape == (12, 3)
+    assert tuple(p[5]) == (0, 1, 1) and tuple(p[11]) == (0, 2, 3)
+
+
+# ------------------------------------------------------ LayerNorm and GELU
+
+def test_layer_norm_matches_torch_and_standardises():
+    r = _rng(7)
+    x = r.standard_normal((20, 1280)) * 3 + 1.5
+    g, b = r.standard_normal(1280), r.standard_normal(1280)
+    ref = F.layer_norm(torch.tensor(x), (1280,), torch.tensor(g), torch.tensor(b), eps=1e-6)
+    np.testing.assert_allclose(R.layer_norm(x, g, b, 1e-6), ref.numpy(), atol=1e-12)
+    z = R.layer_norm(x, np.ones(1280), np.zeros(1280), 1e-6)
+    np.testing.assert_allclose(z.mean(axis=1), 0, atol=1e-12)
+    np.testing.assert_allclose(z.var(axis=1), 1, atol=1e-6)
+
+
+def test_gelu_matches_torch_and_identities():
+    x = np.linspace(-8, 8, 1001)
+    ref = F.gelu(torch.tensor(x), approximate="tanh").numpy()
+    np.testing.assert_allclose(R.gelu(x, True), ref, atol=1e-14)
+    np.testing.assert_allclose(R.gelu(x, False), F.gelu(torch.tensor(x)).numpy(), atol=1e-14)
+    assert R.gelu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(R.gelu(x) - R.gelu(-x), x, atol=1e-14)
+
+
+# ----------------------------------------------------------- patch embedding
+
+@pytest.mark.parametrize("H,W", [(28, 56), (112, 112)])
+def test_patch_embed_equals_conv3d(H, W):
+    r = _rng(H + W)
+    img = r.standard_normal((3, H, W))
+    wt = r.standard_normal((24, 3, 2, 14, 14)) * 0.02
+    bias = r.standard_normal(24)
+    got = R.patch_embed(R.patch_unfold(img, 14, 2), wt, bias)  # [gh*gw, 24]
+    clip = torch.tensor(np.stack([img, img], axis=1))[None]  # [1, 3, 2, H, W]: frame repeated
+    ref = F.conv3d(clip, torch.tensor(wt), torch.tensor(bias), stride=(2, 14, 14))  # [1,24,1,gh,gw]
+    ref = ref[0, :, 0].reshape(24, -1).T.numpy()
+    np.testing.assert_allclose(got, ref, atol=1e-12)
+
+
+def test_patch_unfold_layout():
+    img = np.arange(3 * 28 * 42, dtype=np.float64).reshape(3, 28, 42)
+    u = R.patch_unfold(img, 14, 2)
+    assert u.shape == (6, 1176)
+    # patch (h=1, w=2) is raster index 5; element (c=2, t=1, kh=3, kw=4)
+    assert u[5, 2 * 392 + 1 * 196 + 3 * 14 + 4] == img[2, 14 + 3, 28 + 4]
+    np.testing.assert_array_equal(u[:, :196], u[:, 196:392])  # repeated frame
+
+
+# --------------------------------------------------------------------- merge
+
+def test_merge_matches_brute_force_and_maps():
+    t, h, w, C = 2, 4, 6, 3
+    x = np.arange(t * h * w * C, dtype=np.float64).reshape(t * h * w, C)
+    m = R.merge_2x2(x, t, h, w)
+    assert m.shape == (t * h * w // 4, 4 * C)
+    for tt in range(t):
+        for i in range(h // 2):
+            for j in range(w // 2):
+                row = m[tt * (h // 2) * (w // 2) + i * (w // 2) + j]
+                srcs = [(2 * i, 2 * j), (2 * i, 2 * j + 1), (2 * i + 1, 2 * j), (2 * i + 1, 2 * j + 1)]
+                for a, (hh, ww) in enumerate(srcs):
+                    np.testing.assert_array_equal(row[a * C:(a + 1) * C], x[tt * h * w + hh * w + ww])
+    # the block order lists each merged group's members consecutively
+    bo = R.block_order(t, h, w)
+    np.testing.assert_array_equal(bo.reshape(-1, 4), R.merge_source_map(t, h, w))
+    assert sorted(bo.tolist()) == list(range(t * h * w))
+
+
+# ----------------------------------------------------------- layer, projector
+
+def _layer_weights(cfg, seed, affine=True):
+    return S.weights_f64(S.make_weights(cfg, seed=seed, affine=affine, layers=1))
+
+
+def test_layer_without_rope_matches_torch_modules():
+    cfg = S.get_config("tiny", use_rope=False)
+    w = _layer_weights(cfg, 11)
+    d, H = cfg["hidden"], cfg["heads"]
+    r = _rng(12)
+    x = r.standard_normal((64, d))
+    mha = torch.nn.MultiheadAttention(d, H, bias=True, batch_first=True)
+    ln1, ln2 = torch.nn.LayerNorm(d, eps=1e-6), torch.nn.LayerNorm(d, eps=1e-6)
+    fc1, fc2 = torch.nn.Linear(d, cfg["mlp"]), torch.nn.Linear(cfg["mlp"], d)
+    T = torch.tensor
+    with torch.no_grad():
+        mha.in_proj_weight.copy_(T(w["layers.0.attn.qkv.weight"]))
+        mha.in_proj_bias.copy_(T(w["layers.0.attn.qkv.bias"]))
+        mha.out_proj.weight.copy_(T(w["layers.0.attn.o.weight"]))
+        mha.out_proj.bias.copy_(T(w["layers.0.attn.o.bias"]))
+        for mod, nm in ((ln1, "ln1"), (ln2, "ln2")):
+            mod.weight.copy_(T(w[f"layers.0.{nm}.weight"]))
+            mod.bias.copy_(T(w[f"layers.0.{nm}.bias"]))
+        for mod, nm in ((fc1, "fc1"), (fc2, "fc2")):
+            mod.weight.copy_(T(w[f"layers.0.mlp.{nm}.weight"]))
+            mod.bias.copy_(T(w[f"layers.0.mlp.{nm}.bias"]))
+        xt = T(x)[None]
+        a = ln1(xt)
+        xt = xt + mha(a, a, a, need_weights=False)[0]
+        xt = xt + fc2(F.gelu(fc1(ln2(xt)), approximate="tanh"))
+    np.testing.assert_allclose(R.tower_layer(x, w, 0, cfg, None), xt[0].numpy(), atol=1e-11)
+
+
+def test_layer_permutation_equivariance_and_translation_invariance():
+    cfg = S.get_config("tiny")
+    w = _layer_weights(cfg, 13)
+    r = _rng(14)
+    x = r.standard_normal((64, cfg["hidden"]))
+    pos = R.positions_raster(1, 8, 8)
+    perm = r.permutation(64)
+    # RoPE off: permuting the tokens permutes the output
+    y = R.tower_layer(x, w, 0, cfg, None)
+    np.testing.assert_allclose(R.tower_layer(x[perm], w, 0, cfg, None), y[perm], atol=1e-12)
+    # RoPE on: the same holds when positions travel with their tokens
+    y = R.tower_layer(x, w, 0, cfg, pos)
+    np.testing.assert_allclose(R.tower_layer(x[perm], w, 0, cfg, pos[perm]), y[perm], atol=1e-12)
+    # RoPE makes attention depend on relative position only: a common shift of all
+    # positions leaves the block's output unchanged (fails if v were rotated, or only
+    # one of q, k)
+    np.testing.assert_allclose(R.tower_layer(x, w, 0, cfg, pos + np.array([0, 5, 9])), y, atol=1e-10)
+    # and RoPE is not a no-op
+    assert abs(R.tower_layer(x, w, 0, cfg, None) - y).max() > 1e-6
+
+
+def test_projector_matches_torch_modules():
+    cfg = S.get_config("tiny")
+    w = S.weights_f64(S.make_weights(cfg, seed=21, affine=True, layers=0))
+    r = _rng(22)
+    gh = gw = 4
+    x = r.standard_normal((gh * gw, cfg["hidden"]))
+    T = torch.tensor
+    xt = T(x)
+    y = F.linear(F.gelu(F.linear(xt, T(w["proj.patch_fc1.weight"]), T(w["proj.patch_fc1.bias"])),
+                        approximate="tanh"),
+                 T(w["proj.patch_fc2.weight"]), T(w["proj.patch_fc2.bias"]))
+    # torch-side 2x2 grouping: [h, w, C] -> [h/2, 2, w/2, 2, C] -> [h/2, w/2, 2, 2, C]
+    g = y.reshape(gh // 2, 2, gw // 2, 2, -1).permute(0, 2, 1, 3, 4).reshape(gh * gw // 4, -1)
+    z = F.linear(F.gelu(F.linear(g, T(w["proj.merge_fc1.weight"]), T(w["proj.merge_fc1.bias"])),
+                        approximate="tanh"),
+                 T(w["proj.merge_fc2.weight"]), T(w["proj.merge_fc2.bias"]))
+    np.testing.assert_allclose(R.projector(x, w, cfg, 1, gh, gw), z.numpy(), atol=1e-12)
+
+
+def test_forward_is_order_independent_under_block_order():
+    # The GPU keeps tokens in 2x2-block order; the tower output, permuted back, must
+    # equal the raster-order tower, because positions travel with the tokens.
+    cfg = S.get_config("tiny")
+    w = S.weights_f64(S.make_weights(cfg, affine=True))
+    px = S.make_pixels(cfg, batch=1).astype(np.float64)
+    ref = R.forward(px, w, cfg)
+    gh, gw = 8, 8
+    bo = R.block_order(1, gh, gw)
+    x = R.patch_embed(R.patch_unfold(px[0], 14, 2), w["embeddings.proj.weight"],
+                      w["embeddings.proj.bias"])[bo]
+    pos = R.positions_raster(1, gh, gw)[bo]
+    for i in range(cfg["layers"]):
+        x = R.tower_layer(x, w, i, cfg, pos)
+    np.testing.assert_allclose(x, ref["tower"][0][bo], atol=1e-11)
+
+
+# ------------------------------------------------------------- shape facts
+
+def test_shape_facts_from_pages():
+    facts = json.load(open(GOLDEN))
+    for e in facts["images"]:
+        g = R.token_grid(tuple(e["image"]), patch=facts["tower"]["patch"])
+        assert (g["t"], g["h"], g["w"]) == tuple(e["grid"]), e["cite"]
+        assert g["tokens"] == e["tokens"], e["cite"]
+        if "merged_tokens" in e:
+            assert g["merged"] == e["merged_tokens"], e["cite"]
+    pj = facts["projector"]
+    assert 4 * pj["hidden_size"] == pj["merged_hidden_size"]
+    cfg = S.get_config("tower448")
+    names = [n for n, _, _ in S.weight_names(cfg) if n.startswith("proj.")]
+    assert len(names) == pj["tensors"]
+
+
+def test_shape_facts_one_full_width_layer_448():
+    # 448x448 -> 1024 tower tokens of 1280 -> 256 merged of 5120 -> 256 x 6144.
+    facts = json.load(open(GOLDEN))["images"][0]
+    cfg = S.get_config("tower448", layers=1)
+    w = S.weights_f64(S.make_weights(cfg, layers=1))
+    px = S.make_pixels(cfg, batch=1).astype(np.float64)
+    res = R.forward(px, w, cfg)
+    assert res["tower"].shape == (1, facts["tokens"], facts["tower_width"])
+    assert res["merged"].shape == (1, facts["merged_tokens"], facts["merged_width"])
+    assert res["out"].shape == (1, facts["merged_tokens"], facts["projected_width"])
+    assert np.isfinite(res["out"]).all()
+
+
+def test_tiny_shape_facts():
+    cfg = S.get_config("tiny")
+    w = S.weights_f64(S.make_weights(cfg))
+    res = R.forward(S.make_pixels(cfg).astype(np.float64), w, cfg)
+    assert res["tower"].shape == (1, 64, 128)
+    assert res["merged"].shape == (1, 16, 512)
+    assert res["out"].shape == (1, 16, 256)
