@@ -49,7 +49,8 @@ import numpy as np
 __all__ = [
     "token_grid", "patch_unfold", "patch_embed", "layer_norm", "gelu",
     "rope_inv_freq", "positions_raster", "apply_rope_3d", "attention",
-    "attention_probs", "tower_layer", "merge_2x2", "projector", "forward",
+    "attention_probs", "tower_layer", "tower_layer_rows", "merge_2x2", "projector",
+    "projector_rows", "forward",
     "block_order", "merge_source_map",
 ]
 
@@ -218,6 +219,33 @@ def tower_layer(x: np.ndarray, w: dict, i: int, cfg: dict, pos: np.ndarray | Non
     return x + hmid @ w[p + "mlp.fc2.weight"].T + w[p + "mlp.fc2.bias"]
 
 
+def tower_layer_rows(x: np.ndarray, w: dict, i: int, cfg: dict, pos: np.ndarray | None,
+                     rows) -> np.ndarray:
+    """tower_layer evaluated only at the token rows ``rows`` (same definition: every
+    key and value still comes from all tokens).  Used to check large images on a
+    sample of outputs."""
+    p = f"layers.{i}."
+    N, d = x.shape
+    H, D = cfg["heads"], cfg["head_dim"]
+    rows = np.asarray(rows)
+    xn = layer_norm(x, w[p + "ln1.weight"], w[p + "ln1.bias"], cfg["ln_eps"])
+    qkv = xn @ w[p + "attn.qkv.weight"].T + w[p + "attn.qkv.bias"]
+    q = qkv[:, 0 * d:1 * d].reshape(N, H, D)
+    k = qkv[:, 1 * d:2 * d].reshape(N, H, D)
+    v = qkv[:, 2 * d:3 * d].reshape(N, H, D)
+    if pos is not None:
+        q = apply_rope_3d(q[rows], pos[rows], cfg["rope_sections"], cfg["rope_theta"])
+        k = apply_rope_3d(k, pos, cfg["rope_sections"], cfg["rope_theta"])
+    else:
+        q = q[rows]
+    o = attention(q.transpose(1, 0, 2), k.transpose(1, 0, 2), v.transpose(1, 0, 2),
+                  1.0 / np.sqrt(D)).reshape(len(rows), d)
+    xr = x[rows] + o @ w[p + "attn.o.weight"].T + w[p + "attn.o.bias"]
+    xn = layer_norm(xr, w[p + "ln2.weight"], w[p + "ln2.bias"], cfg["ln_eps"])
+    hmid = gelu(xn @ w[p + "mlp.fc1.weight"].T + w[p + "mlp.fc1.bias"], cfg["gelu_tanh"])
+    return xr + hmid @ w[p + "mlp.fc2.weight"].T + w[p + "mlp.fc2.bias"]
+
+
 # ------------------------------------------------------- merge and projector
 
 def merge_2x2(x: np.ndarray, t: int, h: int, w: int) -> np.ndarray:
@@ -243,6 +271,19 @@ def projector(x: np.ndarray, w: dict, cfg: dict, t: int, h: int, w_: int) -> np.
     y = gelu(x @ w["proj.patch_fc1.weight"].T + w["proj.patch_fc1.bias"], g)
     y = y @ w["proj.patch_fc2.weight"].T + w["proj.patch_fc2.bias"]
     ym = merge_2x2(y, t, h, w_)
+    z = gelu(ym @ w["proj.merge_fc1.weight"].T + w["proj.merge_fc1.bias"], g)
+    return z @ w["proj.merge_fc2.weight"].T + w["proj.merge_fc2.bias"]
+
+
+def projector_rows(x: np.ndarray, w: dict, cfg: dict, t: int, h: int, w_: int,
+                   merged_rows) -> np.ndarray:
+    """projector evaluated only at the merged tokens ``merged_rows``: each needs just
+    the four tower tokens it gathers (merge_source_map)."""
+    src = merge_source_map(t, h, w_)[np.asarray(merged_rows)]  # [n, 4]
+    g = cfg["proj_gelu_tanh"]
+    y = gelu(x[src.ravel()] @ w["proj.patch_fc1.weight"].T + w["proj.patch_fc1.bias"], g)
+    y = y @ w["proj.patch_fc2.weight"].T + w["proj.patch_fc2.bias"]
+    ym = y.reshape(len(src), -1)
     z = gelu(ym @ w["proj.merge_fc1.weight"].T + w["proj.merge_fc1.bias"], g)
     return z @ w["proj.merge_fc2.weight"].T + w["proj.merge_fc2.bias"]
 

@@ -1,0 +1,144 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads and exports every
+symbol include/vt.h declares, configuration and argument checks return the documented
+status codes, the workspace plan is affine in the token count, and the index maps
+(2x2-block token order, RoPE positions, merge gather) equal the oracle's exactly.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import vit_ref as R
+from vision_transformer_encoder_vit_b200 import synthetic as S
+from vision_transformer_encoder_vit_b200 import vt as V
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "vt.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^VT_API\s+[\w\s\*]+?\b(vt_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = _declared()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(V.lib, n), f"{n} missing from libvt.so"
+        assert n in V.EXPORTED, f"{n} has no binding"
+
+
+def _status(e):
+    return e.value.name
+
+
+def test_create_validates_config():
+    cfg = S.get_config("tower448")
+    h = V.vt_create(cfg)
+    V.vt_destroy(h)
+    bad = [
+        dict(heads=15),                      # heads * head_dim != hidden
+        dict(rope_sections=(16, 32, 30)),    # does not sum to head_dim
+        dict(rope_sections=(15, 33, 32)),    # odd section
+        dict(mlp=0),
+    ]
+    for b in bad:
+        with pytest.raises(V.VtError) as e:
+            V.vt_create(dict(cfg, **b))
+        assert _status(e) == "VT_ERR_INVALID_ARG", b
+    for b in (dict(merge=3), dict(head_dim=64, heads=20, rope_sections=(16, 24, 24))):
+        with pytest.raises(V.VtError) as e:
+            V.vt_create(dict(cfg, **b))
+        assert _status(e) == "VT_ERR_UNSUPPORTED", b
+
+
+def test_forward_before_load_and_grid_errors():
+    h = V.vt_create(S.get_config("tiny"))
+    with pytest.raises(V.VtError) as e:
+        V.vt_forward(h, 16, (1, 8, 8), 1, 16, None, 16, 1 << 20)
+    assert _status(e) == "VT_ERR_NOT_LOADED"
+    for grid, code in [((1, 7, 8), "VT_ERR_SHAPE"), ((2, 8, 8), "VT_ERR_SHAPE"),
+                       ((1, 8, 8194), "VT_ERR_SHAPE"), ((0, 8, 8), "VT_ERR_INVALID_ARG")]:
+        with pytest.raises(V.VtError) as e:
+            V.vt_workspace_bytes(h, 1, grid)
+        assert _status(e) == code, grid
+    with pytest.raises(V.VtError) as e:
+        V.vt_workspace_bytes(h, 0, (1, 8, 8))
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    V.vt_destroy(h)
+
+
+def test_load_weights_rejects_missing_names_without_touching_the_device():
+    h = V.vt_create(S.get_config("tiny"))
+    with pytest.raises(V.VtError) as e:
+        V.vt_load_weights(h, {})
+    assert _status(e) == "VT_ERR_WEIGHT"
+    assert "embeddings.proj.weight" in str(e.value)
+    V.vt_destroy(h)
+
+
+def test_linear_and_attention_argument_checks():
+    with pytest.raises(V.VtError) as e:
+        V.vt_linear(16, 16, None, None, 16, 4, 12, 16, 0)  # N not a multiple of 8
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    with pytest.raises(V.VtError) as e:
+        V.vt_linear(16, 16, None, None, 16, 4, 16, 16, 3)
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    with pytest.raises(V.VtError) as e:
+        V.vt_attention_prepared(16, 16, 16, 8, 16, 1, 1, 8, 48, 0.1)
+    assert _status(e) == "VT_ERR_UNSUPPORTED"
+    with pytest.raises(V.VtError) as e:
+        V.vt_attention_prepared(16, 16, 16, 4, 16, 1, 1, 8, 80, 0.1)  # ld_vt < N
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    with pytest.raises(V.VtError) as e:
+        V.vt_attention(16, 16, 16, 16, 1, 2, 8, 80, 16, (16, 32, 30), 1e4, 0.1, 16, 1 << 30)
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("grid", [(1, 2, 2), (1, 4, 6), (1, 8, 8), (1, 32, 32), (1, 6, 2)])
+def test_index_maps_equal_oracle(grid):
+    order, pos, merge = V.vt_index_maps(grid)
+    np.testing.assert_array_equal(np.asarray(order), R.block_order(*grid))
+    np.testing.assert_array_equal(np.asarray(pos), R.positions_raster(*grid))
+    np.testing.assert_array_equal(np.asarray(merge), R.merge_source_map(*grid))
+
+
+def test_workspace_is_affine_in_tokens():
+    cfg = S.get_config("tower448")
+    h = V.vt_create(cfg)
+    sizes = {}
+    for side in (2, 4, 8, 16, 32, 64, 80, 128, 144, 256):
+        sizes[side * side] = V.vt_workspace_bytes(h, 1, (1, side, side))
+    ns = np.array(sorted(sizes))
+    ws = np.array([sizes[n] for n in ns], dtype=np.float64)
+    # fit ws = a + b * N on the large sizes; every size lies within the per-buffer
+    # 256-byte rounding of that line (no N^2 term)
+    b = (ws[-1] - ws[-3]) / (ns[-1] - ns[-3])
+    a = ws[-1] - b * ns[-1]
+    assert np.all(np.abs(ws - (a + b * ns)) <= 16 * 256), (a, b)
+    # per token: the residual stream x (2d bytes) plus the larger of the tower phase
+    # (LN out, q, k, v^T, o: 5 x 2d, MLP hidden 2m) and the projector phase (two
+    # P-wide activations and a quarter-row merged hidden: 2P + 2P + 2P/4)
+    d, m, P = 1280, 5120, 6144
+    assert b == pytest.approx(2 * d + max(5 * 2 * d + 2 * m, 2 * P + 2 * P + 2 * P / 4), rel=0.01)
+    # the pages' untiled attention alone needs 6 N^2 bytes for scores + probabilities
+    # (25.8 GB at 65536 tokens); the whole forward's workspace here is under 2 GB
+    assert sizes[256 * 256] < 6 * (256 * 256) ** 2 / 10
+    # batch scales the same way
+    assert V.vt_workspace_bytes(h, 8, (1, 32, 32)) <= 8 * sizes[1024] + 16 * 256
+    V.vt_destroy(h)
+
+
+def test_attention_workspace_linear():
+    s1 = V.vt_attention_workspace_bytes(1, 16, 6400, 80)
+    s2 = V.vt_attention_workspace_bytes(1, 16, 65536, 80)
+    assert s1 == 3 * 16 * 80 * 6400 * 2
+    assert s2 == 3 * 16 * 80 * 65536 * 2
+    assert V.vt_attention_workspace_bytes(1, 1, 5, 80) == 3 * 80 * 8 * 2  # ragged N rounds to 8 columns
+
+
+def test_last_error_message_is_thread_local_string():
+    with pytest.raises(V.VtError):
+        V.vt_linear(None, 16, None, None, 16, 4, 16, 16, 0)
+    assert "NULL" in V.vt_last_error()

@@ -378,3 +378,18 @@ def test_tiny_shape_facts():
     assert res["tower"].shape == (1, 64, 128)
     assert res["merged"].shape == (1, 16, 512)
     assert res["out"].shape == (1, 16, 256)
+
+
+def test_row_sampled_layer_and_projector_equal_full():
+    cfg = S.get_config("tiny")
+    w = S.weights_f64(S.make_weights(cfg, seed=31, affine=True, layers=1))
+    x = _rng(32).standard_normal((64, cfg["hidden"]))
+    pos = R.positions_raster(1, 8, 8)
+    rows = np.array([0, 9, 33, 63])
+    np.testing.assert_allclose(R.tower_layer_rows(x, w, 0, cfg, pos, rows),
+                               R.tower_layer(x, w, 0, cfg, pos)[rows], atol=1e-12)
+    np.testing.assert_allclose(R.tower_layer_rows(x, w, 0, cfg, None, rows),
+                               R.tower_layer(x, w, 0, cfg, None)[rows], atol=1e-12)
+    mrows = np.array([0, 5, 15])
+    np.testing.assert_allclose(R.projector_rows(x, w, cfg, 1, 8, 8, mrows),
+                               R.projector(x, w, cfg, 1, 8, 8)[mrows], atol=1e-12)

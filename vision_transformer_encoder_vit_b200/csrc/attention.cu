@@ -1,0 +1,405 @@
+// Bidirectional (non-causal) multi-head attention for sm_100a, flash style:
+// O_h = softmax(q_h k_h^T * scale) v_h per image and head, computed one 128-row
+// query tile per CTA while 128-key tiles stream through a TMA ring.  No [N, N]
+// buffer exists anywhere; memory traffic is q, k, v in and o out.
+//
+// The operation is the ViT self-attention of the "MiniMax-M3 Vision" model card
+// (Architecture table: 16 heads over hidden 1280).  The loader page
+// "spark_model/layers/vision_encoder/enc_impl/init.rs" (VisionScratch and the doc
+// comment of CEILING_MAX_PATCHES) builds the full [seq, seq] score matrix per head and
+// notes that larger images need tiled attention; this kernel is that tiled form.
+//
+// CTA = 6 warps.  Warp 0 issues TMA loads (Q once, then K and V^T tiles).  Warp 1
+// allocates TMEM and issues the MMAs from one thread:
+//     S_j = Q K_j^T          -> TMEM columns [128 * (j & 1), +128)   (fp32)
+//     O  += P_j V_j          -> TMEM columns [256, 256 + D)          (fp32)
+// Warps 2..5 (one thread per query row) run the online softmax: load S_j from TMEM,
+// exponentiate with a lazily updated running maximum, write P_j (bf16) into a
+// 128-byte-swizzled shared tile for the next MMA, rescale O in TMEM only when the
+// maximum grows by more than 2^8, and finally write O / l.
+//
+// Operand layouts: q, k are [B, H, N, D] (D contiguous), used K-major; v is given
+// transposed, vt [B, H, D, ld_vt], so that V_j^T is K-major too.  A head of 80
+// channels is staged as a 64-channel chunk with 128-byte swizzle plus a 16-channel
+// chunk with 32-byte swizzle, so no padding is computed.
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vt {
+namespace {
+
+__device__ unsigned int g_attn_err;
+
+constexpr int kThreads = 192;
+
+__host__ __device__ constexpr uint32_t layout_code(int swizzle_bytes) {
+  return swizzle_bytes == 128 ? 2u : swizzle_bytes == 64 ? 4u : 6u;
+}
+
+template <int D>
+struct AttnShape {
+  static constexpr int BM = 128;  // query rows per CTA
+  static constexpr int BN = 128;  // keys per tile
+  static constexpr int C0 = D >= 64 ? 64 : D;  // channels of chunk 0
+  static constexpr int C1 = D - C0;            // channels of chunk 1 (0 if none)
+  static constexpr int SW0 = C0 * 2, SW1 = C1 * 2;  // row bytes = swizzle span
+  static constexpr uint32_t LAY0 = layout_code(SW0), LAY1 = layout_code(SW1);
+  static constexpr int SBO0 = 8 * SW0, SBO1 = 8 * SW1;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q1_OFF = BM * C0 * 2;
+  static constexpr int K_BYTES = BN * D * 2;
+  static constexpr int K1_OFF = BN * C0 * 2;
+  static constexpr int V_BYTES = D * BN * 2;  // two [D x 64] boxes
+  static constexpr int V1_OFF = D * 64 * 2;
+  static constexpr int KV_BYTES = K_BYTES + V_BYTES;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int AVAIL = 227 * 1024 - 1024 - BAR_BYTES - Q_BYTES - 2 * P_BYTES;
+  static constexpr int STAGES = AVAIL / KV_BYTES > 4 ? 4 : AVAIL / KV_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_BYTES + 2 * P_BYTES + BAR_BYTES;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(C0 == 16 || C0 == 32 || C0 == 64, "chunk 0 width");
+  static_assert(C1 == 0 || C1 == 16 || C1 == 32 || C1 == 64, "chunk 1 width");
+  static_assert(D % 16 == 0 && D <= 128, "head_dim");
+  static_assert(STAGES >= 2, "shared memory");
+  static_assert(Q1_OFF % 1024 == 0 && K1_OFF % 1024 == 0 && V1_OFF % 1024 == 0 && KV_BYTES % 1024 == 0 &&
+                    Q_BYTES % 1024 == 0,
+                "1024-byte alignment of swizzled tiles");
+};
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_test(bar, parity)) {
+    if (global_ns() - t0 > VT_WAIT_LIMIT_NS) {
+      atomicOr(&g_attn_err, VT_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ uint64_t qk_desc(uint32_t tile_addr, int ks) {
+  using S = AttnShape<D>;
+  const int c = ks * 16;
+  if (c < S::C0) return smem_desc(tile_addr + c * 2, S::SBO0, S::LAY0);
+  return smem_desc(tile_addr + S::BM * S::C0 * 2 + (c - S::C0) * 2, S::SBO1, S::LAY1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_tcgen05(const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
+                     const __grid_constant__ CUtensorMap tmK0, const __grid_constant__ CUtensorMap tmK1,
+                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using S = AttnShape<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + S::Q_BYTES;                  // per stage: K tile then V^T tile
+  uint8_t* sP = sKV + S::STAGES * S::KV_BYTES;     // two P tiles
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * S::P_BYTES);
+  uint64_t* q_full = bar;
+  uint64_t* kv_full = bar + 1;
+  uint64_t* kv_empty = kv_full + S::STAGES;
+  uint64_t* s_full = kv_empty + S::STAGES;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* drain = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* armed = const_cast<int*>(abort_flag + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int N = p.N;
+  const int nkv = (N + S::BN - 1) / S::BN;
+  const int bh = b * p.H + h;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      armed[s] = -1;
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    armed[S::STAGES] = -1;  // q tile
+    *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_attn_err) != 0) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort_flag != 0;
+
+  if (!skip && warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- loads
+      tma_prefetch_desc(&tmQ0);
+      tma_prefetch_desc(&tmK0);
+      tma_prefetch_desc(&tmV);
+      const int qrow = bh * N + qt * S::BM;
+      mbar_arrive_expect_tx(q_full, S::Q_BYTES);
+      tma_load_2d(sQ, &tmQ0, q_full, 0, qrow);
+      if (S::C1) tma_load_2d(sQ + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow);
+      armed[S::STAGES] = 0;
+      const int krow = bh * N;
+      const int vrow = bh * D;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % S::STAGES;
+        const uint32_t ph = (j / S::STAGES) & 1;
+        if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, &g_attn_err)) break;
+        uint8_t* sK = sKV + s * S::KV_BYTES;
+        uint8_t* sV = sK + S::K_BYTES;
+        mbar_arrive_expect_tx(&kv_full[s], S::KV_BYTES);
+        tma_load_2d(sK, &tmK0, &kv_full[s], 0, krow + j * S::BN);
+        if (S::C1) tma_load_2d(sK + S::K1_OFF, &tmK1, &kv_full[s], S::C0, krow + j * S::BN);
+        tma_load_2d(sV, &tmV, &kv_full[s], j * S::BN, vrow);
+        tma_load_2d(sV + S::V1_OFF, &tmV, &kv_full[s], j * S::BN + 64, vrow);
+        armed[s] = static_cast<int>(ph);
+      }
+      if (*abort_flag) {
+        if (armed[S::STAGES] >= 0) drain_wait(q_full, 0);
+        for (int s = 0; s < S::STAGES; ++s)
+          if (armed[s] >= 0) drain_wait(&kv_full[s], static_cast<uint32_t>(armed[s]));
+      }
+    }
+  } else if (!skip && warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BN);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D);
+      const uint32_t tO = tmem + 256;
+      const uint32_t q_addr = smem_u32(sQ);
+      bool issued = false;
+      bool ok = mbar_wait(q_full, 0, abort_flag, &g_attn_err);
+      auto issue_pv = [&](int i) -> bool {
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort_flag, &g_attn_err)) return false;
+        tc_fence_after();
+        const uint32_t p_addr = smem_u32(sP + (i & 1) * S::P_BYTES);
+        const uint32_t v_addr = smem_u32(sKV + (i % S::STAGES) * S::KV_BYTES + S::K_BYTES);
+#pragma unroll
+        for (int ks = 0; ks < S::BN / 16; ++ks) {
+          const uint64_t ad = smem_desc(p_addr + (ks >> 2) * (S::BM * 128) + (ks & 3) * 32, 1024, 2);
+          const uint64_t bd = smem_desc(v_addr + (ks >> 2) * S::V1_OFF + (ks & 3) * 32, 1024, 2);
+          umma_bf16(tO, ad, bd, idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[i % S::STAGES]);
+        umma_commit(o_done);
+        return true;
+      };
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % S::STAGES;
+        if (!mbar_wait(&kv_full[s], (j / S::STAGES) & 1, abort_flag, &g_attn_err)) {
+          ok = false;
+          break;
+        }
+        if (j >= 2 && !mbar_wait(&s_free[j & 1], ((j >> 1) - 1) & 1, abort_flag, &g_attn_err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sKV + s * S::KV_BYTES);
+        const uint32_t tS = tmem + (j & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma_bf16(tS, qk_desc<D>(q_addr, ks), qk_desc<D>(k_addr, ks), idesc_s, ks > 0 ? 1u : 0u);
+        issued = true;
+        umma_commit(&s_full[j & 1]);
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) issue_pv(nkv - 1);
+      if (*abort_flag && issued) {
+        umma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else if (!skip) {
+    // ------------------------------------------------------------- softmax
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tO = tmem + 256 + lane_off;
+    const float sl2 = p.scale * 1.4426950408889634f;  // scale * log2(e)
+    float m_ref = -INFINITY;  // running maximum of s * sl2 used as the exponent origin
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int buf = j & 1;
+      if (!mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, &g_attn_err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[S::BN];
+      {
+        uint32_t raw[32];
+#pragma unroll
+        for (int c = 0; c < S::BN; c += 32) {
+          tmem_ld32(tmem + buf * 128 + c + lane_off, raw);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(raw[i]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[buf]);
+      const int valid = N - j * S::BN;
+      if (valid < S::BN) {
+#pragma unroll
+        for (int c = 0; c < S::BN; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < S::BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = mx * sl2;
+      bool need = false;
+      if (j == 0) {
+        m_ref = m_new;
+      } else {
+        need = m_new > m_ref + 8.0f;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        // O must be scaled before P_j V_j accumulates: wait for P_{j-1} V_{j-1}.
+        if (!mbar_wait(o_done, (j - 1) & 1, abort_flag, &g_attn_err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+        if (need) {
+          m_ref = m_new;
+          l *= alpha;
+        }
+#pragma unroll
+        for (int c = 0; c < D; c += 16) {
+          uint32_t o[16];
+          tmem_ld16(tO + c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16(tO + c, o);
+        }
+        tmem_st_wait();
+      }
+      // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
+      uint8_t* pbuf = sP + buf * S::P_BYTES;
+      const float neg = -m_ref;
+#pragma unroll
+      for (int c16 = 0; c16 < S::BN / 8; ++c16) {
+        float e[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          e[i] = fast_exp2(fmaf(s[c16 * 8 + i], sl2, neg));
+          l += e[i];
+        }
+        const int blk = c16 >> 3, cc = c16 & 7;
+        uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+        *dst = pack_bf16x8(e);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[buf]);
+    }
+    if (ok) {
+      // wait for the last two P V products (phases are checked in order)
+      if (nkv >= 2) ok = mbar_wait(o_done, (nkv - 2) & 1, abort_flag, &g_attn_err);
+      if (ok) ok = mbar_wait(o_done, (nkv - 1) & 1, abort_flag, &g_attn_err);
+    }
+    if (ok) {
+      tc_fence_after();
+      float o[D];
+      load_cols<D>(tO, o);
+      const int n = qt * S::BM + r;
+      if (n < N) {
+        const float inv = 1.0f / l;
+#pragma unroll
+        for (int i = 0; i < D; ++i) o[i] *= inv;
+        bf16* dst = static_cast<bf16*>(p.o) + (static_cast<size_t>(b) * N + n) * (p.H * D) + h * D;
+#pragma unroll
+        for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(o + 8 * g);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, S::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
+  using S = AttnShape<D>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_fwd_tcgen05<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const uint64_t rows = static_cast<uint64_t>(p.B) * p.H * p.N;
+  CUtensorMap q0, q1, k0, k1, v;
+  if (!make_tmap_2d(&q0, p.q, rows, D, D, S::BM, S::C0, S::SW0)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&k0, p.k, rows, D, D, S::BN, S::C0, S::SW0)) return cudaErrorInvalidValue;
+  if (S::C1) {
+    if (!make_tmap_2d(&q1, p.q, rows, D, D, S::BM, S::C1, S::SW1)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&k1, p.k, rows, D, D, S::BN, S::C1, S::SW1)) return cudaErrorInvalidValue;
+  } else {
+    q1 = q0;
+    k1 = k0;
+  }
+  if (!make_tmap_2d(&v, p.vt, static_cast<uint64_t>(p.B) * p.H * D, p.N, p.ld_vt, D, 64, 128))
+    return cudaErrorInvalidValue;
+  dim3 grid((p.N + S::BM - 1) / S::BM, p.H, p.B);
+  attn_fwd_tcgen05<D><<<grid, kThreads, S::SMEM_BYTES, stream>>>(q0, q1, k0, k1, v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
+  if (p.B <= 0 || p.H <= 0 || p.N <= 0) return cudaSuccess;
+  switch (p.D) {
+    case 32: return launch_d<32>(p, stream);
+    case 64: return launch_d<64>(p, stream);
+    case 80: return launch_d<80>(p, stream);
+    case 96: return launch_d<96>(p, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+unsigned int attention_read_clear_error(cudaStream_t stream) {
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_attn_err, sizeof(v), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return 0;
+  cudaStreamSynchronize(stream);
+  if (v) {
+    cudaMemcpyToSymbolAsync(g_attn_err, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+    cudaStreamSynchronize(stream);
+  }
+  return v;
+}
+
+}  // namespace vt

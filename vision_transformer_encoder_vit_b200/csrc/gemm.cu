@@ -1,0 +1,346 @@
+// Persistent bf16 GEMM for sm_100a: TMA -> shared-memory ring -> tcgen05.mma (fp32
+// accumulator in TMEM) -> tcgen05.ld epilogue with fused bias / GELU / residual, or
+// with the QKV epilogue that applies 3D RoPE and writes the attention layouts.
+//
+// Computes out[M, N] = act(A[M, K] * W[N, K]^T + bias) (+ resid), the form of every
+// linear layer of the tower and projector ("MiniMax-M3 Vision" model card,
+// Architecture table: Conv3d patch embed, qkv / o projections, MLP 1280 -> 5120 -> 1280
+// with GELU, projector Linear(1280,6144), GELU, Linear(6144,6144), Linear(24576,6144),
+// GELU, Linear(6144,6144)).
+//
+// CTA = 6 warps: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the MMAs
+// (one thread), warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Tiles are 128 x BN with a 64-deep K step (one 128-byte swizzle atom), a
+// STAGES-deep ring of operand tiles, and two TMEM accumulators so that the epilogue
+// of one tile overlaps the main loop of the next.  Tiles are walked m-fastest by a
+// persistent grid (one CTA per SM), so concurrently running CTAs share the same
+// weight tile through L2.
+#include "ptx.cuh"
+#include "internal.h"
+
+namespace vt {
+namespace {
+
+__device__ unsigned int g_gemm_err;
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct GemmShape {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int ACC_COLS = BN <= 128 ? 128 : 256;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tiles must keep 1024-byte alignment");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+// Head layouts the QKV epilogue supports: head_dim and the three RoPE sections.
+struct Rope0 { static constexpr int D = 0, S0 = 0, S1 = 0, S2 = 0; };
+struct Rope80 { static constexpr int D = 80, S0 = 16, S1 = 32, S2 = 32; };
+struct Rope32 { static constexpr int D = 32, S0 = 8, S1 = 12, S2 = 12; };
+
+// Rotates the pairs (off + j, off + j + S/2) of one axis block in place.
+template <int OFF, int S>
+__device__ __forceinline__ void rope_block(float* v, const float2* tab_axis_pos) {
+#pragma unroll
+  for (int j = 0; j < S / 2; ++j) {
+    const float2 cs = tab_axis_pos[j];
+    const float a = v[OFF + j], b = v[OFF + j + S / 2];
+    v[OFF + j] = a * cs.x - b * cs.y;
+    v[OFF + j + S / 2] = b * cs.x + a * cs.y;
+  }
+}
+
+// Bounded wait used only while tearing down after an abort.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_test(bar, parity)) {
+    if (global_ns() - t0 > VT_WAIT_LIMIT_NS) {
+      atomicOr(&g_gemm_err, VT_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int BN, class RL>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmParams p) {
+  using S = GemmShape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S::STAGES * S::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tfull = empty + S::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* armed = const_cast<int*>(abort_flag + 1);  // last phase armed per stage, -1 = never
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m_tiles = (p.M + kBM - 1) / kBM;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int nk = (p.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      armed[s] = -1;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_gemm_err) != 0) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const bool skip = *abort_flag != 0;
+
+  if (!skip && warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int mb = tile % m_tiles, nb = tile / m_tiles;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
+          tma_load_2d(sA + stage * S::A_BYTES, &tmA, &full[stage], kb * kBK, mb * kBM);
+          tma_load_2d(sB + stage * S::B_BYTES, &tmB, &full[stage], kb * kBK, nb * BN);
+          armed[stage] = static_cast<int>(phase);
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {  // let every load already issued land before the CTA exits
+        for (int s = 0; s < S::STAGES; ++s)
+          if (armed[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(armed[s]));
+      }
+    }
+  } else if (!skip && warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------------- MMA
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, &g_gemm_err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, &g_gemm_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * S::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * S::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            umma_bf16(d_tmem, smem_desc(a_addr + kk * 32, 1024, 2), smem_desc(b_addr + kk * 32, 1024, 2), idesc,
+                      (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          umma_commit(&empty[stage]);
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      if (*abort_flag && issued_any) {  // wait for MMAs in flight before TMEM is freed
+        umma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else if (!skip) {
+    // ------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
+      tc_fence_after();
+      const int mb = tile % m_tiles, nb = tile / m_tiles;
+      const int row = mb * kBM + quad * 32 + lane;
+      const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
+      if constexpr (RL::D == 0) {
+        const bf16* bias = static_cast<const bf16*>(p.bias);
+        const bf16* resid = static_cast<const bf16*>(p.resid);
+        bf16* out = static_cast<bf16*>(p.out);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          const int col = nb * BN + c0;
+          if (col >= p.N) break;
+          float v[32];
+          load_cols<32>(t_row + c0, v);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int cg = col + 8 * g;
+            if (cg < p.N) {
+              if (bias) add_bf16x8(v + 8 * g, *reinterpret_cast<const uint4*>(bias + cg));
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float x = v[8 * g + i];
+                if (p.act == ACT_GELU_TANH) x = gelu_tanh(x);
+                else if (p.act == ACT_GELU_ERF) x = gelu_erf(x);
+                v[8 * g + i] = x;
+              }
+              if (row < p.M) {
+                if (resid)
+                  add_bf16x8(v + 8 * g,
+                             *reinterpret_cast<const uint4*>(resid + static_cast<size_t>(row) * p.ldr + cg));
+                *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.ldo + cg) = pack_bf16x8(v + 8 * g);
+              }
+            }
+          }
+        }
+      } else {
+        constexpr int D = RL::D;
+        constexpr int HPT = BN / D;
+        const bf16* bias = static_cast<const bf16*>(p.bias);
+        const int width = p.heads * D;
+        int b = 0, n = 0, tp = 0, hp = 0, wp = 0;
+        if (row < p.M) {
+          b = row / p.ntok;
+          n = row - b * p.ntok;
+          token_position(n, p.gh, p.gw, p.order, &tp, &hp, &wp);
+        }
+#pragma unroll 1
+        for (int hh = 0; hh < HPT; ++hh) {
+          const int col = nb * BN + hh * D;
+          if (col >= p.N) break;
+          float v[D];
+          load_cols<D>(t_row + hh * D, v);
+          if (bias) {
+#pragma unroll
+            for (int g = 0; g < D / 8; ++g) add_bf16x8(v + 8 * g, *reinterpret_cast<const uint4*>(bias + col + 8 * g));
+          }
+          const int which = col / width;
+          const int head = (col - which * width) / D;
+          if (row < p.M) {
+            if (which < 2) {
+              if (p.rope) {
+                const float2* tab = p.rope_tab;
+                rope_block<0, RL::S0>(v, tab + (static_cast<size_t>(0 * kRopeMaxPos + tp) * kRopePairs));
+                rope_block<RL::S0, RL::S1>(v, tab + (static_cast<size_t>(1 * kRopeMaxPos + hp) * kRopePairs));
+                rope_block<RL::S0 + RL::S1, RL::S2>(v, tab + (static_cast<size_t>(2 * kRopeMaxPos + wp) * kRopePairs));
+              }
+              bf16* dst = static_cast<bf16*>(which == 0 ? p.q : p.k) +
+                          ((static_cast<size_t>(b) * p.heads + head) * p.ntok + n) * D;
+#pragma unroll
+              for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(v + 8 * g);
+            } else {
+              bf16* dst = static_cast<bf16*>(p.vt) + (static_cast<size_t>(b) * p.heads + head) * D * p.ld_vt + n;
+#pragma unroll
+              for (int d = 0; d < D; ++d) dst[static_cast<size_t>(d) * p.ld_vt] = __float2bfloat16_rn(v[d]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+template <int BN, class RL>
+cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
+  using S = GemmShape<BN>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05<BN, RL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, p.A, p.M, p.K, p.lda, kBM, kBK, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN, kBK, 128)) return cudaErrorInvalidValue;
+  const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  gemm_bf16_tcgen05<BN, RL><<<grid, kThreads, S::SMEM_BYTES, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) {
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0) return cudaSuccess;
+  if (qkv_mode) {
+    if (p.head_dim == 80 && p.sections[0] == 16 && p.sections[1] == 32 && p.sections[2] == 32)
+      return launch_one<240, Rope80>(p, stream);
+    if (p.head_dim == 32 && p.sections[0] == 8 && p.sections[1] == 12 && p.sections[2] == 12)
+      return launch_one<256, Rope32>(p, stream);
+    return cudaErrorNotSupported;
+  }
+  // Wide tiles when they still fill the SMs; narrower ones for small problems.
+  const int sms = device_sm_count();
+  const long tiles256 = static_cast<long>((p.M + kBM - 1) / kBM) * ((p.N + 255) / 256);
+  if (tiles256 >= sms || p.N > 256 * 8) return launch_one<256, Rope0>(p, stream);
+  return launch_one<128, Rope0>(p, stream);
+}
+
+unsigned int gemm_read_clear_error(cudaStream_t stream) {
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_gemm_err, sizeof(v), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return 0;
+  cudaStreamSynchronize(stream);
+  if (v) {
+    cudaMemcpyToSymbolAsync(g_gemm_err, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+    cudaStreamSynchronize(stream);
+  }
+  return v;
+}
+
+}  // namespace vt

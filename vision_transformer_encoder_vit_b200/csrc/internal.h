@@ -1,0 +1,111 @@
+// Internal declarations shared by the C-ABI layer (vt_api.cpp) and the kernel
+// translation units.  Not part of the public interface (include/vt.h is).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace vt {
+
+// Token order of the activations of one image.
+enum TokenOrder : int { ORDER_RASTER = 0, ORDER_BLOCK = 1 };
+
+// Maximum position along any grid axis that the RoPE tables cover.
+constexpr int kRopeMaxPos = 4096;
+// Pairs per axis the tables hold (head_dim up to 2 * 3 * 32).
+constexpr int kRopePairs = 32;
+
+// Decodes token n of an image with grid (gt, gh, gw) in the given order into its
+// (t, h, w) patch position.  Block order lists the 4 members of every 2x2 group
+// consecutively: (0,0), (0,1), (1,0), (1,1); groups follow raster order.
+__host__ __device__ inline void token_position(int n, int gh, int gw, int order, int* t, int* h, int* w) {
+  const int per_t = gh * gw;
+  *t = n / per_t;
+  const int r = n - *t * per_t;
+  if (order == ORDER_BLOCK) {
+    const int m = r >> 2, q = r & 3, hw2 = gw >> 1;
+    const int i = m / hw2, j = m - (m / hw2) * hw2;
+    *h = 2 * i + (q >> 1);
+    *w = 2 * j + (q & 1);
+  } else {
+    *h = r / gw;
+    *w = r - (r / gw) * gw;
+  }
+}
+
+// ------------------------------------------------------------------ GEMM
+
+enum GemmAct : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2 };
+
+// out[M, N] = act(A[M, K] * W[N, K]^T + bias) (+ resid), bf16 in and out, fp32 accumulate.
+struct GemmParams {
+  int M, N, K;
+  const void* A;      // [M, lda] bf16
+  int lda;            // elements, multiple of 8
+  const void* W;      // [N, ldw] bf16
+  int ldw;
+  const void* bias;   // [N] bf16 or null
+  const void* resid;  // [M, ldr] bf16 or null (may alias out)
+  int ldr;
+  void* out;          // [M, ldo] bf16
+  int ldo;
+  int act;
+  // QKV mode: output columns are [q | k | v], each heads*head_dim wide.  q and k are
+  // rotated (3D RoPE) and written [B, heads, ntok, head_dim]; v is written transposed
+  // [B, heads, head_dim, ld_vt].
+  void* q;
+  void* k;
+  void* vt;
+  int heads, head_dim, ntok, ld_vt;
+  int gt, gh, gw, order;
+  int rope;                 // 0: no rotation
+  int sections[3];
+  const float2* rope_tab;   // [3][kRopeMaxPos][kRopePairs] (cos, sin)
+};
+
+// Returns a CUDA error code (cudaSuccess on success); host-side shape checks are the
+// caller's job.
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode);
+unsigned int gemm_read_clear_error(cudaStream_t stream);
+
+// ------------------------------------------------------------- attention
+
+struct AttnParams {
+  const void* q;   // [B, H, N, D] bf16, rotated
+  const void* k;   // [B, H, N, D] bf16, rotated
+  const void* vt;  // [B, H, D, ld_vt] bf16
+  void* o;         // [B, N, H * D] bf16
+  int B, H, N, D, ld_vt;
+  float scale;
+};
+cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream);
+unsigned int attention_read_clear_error(cudaStream_t stream);
+
+// -------------------------------------------------------- memory-bound ops
+
+cudaError_t launch_layernorm(const void* x, const void* gamma, const void* beta, void* y, int rows, int cols,
+                             float eps, cudaStream_t stream);
+// pixels [B, 3, H, W] fp32 -> patch vectors [B * gh * gw, 3 * tp * p * p] bf16 in `order`.
+cudaError_t launch_patch_unfold(const float* pixels, void* out, int B, int H, int W, int patch, int tp,
+                                int order, cudaStream_t stream);
+// Row gather: out[r] = in[src(r)] where src maps between raster and block order.
+// to_block != 0: out is block order, in is raster.  Rows of `cols` bf16 each.
+cudaError_t launch_reorder_rows(const void* in, void* out, int B, int gt, int gh, int gw, int cols, int to_block,
+                                cudaStream_t stream);
+// q, k [B, H, N, D] -> rotated copies; v [B, H, N, D] -> vt [B, H, D, ld_vt].
+// pos: device [N, 3] int32 (t, h, w) or null for no rotation.
+cudaError_t launch_attention_prep(const void* q, const void* k, const void* v, void* qr, void* kr, void* vt,
+                                  int B, int H, int N, int D, int ld_vt, const int32_t* pos,
+                                  const int sections[3], float theta, cudaStream_t stream);
+
+// -------------------------------------------------------------------- TMA
+
+// Creates a 2D tiled tensor map over a row-major bf16 matrix [rows, cols] with row
+// stride ld (elements) and box [box_rows, box_cols]; swizzle_bytes in {0, 32, 64, 128}.
+bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                  uint32_t box_rows, uint32_t box_cols, int swizzle_bytes);
+
+int device_sm_count();
+
+}  // namespace vt

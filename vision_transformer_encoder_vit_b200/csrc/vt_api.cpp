@@ -1,0 +1,776 @@
+// C ABI of libvt (declared in include/vt.h): handle, configuration checks, weight
+// table, workspace plan, launch sequences, error reporting and launch profiling.
+// Host code only; every step of the computation runs in the kernels of gemm.cu,
+// attention.cu and elementwise.cu.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/vt.h"
+#include "internal.h"
+
+using namespace vt;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+vt_status fail(vt_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+vt_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(VT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int round8(int x) { return (x + 7) & ~7; }
+
+// ---------------------------------------------------------------- profiling
+
+enum { CLS_GEMM = 0, CLS_ATTN = 1, CLS_LN = 2, CLS_UNFOLD = 3, CLS_REORDER = 4, CLS_PREP = 5, CLS_COUNT = 6 };
+
+struct ProfRec {
+  int cls;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  double ms[CLS_COUNT] = {0}, flops[CLS_COUNT] = {0}, bytes[CLS_COUNT] = {0};
+  int64_t n[CLS_COUNT] = {0};
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Profiler g_prof;
+
+// Brackets one launch with events when profiling is on.
+struct ProfScope {
+  int cls;
+  double flops, bytes;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  ProfScope(int c, double f, double b, cudaStream_t s) : cls(c), flops(f), bytes(b), st(s) {
+    if (g_prof.on) {
+      std::lock_guard<std::mutex> l(g_prof.mu);
+      a = g_prof.get();
+      cudaEventRecord(a, st);
+    }
+  }
+  ~ProfScope() {
+    if (a) {
+      std::lock_guard<std::mutex> l(g_prof.mu);
+      cudaEvent_t b = g_prof.get();
+      cudaEventRecord(b, st);
+      g_prof.recs.push_back({cls, a, b, flops, bytes});
+    }
+  }
+};
+
+// ------------------------------------------------------------ kernel calls
+
+vt_status run_gemm(GemmParams p, cudaStream_t st) {
+  ProfScope ps(CLS_GEMM, 2.0 * p.M * static_cast<double>(p.N) * p.K, 0, st);
+  cudaError_t e = launch_gemm(p, st, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return VT_OK;
+}
+
+GemmParams gemm_params(const void* A, int lda, const void* W, int ldw, const void* bias, const void* resid,
+                       int ldr, void* out, int ldo, int M, int N, int K, int act) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.A = A;
+  p.lda = lda;
+  p.W = W;
+  p.ldw = ldw;
+  p.bias = bias;
+  p.resid = resid;
+  p.ldr = ldr;
+  p.out = out;
+  p.ldo = ldo;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.act = act;
+  return p;
+}
+
+vt_status run_layernorm(const void* x, const void* g, const void* b, void* y, int rows, int cols, float eps,
+                        cudaStream_t st) {
+  ProfScope ps(CLS_LN, 0, 4.0 * rows * static_cast<double>(cols), st);
+  cudaError_t e = launch_layernorm(x, g, b, y, rows, cols, eps, st);
+  if (e != cudaSuccess) return cuda_fail(e, "layernorm launch");
+  return VT_OK;
+}
+
+vt_status run_attention(const AttnParams& p, cudaStream_t st) {
+  const double flops = 4.0 * p.B * p.H * static_cast<double>(p.N) * p.N * p.D;
+  ProfScope ps(CLS_ATTN, flops, 8.0 * p.B * p.H * static_cast<double>(p.N) * p.D, st);
+  cudaError_t e = launch_attention(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return VT_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ handle
+
+struct vt_handle {
+  vt_config cfg;
+  bool loaded = false;
+  struct Layer {
+    const void *ln1_w, *ln1_b, *qkv_w, *qkv_b, *o_w, *o_b, *ln2_w, *ln2_b, *fc1_w, *fc1_b, *fc2_w, *fc2_b;
+  };
+  const void *pe_w = nullptr, *pe_b = nullptr;
+  std::vector<Layer> layers;
+  const void *pa1_w, *pa1_b, *pa2_w, *pa2_b, *pb1_w, *pb1_b, *pb2_w, *pb2_b;
+  void* qkv_pack = nullptr;  // owned: fused [3d, d] weights + [3d] biases per layer
+  float2* rope_tab = nullptr;  // owned: [3][kRopeMaxPos][kRopePairs]
+};
+
+namespace {
+
+bool qkv_layout_supported(const vt_config& c) {
+  if (c.head_dim == 80 && c.rope_sections[0] == 16 && c.rope_sections[1] == 32 && c.rope_sections[2] == 32) return true;
+  if (c.head_dim == 32 && c.rope_sections[0] == 8 && c.rope_sections[1] == 12 && c.rope_sections[2] == 12) return true;
+  return false;
+}
+
+struct Plan {
+  int N, M, Mm, ld_vt;
+  size_t x, xn, q, k, vt, o, hmid, unfold, y1, y2, z1, total;
+};
+
+Plan make_plan(const vt_config& c, int B, int t, int h, int w) {
+  Plan p;
+  p.N = t * h * w;
+  p.M = B * p.N;
+  p.Mm = p.M / 4;
+  p.ld_vt = round8(p.N);
+  const size_t d = c.hidden, M = p.M;
+  const size_t K0 = 3ull * c.temporal_patch * c.patch * c.patch;
+  size_t off = 0;
+  p.x = off;
+  off += align256(M * d * 2);
+  const size_t base = off;
+  // tower phase
+  size_t o2 = base;
+  p.xn = o2;
+  o2 += align256(M * d * 2);
+  p.q = o2;
+  o2 += align256(M * d * 2);
+  p.k = o2;
+  o2 += align256(M * d * 2);
+  p.vt = o2;
+  o2 += align256(static_cast<size_t>(B) * c.heads * c.head_dim * p.ld_vt * 2);
+  p.o = o2;
+  o2 += align256(M * d * 2);
+  p.hmid = o2;
+  o2 += align256(M * std::max<size_t>(c.mlp, K0) * 2);
+  p.unfold = p.hmid;  // only live before the first layer
+  // projector phase (reuses the tower-phase space)
+  size_t o3 = base;
+  p.y1 = o3;
+  o3 += align256(M * static_cast<size_t>(c.proj_hidden) * 2);
+  p.y2 = o3;
+  o3 += align256(M * static_cast<size_t>(c.proj_hidden) * 2);
+  p.z1 = o3;
+  o3 += align256(static_cast<size_t>(p.Mm) * c.proj_hidden * 2);
+  p.total = std::max(o2, o3);
+  return p;
+}
+
+vt_status check_grid(const vt_handle* h, int B, const int32_t* g, int* t, int* gh, int* gw) {
+  if (!g) return fail(VT_ERR_INVALID_ARG, "grid_thw is NULL");
+  if (B <= 0) return fail(VT_ERR_INVALID_ARG, "batch must be positive (got %d)", B);
+  *t = g[0];
+  *gh = g[1];
+  *gw = g[2];
+  if (*t <= 0 || *gh <= 0 || *gw <= 0) return fail(VT_ERR_INVALID_ARG, "grid_thw must be positive");
+  if (*t != 1) return fail(VT_ERR_SHAPE, "only t = 1 (still images) is supported, got t = %d", *t);
+  if ((*gh % h->cfg.merge) || (*gw % h->cfg.merge))
+    return fail(VT_ERR_SHAPE, "grid %dx%d is not a multiple of the %dx%d merge", *gh, *gw, h->cfg.merge, h->cfg.merge);
+  if (*gh > kRopeMaxPos || *gw > kRopeMaxPos)
+    return fail(VT_ERR_SHAPE, "grid side above %d patches", kRopeMaxPos);
+  const long long M = static_cast<long long>(B) * (*t) * (*gh) * (*gw);
+  if (M > (1ll << 30)) return fail(VT_ERR_SHAPE, "too many tokens in one call (%lld)", M);
+  return VT_OK;
+}
+
+// One pre-LN layer over M tokens stored at x (in place).
+vt_status run_layer(vt_handle* h, int i, const void* x_in, void* x, int B, int gt, int gh, int gw, int order,
+                    char* ws, const Plan& pl, cudaStream_t st) {
+  const vt_config& c = h->cfg;
+  const vt_handle::Layer& L = h->layers[i];
+  const int d = c.hidden, M = pl.M;
+  void* xn = ws + pl.xn;
+  vt_status s = run_layernorm(x_in, L.ln1_w, L.ln1_b, xn, M, d, c.ln_eps, st);
+  if (s) return s;
+  {
+    GemmParams p = gemm_params(xn, d, L.qkv_w, d, L.qkv_b, nullptr, 0, nullptr, 0, M, 3 * d, d, ACT_NONE);
+    p.q = ws + pl.q;
+    p.k = ws + pl.k;
+    p.vt = ws + pl.vt;
+    p.heads = c.heads;
+    p.head_dim = c.head_dim;
+    p.ntok = pl.N;
+    p.ld_vt = pl.ld_vt;
+    p.gt = gt;
+    p.gh = gh;
+    p.gw = gw;
+    p.order = order;
+    p.rope = c.use_rope;
+    p.sections[0] = c.rope_sections[0];
+    p.sections[1] = c.rope_sections[1];
+    p.sections[2] = c.rope_sections[2];
+    p.rope_tab = h->rope_tab;
+    ProfScope ps(CLS_GEMM, 2.0 * M * 3.0 * d * d, 0, st);
+    cudaError_t e = launch_gemm(p, st, 1);
+    if (e != cudaSuccess) return cuda_fail(e, "qkv gemm launch");
+  }
+  {
+    AttnParams a;
+    a.q = ws + pl.q;
+    a.k = ws + pl.k;
+    a.vt = ws + pl.vt;
+    a.o = ws + pl.o;
+    a.B = B;
+    a.H = c.heads;
+    a.N = pl.N;
+    a.D = c.head_dim;
+    a.ld_vt = pl.ld_vt;
+    a.scale = 1.0f / std::sqrt(static_cast<float>(c.head_dim));
+    if ((s = run_attention(a, st))) return s;
+  }
+  if ((s = run_gemm(gemm_params(ws + pl.o, d, L.o_w, d, L.o_b, x_in, d, x, d, M, d, d, ACT_NONE), st))) return s;
+  if ((s = run_layernorm(x, L.ln2_w, L.ln2_b, xn, M, d, c.ln_eps, st))) return s;
+  const int act = c.gelu_tanh ? ACT_GELU_TANH : ACT_GELU_ERF;
+  if ((s = run_gemm(gemm_params(xn, d, L.fc1_w, d, L.fc1_b, nullptr, 0, ws + pl.hmid, c.mlp, M, c.mlp, d, act), st)))
+    return s;
+  return run_gemm(gemm_params(ws + pl.hmid, c.mlp, L.fc2_w, c.mlp, L.fc2_b, x, d, x, d, M, d, c.mlp, ACT_NONE), st);
+}
+
+// Projector on block-ordered tokens x [M, d] -> out [M/4, proj_out].
+vt_status run_projector(vt_handle* h, const void* x, void* out, char* ws, const Plan& pl, cudaStream_t st) {
+  const vt_config& c = h->cfg;
+  const int d = c.hidden, P = c.proj_hidden, M = pl.M, Mm = pl.Mm;
+  const int act = c.proj_gelu_tanh ? ACT_GELU_TANH : ACT_GELU_ERF;
+  vt_status s;
+  if ((s = run_gemm(gemm_params(x, d, h->pa1_w, d, h->pa1_b, nullptr, 0, ws + pl.y1, P, M, P, d, act), st))) return s;
+  if ((s = run_gemm(gemm_params(ws + pl.y1, P, h->pa2_w, P, h->pa2_b, nullptr, 0, ws + pl.y2, P, M, P, P, ACT_NONE),
+                    st)))
+    return s;
+  // Four consecutive block-ordered rows of y2 are one merged token: a [M/4, 4P] view.
+  if ((s = run_gemm(gemm_params(ws + pl.y2, 4 * P, h->pb1_w, 4 * P, h->pb1_b, nullptr, 0, ws + pl.z1, P, Mm, P, 4 * P,
+                                act),
+                    st)))
+    return s;
+  return run_gemm(
+      gemm_params(ws + pl.z1, P, h->pb2_w, P, h->pb2_b, nullptr, 0, out, c.proj_out, Mm, c.proj_out, P, ACT_NONE), st);
+}
+
+vt_status check_loaded(const vt_handle* h) {
+  if (!h) return fail(VT_ERR_INVALID_ARG, "handle is NULL");
+  if (!h->loaded) return fail(VT_ERR_NOT_LOADED, "weights are not loaded");
+  return VT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vt_last_error(void) { return g_last_error.c_str(); }
+
+vt_status vt_create(const vt_config* cfg, vt_handle** out) {
+  if (!cfg || !out) return fail(VT_ERR_INVALID_ARG, "cfg and out must not be NULL");
+  const vt_config& c = *cfg;
+  if (c.layers < 0 || c.hidden <= 0 || c.heads <= 0 || c.head_dim <= 0 || c.mlp <= 0 || c.patch <= 0 ||
+      c.temporal_patch <= 0 || c.merge <= 0 || c.proj_hidden <= 0 || c.proj_out <= 0)
+    return fail(VT_ERR_INVALID_ARG, "sizes must be positive");
+  if (c.heads * c.head_dim != c.hidden)
+    return fail(VT_ERR_INVALID_ARG, "heads * head_dim (%d * %d) != hidden (%d)", c.heads, c.head_dim, c.hidden);
+  for (int a = 0; a < 3; ++a)
+    if (c.rope_sections[a] < 0 || (c.rope_sections[a] & 1))
+      return fail(VT_ERR_INVALID_ARG, "rope section %d must be even and non-negative", a);
+  if (c.rope_sections[0] + c.rope_sections[1] + c.rope_sections[2] != c.head_dim)
+    return fail(VT_ERR_INVALID_ARG, "rope sections must sum to head_dim");
+  if (c.rope_sections[0] / 2 > kRopePairs || c.rope_sections[1] / 2 > kRopePairs || c.rope_sections[2] / 2 > kRopePairs)
+    return fail(VT_ERR_UNSUPPORTED, "rope section wider than %d channels", 2 * kRopePairs);
+  if (!(c.rope_theta > 0.f) || !(c.ln_eps > 0.f)) return fail(VT_ERR_INVALID_ARG, "rope_theta and ln_eps must be > 0");
+  if (c.merge != 2) return fail(VT_ERR_UNSUPPORTED, "only a 2x2 merge is supported");
+  if (!qkv_layout_supported(c))
+    return fail(VT_ERR_UNSUPPORTED, "head_dim %d with sections %d/%d/%d has no fused QKV kernel", c.head_dim,
+                c.rope_sections[0], c.rope_sections[1], c.rope_sections[2]);
+  if (c.hidden % 8 || c.mlp % 8 || c.proj_hidden % 8 || c.proj_out % 8)
+    return fail(VT_ERR_UNSUPPORTED, "widths must be multiples of 8");
+  vt_handle* h = new vt_handle();
+  h->cfg = c;
+  *out = h;
+  return VT_OK;
+}
+
+vt_status vt_destroy(vt_handle* h) {
+  if (!h) return VT_OK;
+  if (h->qkv_pack || h->rope_tab) cudaDeviceSynchronize();
+  if (h->qkv_pack) cudaFree(h->qkv_pack);
+  if (h->rope_tab) cudaFree(h->rope_tab);
+  delete h;
+  return VT_OK;
+}
+
+vt_status vt_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out) {
+  if (!h || !out) return fail(VT_ERR_INVALID_ARG, "handle and out must not be NULL");
+  int t, gh, gw;
+  vt_status s = check_grid(h, B, grid_thw, &t, &gh, &gw);
+  if (s) return s;
+  *out = make_plan(h->cfg, B, t, gh, gw).total;
+  return VT_OK;
+}
+
+vt_status vt_load_weights(vt_handle* h, const vt_weight* w, int n) {
+  if (!h || (!w && n > 0) || n < 0) return fail(VT_ERR_INVALID_ARG, "bad arguments");
+  const vt_config& c = h->cfg;
+  std::map<std::string, const vt_weight*> byname;
+  for (int i = 0; i < n; ++i) {
+    if (!w[i].name || !w[i].data) return fail(VT_ERR_WEIGHT, "weight %d has a NULL name or data", i);
+    if (!aligned16(w[i].data)) return fail(VT_ERR_WEIGHT, "%s is not 16-byte aligned", w[i].name);
+    if (!byname.emplace(w[i].name, &w[i]).second) return fail(VT_ERR_WEIGHT, "duplicate weight %s", w[i].name);
+  }
+  std::map<std::string, bool> used;
+  auto get = [&](const std::string& name, std::vector<int64_t> shape, const void** dst) -> vt_status {
+    auto it = byname.find(name);
+    if (it == byname.end()) return fail(VT_ERR_WEIGHT, "missing weight %s", name.c_str());
+    const vt_weight& t = *it->second;
+    bool ok = t.ndim == static_cast<int>(shape.size());
+    for (size_t i = 0; ok && i < shape.size(); ++i) ok = t.shape[i] == shape[i];
+    if (!ok) return fail(VT_ERR_WEIGHT, "weight %s has the wrong shape", name.c_str());
+    used[name] = true;
+    *dst = t.data;
+    return VT_OK;
+  };
+  const int64_t d = c.hidden, m = c.mlp, P = c.proj_hidden, Po = c.proj_out;
+  vt_status s;
+  if ((s = get("embeddings.proj.weight", {d, 3, c.temporal_patch, c.patch, c.patch}, &h->pe_w))) return s;
+  if ((s = get("embeddings.proj.bias", {d}, &h->pe_b))) return s;
+  std::vector<vt_handle::Layer> layers(c.layers);
+  std::vector<int> needs_pack;
+  for (int i = 0; i < c.layers; ++i) {
+    const std::string p = "layers." + std::to_string(i) + ".";
+    vt_handle::Layer& L = layers[i];
+    if ((s = get(p + "ln1.weight", {d}, &L.ln1_w)) || (s = get(p + "ln1.bias", {d}, &L.ln1_b)) ||
+        (s = get(p + "ln2.weight", {d}, &L.ln2_w)) || (s = get(p + "ln2.bias", {d}, &L.ln2_b)) ||
+        (s = get(p + "attn.o.weight", {d, d}, &L.o_w)) || (s = get(p + "attn.o.bias", {d}, &L.o_b)) ||
+        (s = get(p + "mlp.fc1.weight", {m, d}, &L.fc1_w)) || (s = get(p + "mlp.fc1.bias", {m}, &L.fc1_b)) ||
+        (s = get(p + "mlp.fc2.weight", {d, m}, &L.fc2_w)) || (s = get(p + "mlp.fc2.bias", {d}, &L.fc2_b)))
+      return s;
+    if (byname.count(p + "attn.qkv.weight")) {
+      if ((s = get(p + "attn.qkv.weight", {3 * d, d}, &L.qkv_w)) || (s = get(p + "attn.qkv.bias", {3 * d}, &L.qkv_b)))
+        return s;
+    } else {
+      needs_pack.push_back(i);
+    }
+  }
+  if ((s = get("proj.patch_fc1.weight", {P, d}, &h->pa1_w)) || (s = get("proj.patch_fc1.bias", {P}, &h->pa1_b)) ||
+      (s = get("proj.patch_fc2.weight", {P, P}, &h->pa2_w)) || (s = get("proj.patch_fc2.bias", {P}, &h->pa2_b)) ||
+      (s = get("proj.merge_fc1.weight", {P, 4 * P}, &h->pb1_w)) || (s = get("proj.merge_fc1.bias", {P}, &h->pb1_b)) ||
+      (s = get("proj.merge_fc2.weight", {Po, P}, &h->pb2_w)) || (s = get("proj.merge_fc2.bias", {Po}, &h->pb2_b)))
+    return s;
+  // Separate q, k, v: gather the pointers now, pack after every name is checked.
+  std::vector<const void*> sep(needs_pack.size() * 6);
+  for (size_t j = 0; j < needs_pack.size(); ++j) {
+    const std::string p = "layers." + std::to_string(needs_pack[j]) + ".attn.";
+    const char* parts[3] = {"q", "k", "v"};
+    for (int a = 0; a < 3; ++a) {
+      if ((s = get(p + parts[a] + ".weight", {d, d}, &sep[j * 6 + a])) ||
+          (s = get(p + parts[a] + ".bias", {d}, &sep[j * 6 + 3 + a])))
+        return s;
+    }
+  }
+  for (auto& kv : byname)
+    if (!used.count(kv.first)) return fail(VT_ERR_WEIGHT, "unknown weight %s", kv.first.c_str());
+
+  // Device-side state: fused qkv packs and RoPE tables.
+  if (h->qkv_pack) {
+    cudaFree(h->qkv_pack);
+    h->qkv_pack = nullptr;
+  }
+  if (!needs_pack.empty()) {
+    const size_t per = align256(3 * d * d * 2) + align256(3 * d * 2);
+    cudaError_t e = cudaMalloc(&h->qkv_pack, per * needs_pack.size());
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(qkv pack)");
+    for (size_t j = 0; j < needs_pack.size(); ++j) {
+      char* base = static_cast<char*>(h->qkv_pack) + j * per;
+      char* bias = base + align256(3 * d * d * 2);
+      for (int a = 0; a < 3; ++a) {
+        if ((e = cudaMemcpy(base + a * d * d * 2, sep[j * 6 + a], d * d * 2, cudaMemcpyDeviceToDevice)) ||
+            (e = cudaMemcpy(bias + a * d * 2, sep[j * 6 + 3 + a], d * 2, cudaMemcpyDeviceToDevice)))
+          return cuda_fail(e, "packing q/k/v");
+      }
+      layers[needs_pack[j]].qkv_w = base;
+      layers[needs_pack[j]].qkv_b = bias;
+    }
+  }
+  if (!h->rope_tab) {
+    std::vector<float2> tab(static_cast<size_t>(3) * kRopeMaxPos * kRopePairs, make_float2(1.f, 0.f));
+    for (int a = 0; a < 3; ++a) {
+      const int sec = c.rope_sections[a];
+      for (int pos = 0; pos < kRopeMaxPos; ++pos)
+        for (int j = 0; j < sec / 2; ++j) {
+          const double ang = pos * std::pow(static_cast<double>(c.rope_theta), -2.0 * j / sec);
+          tab[(static_cast<size_t>(a) * kRopeMaxPos + pos) * kRopePairs + j] =
+              make_float2(static_cast<float>(std::cos(ang)), static_cast<float>(std::sin(ang)));
+        }
+    }
+    cudaError_t e = cudaMalloc(&h->rope_tab, tab.size() * sizeof(float2));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(rope tables)");
+    if ((e = cudaMemcpy(h->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice)))
+      return cuda_fail(e, "uploading rope tables");
+  }
+  h->layers = layers;
+  h->loaded = true;
+  return VT_OK;
+}
+
+vt_status vt_forward(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* out, void* tower_out,
+                     void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!pixels || !out || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, out and ws must not be NULL");
+  if (!aligned16(pixels) || !aligned16(out) || !aligned16(ws) || (tower_out && !aligned16(tower_out)))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  const vt_config& c = h->cfg;
+  const Plan pl = make_plan(c, B, t, gh, gw);
+  if (ws_bytes < pl.total)
+    return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, pl.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  void* x = w + pl.x;
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  {
+    ProfScope ps(CLS_UNFOLD, 0, pl.M * (4.0 * 3 * c.patch * c.patch + 2.0 * K0), st);
+    cudaError_t e = launch_patch_unfold(pixels, w + pl.unfold, B, gh * c.patch, gw * c.patch, c.patch,
+                                        c.temporal_patch, ORDER_BLOCK, st);
+    if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
+  }
+  if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0,
+                                ACT_NONE),
+                    st)))
+    return s;
+  for (int i = 0; i < c.layers; ++i)
+    if ((s = run_layer(h, i, x, x, B, t, gh, gw, ORDER_BLOCK, w, pl, st))) return s;
+  if (tower_out) {
+    ProfScope ps(CLS_REORDER, 0, 4.0 * pl.M * c.hidden, st);
+    cudaError_t e = launch_reorder_rows(x, tower_out, B, t, gh, gw, c.hidden, 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+  }
+  return run_projector(h, x, out, w, pl, st);
+}
+
+vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out) {
+  size_t base;
+  vt_status s = vt_workspace_bytes(h, B, grid_thw, &base);
+  if (s) return s;
+  const vt_config& c = h->cfg;
+  const size_t N = static_cast<size_t>(grid_thw[0]) * grid_thw[1] * grid_thw[2];
+  const size_t px = static_cast<size_t>(B) * 3 * N * c.patch * c.patch * 4;
+  const size_t o = static_cast<size_t>(B) * (N / 4) * c.proj_out * 2;
+  *out = align256(base) + align256(px) + align256(o);
+  return VT_OK;
+}
+
+vt_status vt_forward_host(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B, void* out_host,
+                          void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!pixels_host || !out_host || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, out and ws must not be NULL");
+  size_t need, base;
+  if ((s = vt_forward_host_workspace_bytes(h, B, grid_thw, &need))) return s;
+  if (ws_bytes < need) return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+  vt_workspace_bytes(h, B, grid_thw, &base);
+  const vt_config& c = h->cfg;
+  const size_t N = static_cast<size_t>(grid_thw[0]) * grid_thw[1] * grid_thw[2];
+  const size_t px = static_cast<size_t>(B) * 3 * N * c.patch * c.patch * 4;
+  const size_t o = static_cast<size_t>(B) * (N / 4) * c.proj_out * 2;
+  char* w = static_cast<char*>(ws);
+  float* dpx = reinterpret_cast<float*>(w + align256(base));
+  char* dout = w + align256(base) + align256(px);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(dpx, pixels_host, px, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copying pixels to the device");
+  if ((s = vt_forward(h, dpx, grid_thw, B, dout, nullptr, ws, base, stream))) return s;
+  if ((e = cudaMemcpyAsync(out_host, dout, o, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return cuda_fail(e, "copying the output to the host");
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream synchronisation");
+  return VT_OK;
+}
+
+vt_status vt_tower_layer(vt_handle* h, int layer, const void* x_in, void* x_out, const int32_t* grid_thw, int B,
+                         void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (layer < 0 || layer >= h->cfg.layers) return fail(VT_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (!x_in || !x_out || !ws) return fail(VT_ERR_INVALID_ARG, "x_in, x_out and ws must not be NULL");
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  const Plan pl = make_plan(h->cfg, B, t, gh, gw);
+  if (ws_bytes < pl.total) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, pl.total);
+  return run_layer(h, layer, x_in, x_out, B, t, gh, gw, ORDER_RASTER, static_cast<char*>(ws), pl,
+                   static_cast<cudaStream_t>(stream));
+}
+
+vt_status vt_patch_embed(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* x_out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!pixels || !x_out || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, x_out and ws must not be NULL");
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  const vt_config& c = h->cfg;
+  const Plan pl = make_plan(c, B, t, gh, gw);
+  if (ws_bytes < pl.total) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, pl.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  cudaError_t e = launch_patch_unfold(pixels, w + pl.unfold, B, gh * c.patch, gw * c.patch, c.patch, c.temporal_patch,
+                                      ORDER_RASTER, st);
+  if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
+  return run_gemm(
+      gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x_out, c.hidden, pl.M, c.hidden, K0, ACT_NONE),
+      st);
+}
+
+vt_status vt_merge_project(vt_handle* h, const void* tower, const int32_t* grid_thw, int B, void* out, void* ws,
+                           size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!tower || !out || !ws) return fail(VT_ERR_INVALID_ARG, "tower, out and ws must not be NULL");
+  if (!aligned16(tower) || !aligned16(out) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  const Plan pl = make_plan(h->cfg, B, t, gh, gw);
+  if (ws_bytes < pl.total) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, pl.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  {
+    ProfScope ps(CLS_REORDER, 0, 4.0 * pl.M * h->cfg.hidden, st);
+    cudaError_t e = launch_reorder_rows(tower, w + pl.x, B, t, gh, gw, h->cfg.hidden, 1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+  }
+  return run_projector(h, w + pl.x, out, w, pl, st);
+}
+
+vt_status vt_attention_workspace_bytes(int B, int H, int N, int D, size_t* out) {
+  if (!out || B <= 0 || H <= 0 || N <= 0 || D <= 0) return fail(VT_ERR_INVALID_ARG, "bad arguments");
+  const size_t ldv = static_cast<size_t>(round8(N));
+  *out = 3 * align256(static_cast<size_t>(B) * H * D * ldv * 2);
+  return VT_OK;
+}
+
+static vt_status check_attn_dims(int B, int H, int N, int D, float scale) {
+  if (B <= 0 || H <= 0 || N <= 0) return fail(VT_ERR_INVALID_ARG, "B, H, N must be positive");
+  if (!(scale > 0.f)) return fail(VT_ERR_INVALID_ARG, "scale must be positive");
+  if (D != 32 && D != 64 && D != 80 && D != 96) return fail(VT_ERR_UNSUPPORTED, "head_dim %d has no kernel", D);
+  if (static_cast<long long>(B) * H * N > (1ll << 31) - 256) return fail(VT_ERR_SHAPE, "too many rows");
+  return VT_OK;
+}
+
+vt_status vt_attention_prepared(const void* q, const void* k, const void* vt_, int ld_vt, void* o, int B, int H, int N,
+                                int D, float scale, void* stream) {
+  vt_status s = check_attn_dims(B, H, N, D, scale);
+  if (s) return s;
+  if (!q || !k || !vt_ || !o) return fail(VT_ERR_INVALID_ARG, "NULL operand");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt_) || !aligned16(o))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (ld_vt < N || (ld_vt % 8)) return fail(VT_ERR_INVALID_ARG, "ld_vt must be >= N and a multiple of 8");
+  AttnParams a{q, k, vt_, o, B, H, N, D, ld_vt, scale};
+  return run_attention(a, static_cast<cudaStream_t>(stream));
+}
+
+vt_status vt_attention(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                       const int32_t* pos_thw, const int32_t* sections, float theta, float scale, void* ws,
+                       size_t ws_bytes, void* stream) {
+  vt_status s = check_attn_dims(B, H, N, D, scale);
+  if (s) return s;
+  if (!q || !k || !v || !o || !ws) return fail(VT_ERR_INVALID_ARG, "NULL operand or workspace");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int sec[3] = {0, 0, 0};
+  if (pos_thw) {
+    if (!sections) return fail(VT_ERR_INVALID_ARG, "sections must be given with pos_thw");
+    for (int a = 0; a < 3; ++a) {
+      sec[a] = sections[a];
+      if (sec[a] < 0 || (sec[a] & 1)) return fail(VT_ERR_INVALID_ARG, "rope sections must be even");
+    }
+    if (sec[0] + sec[1] + sec[2] != D) return fail(VT_ERR_INVALID_ARG, "rope sections must sum to head_dim");
+    if (!(theta > 0.f)) return fail(VT_ERR_INVALID_ARG, "theta must be positive");
+  }
+  size_t need;
+  vt_attention_workspace_bytes(B, H, N, D, &need);
+  if (ws_bytes < need) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, need);
+  const int ldv = round8(N);
+  const size_t part = align256(static_cast<size_t>(B) * H * D * ldv * 2);
+  char* w = static_cast<char*>(ws);
+  void* qr = w;
+  void* kr = w + part;
+  void* vt_ = w + 2 * part;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    ProfScope ps(CLS_PREP, 0, 12.0 * B * H * static_cast<double>(N) * D, st);
+    cudaError_t e = launch_attention_prep(q, k, v, qr, kr, vt_, B, H, N, D, ldv, pos_thw, sec, theta, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention preparation launch");
+  }
+  AttnParams a{qr, kr, vt_, o, B, H, N, D, ldv, scale};
+  return run_attention(a, st);
+}
+
+vt_status vt_linear(const void* A, const void* W, const void* bias, const void* resid, void* out, int M, int N, int K,
+                    int act, void* stream) {
+  if (!A || !W || !out) return fail(VT_ERR_INVALID_ARG, "A, W and out must not be NULL");
+  if (M <= 0 || N <= 0 || K <= 0) return fail(VT_ERR_INVALID_ARG, "M, N, K must be positive");
+  if (N % 8 || K % 8) return fail(VT_ERR_INVALID_ARG, "N and K must be multiples of 8");
+  if (act < 0 || act > 2) return fail(VT_ERR_INVALID_ARG, "act must be 0, 1 or 2");
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out) || (bias && !aligned16(bias)) || (resid && !aligned16(resid)))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return run_gemm(gemm_params(A, K, W, K, bias, resid, N, out, N, M, N, K, act), static_cast<cudaStream_t>(stream));
+}
+
+vt_status vt_layernorm(const void* x, const void* gamma, const void* beta, void* y, int rows, int cols, float eps,
+                       void* stream) {
+  if (!x || !gamma || !beta || !y) return fail(VT_ERR_INVALID_ARG, "NULL operand");
+  if (rows <= 0 || cols <= 0 || !(eps > 0.f)) return fail(VT_ERR_INVALID_ARG, "rows, cols, eps must be positive");
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y) || cols % 8)
+    return fail(VT_ERR_INVALID_ARG, "16-byte aligned rows required (cols multiple of 8)");
+  return run_layernorm(x, gamma, beta, y, rows, cols, eps, static_cast<cudaStream_t>(stream));
+}
+
+vt_status vt_patch_unfold(const float* pixels, void* out, int B, int H, int W, int patch, int temporal_patch, int order,
+                          void* stream) {
+  if (!pixels || !out) return fail(VT_ERR_INVALID_ARG, "NULL operand");
+  if (B <= 0 || H <= 0 || W <= 0 || patch <= 0 || temporal_patch <= 0)
+    return fail(VT_ERR_INVALID_ARG, "sizes must be positive");
+  if (H % patch || W % patch) return fail(VT_ERR_SHAPE, "image side not a multiple of the patch");
+  if (order != ORDER_RASTER && order != ORDER_BLOCK) return fail(VT_ERR_INVALID_ARG, "order must be 0 or 1");
+  if (order == ORDER_BLOCK && ((H / patch) % 2 || (W / patch) % 2))
+    return fail(VT_ERR_SHAPE, "block order needs an even grid");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const double rows = static_cast<double>(B) * (H / patch) * (W / patch);
+  ProfScope ps(CLS_UNFOLD, 0, rows * (4.0 * 3 * patch * patch + 2.0 * 3 * temporal_patch * patch * patch), st);
+  cudaError_t e = launch_patch_unfold(pixels, out, B, H, W, patch, temporal_patch, order, st);
+  if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
+  return VT_OK;
+}
+
+vt_status vt_index_maps(const int32_t* g, int32_t* token_order, int32_t* pos_thw, int32_t* merge_src) {
+  if (!g) return fail(VT_ERR_INVALID_ARG, "grid_thw is NULL");
+  const int t = g[0], gh = g[1], gw = g[2];
+  if (t <= 0 || gh <= 0 || gw <= 0) return fail(VT_ERR_INVALID_ARG, "grid must be positive");
+  if (gh % 2 || gw % 2) return fail(VT_ERR_SHAPE, "grid must be even for the 2x2 merge");
+  const int N = t * gh * gw;
+  for (int n = 0; n < N; ++n) {
+    int tt, hh, ww;
+    token_position(n, gh, gw, ORDER_BLOCK, &tt, &hh, &ww);
+    const int raster = (tt * gh + hh) * gw + ww;
+    if (token_order) token_order[n] = raster;
+    if (merge_src) merge_src[(n / 4) * 4 + (n % 4)] = raster;
+    int rt, rh, rw;
+    token_position(n, gh, gw, ORDER_RASTER, &rt, &rh, &rw);
+    if (pos_thw) {
+      pos_thw[3 * n + 0] = rt;
+      pos_thw[3 * n + 1] = rh;
+      pos_thw[3 * n + 2] = rw;
+    }
+  }
+  return VT_OK;
+}
+
+vt_status vt_check(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending launch error");
+  const unsigned int ge = gemm_read_clear_error(st);
+  const unsigned int ae = attention_read_clear_error(st);
+  if (ge || ae) return fail(VT_ERR_TIMEOUT, "kernel wait limit reached (gemm flags %u, attention flags %u)", ge, ae);
+  return VT_OK;
+}
+
+vt_status vt_profile_begin(void* stream) {
+  (void)stream;
+  std::lock_guard<std::mutex> l(g_prof.mu);
+  for (auto& r : g_prof.recs) {
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.recs.clear();
+  for (int c = 0; c < CLS_COUNT; ++c) {
+    g_prof.ms[c] = g_prof.flops[c] = g_prof.bytes[c] = 0;
+    g_prof.n[c] = 0;
+  }
+  g_prof.on = true;
+  return VT_OK;
+}
+
+vt_status vt_profile_end(void* stream) {
+  (void)stream;
+  std::lock_guard<std::mutex> l(g_prof.mu);
+  g_prof.on = false;
+  return VT_OK;
+}
+
+vt_status vt_profile_read(int cls, double* ms, int64_t* launches, double* flops, double* bytes) {
+  if (cls < 0 || cls >= CLS_COUNT) return fail(VT_ERR_INVALID_ARG, "class out of range");
+  std::lock_guard<std::mutex> l(g_prof.mu);
+  for (auto& r : g_prof.recs) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile event");
+    float t = 0;
+    cudaEventElapsedTime(&t, r.a, r.b);
+    g_prof.ms[r.cls] += t;
+    g_prof.flops[r.cls] += r.flops;
+    g_prof.bytes[r.cls] += r.bytes;
+    g_prof.n[r.cls] += 1;
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.recs.clear();
+  if (ms) *ms = g_prof.ms[cls];
+  if (launches) *launches = g_prof.n[cls];
+  if (flops) *flops = g_prof.flops[cls];
+  if (bytes) *bytes = g_prof.bytes[cls];
+  return VT_OK;
+}
+
+}  // extern "C"
