@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark of the ViT tower + 2x2 merge + projector forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload tower448|tower2016|attn65536|...]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on the host cores
+
+One step = one forward of the whole path (patch unfold, patch embedding, 32 layers,
+merge, projector) over one batch of synthetic input resident in HBM.  The timed region
+is K steps, each bracketed by CUDA events on the launching stream, with an L2 flush
+(a 512 MB write) between steps outside the events; barrier + synchronize on both sides;
+the maximum over ranks is reported.  N > 1 runs independent replicas, one per GPU
+(torchrun), each with its own batch: weak scaling, no collective in the data path.
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vision_transformer_encoder_vit_b200 import synthetic as S  # noqa: E402
+
+METRIC = "ViT tower images/s & tokens/s at 448²/2016²; attention+GEMM TFLOP/s vs BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload(name: str) -> dict:
+    """Shape of the benchmarked step."""
+    if name in ("tower448", "tower2016"):
+        cfg = S.get_config(name)
+        t, gh, gw = S.token_grid(cfg)
+        N = t * gh * gw
+        return dict(kind="tower", name=name, cfg=cfg, batch=cfg["batch"], grid=(t, gh, gw), tokens=N,
+                    desc=f"full tower (32 layers) + 2x2 merge + projector, {cfg['batch']} image(s) of "
+                         f"{cfg['image'][0]}x{cfg['image'][1]}")
+    if name.startswith("attn"):
+        n = int(name[4:])
+        side = int(round(n ** 0.5))
+        return dict(kind="attn", name=name, batch=1, grid=(1, side, side), tokens=side * side, heads=16, D=80,
+                    desc=f"attention only, 16 heads x 80, {side}x{side} tokens, 3D RoPE")
+    raise SystemExit(f"unknown workload {name}")
+
+
+def tower_flops(cfg: dict, N: int) -> dict:
+    """Algorithmic FLOPs of one image: 2MNK per GEMM, 4 N^2 d for attention."""
+    d, m, P, Po = cfg["hidden"], cfg["mlp"], cfg["proj_hidden"], cfg["proj_out"]
+    K0 = 3 * cfg["temporal_patch"] * cfg["patch"] ** 2
+    L = cfg["layers"]
+    gemm = 2 * N * K0 * d + L * 2 * N * d * (3 * d + d + 2 * m) + 2 * N * (d * P + P * P) + \
+        2 * (N // 4) * (4 * P * P + P * Po)
+    attn = L * 4 * N * N * d
+    return dict(gemm=gemm, attn=attn, total=gemm + attn)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (start before, stop after)."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), max=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "samples": len(loaded), "reasons": sorted(reasons)}
+
+
+# -------------------------------------------------------------- CPU oracle
+
+def oracle_images_per_s(cfg: dict, budget_s: float = 15.0) -> dict:
+    """Times the fp64 oracle on one image: patch embedding, as many layers as fit in the
+    budget (at least one), and the projector; extrapolates to all layers."""
+    from oracle import vit_ref as R
+    w = S.weights_f64(S.make_weights(cfg, layers=min(cfg["layers"], 4)))
+    px = S.make_pixels(cfg, batch=1)[0].astype(np.float64)
+    t, gh, gw = S.token_grid(cfg)
+    pos = R.positions_raster(t, gh, gw)
+    t0 = time.perf_counter()
+    x = R.patch_embed(R.patch_unfold(px, cfg["patch"], cfg["temporal_patch"]), w["embeddings.proj.weight"],
+                      w["embeddings.proj.bias"])
+    t_embed = time.perf_counter() - t0
+    layer_times = []
+    start = time.perf_counter()
+    i = 0
+    while i < 4 and (i == 0 or time.perf_counter() - start < budget_s * 0.7):
+        t0 = time.perf_counter()
+        x = R.tower_layer(x, w, i, cfg, pos)
+        layer_times.append(time.perf_counter() - t0)
+        i += 1
+    t0 = time.perf_counter()
+    R.projector(x, w, cfg, t, gh, gw)
+    t_proj = time.perf_counter() - t0
+    per_image = t_embed + cfg["layers"] * statistics.mean(layer_times) + t_proj
+    return dict(value=1.0 / per_image, unit="images/s", cores=os.cpu_count(), kind="oracle",
+                sample=f"one {cfg['image'][0]}x{cfg['image'][1]} image: patch embedding, {len(layer_times)} of "
+                       f"{cfg['layers']} layers (mean layer time x {cfg['layers']}), projector; numpy float64",
+                seconds=per_image)
+
+
+def oracle_attention(wl: dict, budget_s: float = 15.0) -> dict:
+    from oracle import vit_ref as R
+    H, D, N = wl["heads"], wl["D"], wl["tokens"]
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((H, N, D)) for _ in range(3))
+    rows = np.arange(min(N, 256))
+    t0 = time.perf_counter()
+    n_heads = 0
+    while n_heads < H and (n_heads == 0 or time.perf_counter() - t0 < budget_s):
+        R.attention(q[n_heads:n_heads + 1], k[n_heads:n_heads + 1], v[n_heads:n_heads + 1], D ** -0.5, rows=rows)
+        n_heads += 1
+    dt = time.perf_counter() - t0
+    per_call = dt / (n_heads * len(rows)) * N * H
+    return dict(value=1.0 / per_call, unit="calls/s", cores=os.cpu_count(), kind="oracle",
+                sample=f"{len(rows)} query rows x {n_heads} heads of the {N}-token attention, scaled to all rows "
+                       f"and {H} heads", seconds=per_call)
+
+
+# --------------------------------------------------------------- reference
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = []
+    for _ in range(args.steps):
+        if wl["kind"] == "tower":
+            r = oracle_images_per_s(wl["cfg"], budget_s=args.ref_budget / max(args.steps, 1))
+        else:
+            r = oracle_attention(wl, budget_s=args.ref_budget / max(args.steps, 1))
+        steps.append(r)
+    value = statistics.mean(s["value"] for s in steps)
+    unit = steps[0]["unit"]
+    line = dict(metric=METRIC, value=value, unit=unit, n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1000.0 * statistics.mean(s["seconds"] for s in steps) *
+                (wl["batch"] if wl["kind"] == "tower" else 1),
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                impl="reference",
+                config=dict(workload=wl["name"], description=wl["desc"], global_batch=wl["batch"],
+                            tokens_per_image=wl["tokens"]),
+                cpu_baseline=dict(value=value, unit=unit, cores=steps[0]["cores"], kind="oracle",
+                                  sample=steps[0]["sample"]),
+                e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    from vision_transformer_encoder_vit_b200 import vt as V
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks, peaks_kind = load_peaks()
+    B = wl["batch"]
+    grid = wl["grid"]
+    N = wl["tokens"]
+
+    if wl["kind"] == "tower":
+        cfg = wl["cfg"]
+        tower = V.Tower(cfg, S.make_weights(cfg))
+        px_host = torch.from_numpy(S.make_pixels(cfg, batch=B, seed=cfg["seed"] + rank)).pin_memory()
+        px = px_host.to(dev)
+        ws = tower.workspace(B, grid)
+        out = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16, device=dev)
+
+        def step():
+            V.vt_forward(tower.h, px, grid, B, out, None, ws, ws.numel(), stream)
+
+        flops = tower_flops(cfg, N)
+        step_flops = B * flops["total"]
+        units_per_step = B
+        unit = "images/s"
+    else:
+        H, D = wl["heads"], wl["D"]
+        q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+                   for a in S.make_qkv(1, H, N, D, 3))
+        pos = torch.from_numpy(
+            np.stack(np.meshgrid(np.zeros(1), np.arange(grid[1]), np.arange(grid[2]), indexing="ij"), -1)
+            .reshape(-1, 3).astype(np.int32)).to(dev)
+        o = torch.empty((1, N, H * D), dtype=torch.bfloat16, device=dev)
+        ws_bytes = V.vt_attention_workspace_bytes(1, H, N, D)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def step():
+            V.vt_attention(q, k, v, o, 1, H, N, D, pos, (16, 32, 32), 10000.0, D ** -0.5, ws, ws_bytes, stream)
+
+        step_flops = 4.0 * H * N * N * D
+        units_per_step = 1
+        unit = "calls/s"
+
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    # warm-up (also compiles nothing: the library is prebuilt; first calls set kernel attributes)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    V.vt_check(stream)
+
+    # optional CUDA graph of one step
+    graph = None
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            s2 = torch.cuda.Stream()
+            s2.wait_stream(stream)
+            with torch.cuda.stream(s2):
+                with torch.cuda.graph(g, stream=s2):
+                    if wl["kind"] == "tower":
+                        V.vt_forward(tower.h, px, grid, B, out, None, ws, ws.numel(), s2)
+                    else:
+                        V.vt_attention(q, k, v, o, 1, H, N, D, pos, (16, 32, 32), 10000.0, D ** -0.5, ws,
+                                       ws_bytes, s2)
+            stream.wait_stream(s2)
+            g.replay()
+            torch.cuda.synchronize()
+            graph = g
+        except Exception as e:  # capture is an optimisation; eager launches are the same kernels
+            print(f"# graph capture failed, timing eager launches: {e}", file=sys.stderr)
+            graph = None
+
+    def timed_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
+    # ---------------- timed region
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        timed_step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    V.vt_check(stream)
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * units_per_step * args.steps / (ms / 1000.0)
+
+    # ---------------- per-kernel-class times of one profiled step (events around each launch)
+    V.vt_profile_begin(stream)
+    for _ in range(args.profile_steps):
+        flush.fill_(1)
+        step()
+    V.vt_profile_end(stream)
+    prof = V.vt_profile_read()
+    launches_per_step = sum(v["launches"] for v in prof.values()) / args.profile_steps
+
+    # ---------------- end to end through the C ABI with host buffers
+    e2e = None
+    if wl["kind"] == "tower":
+        ws_h = torch.empty(V.vt_forward_host_workspace_bytes(tower.h, B, grid), dtype=torch.uint8, device=dev)
+        out_h = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory()
+        V.vt_forward_host(tower.h, px_host, grid, B, out_h, ws_h, ws_h.numel(), stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        e_s.record(stream)
+        for _ in range(args.steps):
+            V.vt_forward_host(tower.h, px_host, grid, B, out_h, ws_h, ws_h.numel(), stream)
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e_s.elapsed_time(e_e)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = dict(value=world * B * args.steps / (e2e_ms / 1000.0), unit=unit,
+                   h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h.numel() * 2),
+                   api="vt_forward_host")
+        del ws_h
+
+    if rank == 0:
+        # dominant kernel class by device time
+        dom = max(("gemm", "attention"), key=lambda c: prof[c]["ms"])
+        p = prof[dom]
+        achieved = p["flops"] / (p["ms"] / 1000.0) / 1e12 if p["ms"] > 0 else 0.0
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = dict(bound="tensor", kernel=("gemm_bf16_tcgen05 (all linear layers)" if dom == "gemm"
+                                                 else "attn_fwd_tcgen05"),
+                        achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
+                        peak_source=f"{peaks_kind} bf16 sustained", traffic=None,
+                        per_launch_flops=p["flops"] / max(p["launches"], 1),
+                        avg_launch_us=1000.0 * p["ms"] / max(p["launches"], 1))
+        classes = {k: dict(ms_per_step=v["ms"] / args.profile_steps,
+                           launches_per_step=v["launches"] / args.profile_steps,
+                           tflops=(v["flops"] / (v["ms"] / 1000.0) / 1e12) if v["ms"] > 0 and v["flops"] else None,
+                           gbs=(v["bytes"] / (v["ms"] / 1000.0) / 1e9) if v["ms"] > 0 and v["bytes"] and
+                           not v["flops"] else None)
+                   for k, v in prof.items() if v["launches"]}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = (oracle_images_per_s(wl["cfg"], args.cpu_budget) if wl["kind"] == "tower"
+                   else oracle_attention(wl, args.cpu_budget))
+            cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        line = dict(
+            metric=METRIC, value=value, unit=unit, n_gpus=world, steps=args.steps, warmup=max(args.warmup, 3),
+            ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+            data="synthetic: seeded N(0,0.02) bf16 weights, U[0,1] ImageNet-normalised pixels",
+            config=dict(workload=wl["name"], description=wl["desc"], per_gpu_batch=B, global_batch=B * world,
+                        tokens_per_image=N, merged_tokens_per_image=N // 4,
+                        l2="flushed (512 MB write) between timed steps", launch="cuda graph" if graph else "eager",
+                        parallelism=f"replicas x{world}"),
+            tokens_per_s=value * N if wl["kind"] == "tower" else None,
+            output_tokens_per_s=value * N // 4 if wl["kind"] == "tower" else None,
+            tflops=world * step_flops * args.steps / (ms / 1000.0) / 1e12,
+            roofline=roofline, kernel_classes=classes,
+            cpu_baseline=cpu, e2e=e2e,
+            gpu_launches=int(round(launches_per_step * args.steps)),
+            clocks=clk,
+        )
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="tower448")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    args = ap.parse_args()
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

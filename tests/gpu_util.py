@@ -10,6 +10,9 @@ Tolerances (written here once, used by every parity test):
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -51,12 +54,23 @@ def rel_l2(g: np.ndarray, o: np.ndarray) -> float:
     return float(np.linalg.norm((g - o).ravel()) / max(np.linalg.norm(o.ravel()), 1e-300))
 
 
+def report(what: str, **fields) -> None:
+    """Appends one JSON line to $VT_PARITY_REPORT (if set): the measured errors."""
+    path = os.environ.get("VT_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(what=what, **fields)) + "\n")
+
+
 def assert_close(g, o, rel=REL_L2_LAYER, rtol=ELEM_RTOL, atol=ELEM_ATOL, what=""):
     g = np.asarray(g, np.float64)
     o = np.asarray(o, np.float64)
     assert g.shape == o.shape, f"{what}: shape {g.shape} != {o.shape}"
     assert np.isfinite(g).all(), f"{what}: non-finite values"
     r = rel_l2(g, o)
+    rms_o = float(np.sqrt(np.mean(o ** 2))) if o.size else 0.0
+    worst = float(np.max(np.abs(g - o) / (rtol * np.abs(o) + atol * rms_o + 1e-300))) if o.size else 0.0
+    report(what, rel_l2=r, gate=rel, worst_elem_over_bound=worst)
     assert r <= rel, f"{what}: relative L2 error {r:.3e} > {rel:.1e}"
     rms = float(np.sqrt(np.mean(o ** 2))) if o.size else 0.0
     bound = rtol * np.abs(o) + atol * rms
