@@ -185,6 +185,25 @@ VT_API vt_status vt_attention(const void* q, const void* k, const void* v, void*
 VT_API vt_status vt_attention_prepared(const void* q, const void* k, const void* vt, int ld_vt, void* o, int B, int H,
                                 int N, int D, float scale, void* stream);
 
+/* vt_attention for callers that cannot allocate device memory, and so cannot pass a
+ * workspace: for example code running inside a host framework whose allocator owns
+ * all device memory, or a plugin interface that hands over only its input and output
+ * buffers.  The pages describe no such entry point; it has no counterpart there.
+ * Arguments and results are those of vt_attention without ws / ws_bytes.  Its scratch
+ * (rotated q and k, transposed v) is a 32 MiB array compiled into the library, which
+ * every GPU that loads libvt holds until the process exits; vt_attention_static_max_bytes
+ * reports the size.  A problem needing more than that (3 * B*H*D*ceil8(N) * 2 bytes)
+ * is rejected with VT_ERR_WORKSPACE before anything is launched.  Nothing is
+ * allocated: no cudaMalloc, cudaFree or allocating library call.  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls share
+ * the array and leave their contents in it; calls whose GPU work overlaps race on it
+ * and must be serialised by the caller. */
+VT_API vt_status vt_attention_static(const void* q, const void* k, const void* v, void* o, int B, int H, int N,
+                                     int D, const int32_t* pos_thw, const int32_t* sections, float theta,
+                                     float scale, void* stream);
+VT_API vt_status vt_attention_static_max_bytes(size_t* out);
+
 /* out[M, N] = act(A[M, K] W[N, K]^T + bias) + resid, bf16 in/out, fp32 accumulation on
  * the tensor cores.  bias [N] and resid [M, N] may be NULL; resid may equal out.
  * act: 0 none, 1 GELU tanh form, 2 GELU erf form.  N and K must be multiples of 8.

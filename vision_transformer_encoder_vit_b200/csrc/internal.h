@@ -108,4 +108,7 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 
 int device_sm_count();
 
+// Sets the calling thread's message returned by vt_last_error().
+void set_error_message(const char* msg);
+
 }  // namespace vt

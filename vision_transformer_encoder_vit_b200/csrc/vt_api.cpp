@@ -140,6 +140,8 @@ vt_status run_attention(const AttnParams& p, cudaStream_t st) {
 
 }  // namespace
 
+void vt::set_error_message(const char* msg) { g_last_error = msg ? msg : ""; }
+
 // ------------------------------------------------------------------ handle
 
 struct vt_handle {

@@ -69,6 +69,8 @@ _SIGS = {
     "vt_attention_workspace_bytes": ([_i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "vt_attention": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i32p, _f, _f, _vp, _sz, _vp]),
     "vt_attention_prepared": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _f, _vp]),
+    "vt_attention_static": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i32p, _f, _f, _vp]),
+    "vt_attention_static_max_bytes": ([ctypes.POINTER(_sz)]),
     "vt_linear": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "vt_layernorm": ([_vp, _vp, _vp, _vp, _i, _i, _f, _vp]),
     "vt_patch_unfold": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
@@ -214,6 +216,20 @@ def vt_attention(q, k, v, o, B, H, N, D, pos_thw, sections, theta, scale, ws, ws
     sec = (ctypes.c_int32 * 3)(*sections) if sections is not None else None
     _check(lib.vt_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _ptr(pos_thw), sec, theta, scale,
                             _ptr(ws), ws_bytes, _stream(stream)), "vt_attention")
+
+
+def vt_attention_static(q, k, v, o, B, H, N, D, pos_thw, sections, theta, scale, stream=None) -> None:
+    """vt_attention without a workspace, for callers that cannot allocate device
+    memory: its scratch is a fixed array inside the library (see include/vt.h)."""
+    sec = (ctypes.c_int32 * 3)(*sections) if sections is not None else None
+    _check(lib.vt_attention_static(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _ptr(pos_thw), sec, theta,
+                                   scale, _stream(stream)), "vt_attention_static")
+
+
+def vt_attention_static_max_bytes() -> int:
+    out = _sz()
+    _check(lib.vt_attention_static_max_bytes(ctypes.byref(out)), "vt_attention_static_max_bytes")
+    return out.value
 
 
 def vt_attention_prepared(q, k, vt, ld_vt, o, B, H, N, D, scale, stream=None) -> None:
