@@ -248,6 +248,11 @@ VT_API const char* vt_last_error(void);
 VT_API vt_status vt_profile_begin(void* stream);
 VT_API vt_status vt_profile_end(void* stream);
 VT_API vt_status vt_profile_read(int cls, double* ms, int64_t* launches, double* flops, double* bytes);
+/* The individual launches of the last profiled interval, in launch order:
+ * vt_profile_launches returns their count (synchronising like vt_profile_read);
+ * vt_profile_launch returns launch i's class, milliseconds, FLOPs and bytes. */
+VT_API vt_status vt_profile_launches(int64_t* count);
+VT_API vt_status vt_profile_launch(int64_t i, int* cls, double* ms, double* flops, double* bytes);
 
 #ifdef __cplusplus
 }

@@ -250,14 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float s[S::BN];
       {
-        uint32_t raw[32];
+        uint32_t raw[S::BN];
+        tmem_ld128(tmem + buf * 128 + lane_off, raw);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < S::BN; c += 32) {
-          tmem_ld32(tmem + buf * 128 + c + lane_off, raw);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(raw[i]);
-        }
+        for (int c = 0; c < S::BN; ++c) s[c] = __uint_as_float(raw[c]);
       }
       tc_fence_before();
       mbar_arrive(&s_free[buf]);
@@ -267,9 +264,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < S::BN; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      // Row maximum with 8 independent partial maxima (short dependency chains).
+      float m8[8];
 #pragma unroll
-      for (int c = 1; c < S::BN; ++c) mx = fmaxf(mx, s[c]);
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < S::BN; c += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_new = mx * sl2;
       bool need = false;
       if (j == 0) {
@@ -303,18 +307,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
       uint8_t* pbuf = sP + buf * S::P_BYTES;
       const float neg = -m_ref;
+      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c16 = 0; c16 < S::BN / 8; ++c16) {
         float e[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          e[i] = fast_exp2(fmaf(s[c16 * 8 + i], sl2, neg));
-          l += e[i];
+          // a quarter of the exponentials on the FMA pipe, the rest on MUFU
+          const float x = fmaf(s[c16 * 8 + i], sl2, neg);
+          e[i] = (i >= 6) ? soft_exp2(x) : fast_exp2(x);
+          l8[i] += e[i];
         }
         const int blk = c16 >> 3, cc = c16 & 7;
         uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
         *dst = pack_bf16x8(e);
       }
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[buf]);

@@ -201,8 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
-      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
-      tc_fence_after();
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
@@ -210,17 +208,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bf16* bias = static_cast<const bf16*>(p.bias);
         const bf16* resid = static_cast<const bf16*>(p.resid);
         bf16* out = static_cast<bf16*>(p.out);
+        // Bias and residual of a 32-column chunk are loaded one chunk ahead (the first
+        // chunk before waiting for the accumulator) so that no global-load latency sits
+        // between the TMEM read and the store.
+        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+        auto prefetch = [&](int col, uint4* bq, uint4* rq) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int cg = col + 8 * g;
+            bq[g] = (bias && cg < p.N) ? __ldg(reinterpret_cast<const uint4*>(bias + cg)) : zero;
+            rq[g] = (resid && cg < p.N && row < p.M)
+                        ? *reinterpret_cast<const uint4*>(resid + static_cast<size_t>(row) * p.ldr + cg)
+                        : zero;
+          }
+        };
+        uint4 bq[4], rq[4];
+        prefetch(nb * BN, bq, rq);
+        if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
           const int col = nb * BN + c0;
           if (col >= p.N) break;
+          uint4 bn_[4] = {zero, zero, zero, zero}, rn_[4] = {zero, zero, zero, zero};
+          if (c0 + 32 < BN) prefetch(col + 32, bn_, rn_);
           float v[32];
           load_cols<32>(t_row + c0, v);
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const int cg = col + 8 * g;
             if (cg < p.N) {
-              if (bias) add_bf16x8(v + 8 * g, *reinterpret_cast<const uint4*>(bias + cg));
+              if (bias) add_bf16x8(v + 8 * g, bq[g]);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 float x = v[8 * g + i];
@@ -229,15 +247,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v[8 * g + i] = x;
               }
               if (row < p.M) {
-                if (resid)
-                  add_bf16x8(v + 8 * g,
-                             *reinterpret_cast<const uint4*>(resid + static_cast<size_t>(row) * p.ldr + cg));
+                if (resid) add_bf16x8(v + 8 * g, rq[g]);
                 *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.ldo + cg) = pack_bf16x8(v + 8 * g);
               }
             }
           }
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            bq[g] = bn_[g];
+            rq[g] = rn_[g];
+          }
         }
       } else {
+        if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
+        tc_fence_after();
         constexpr int D = RL::D;
         constexpr int HPT = BN / D;
         const bf16* bias = static_cast<const bf16*>(p.bias);

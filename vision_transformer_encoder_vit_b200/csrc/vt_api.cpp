@@ -50,10 +50,16 @@ struct ProfRec {
   double flops, bytes;
 };
 
+struct DoneRec {
+  int cls;
+  double ms, flops, bytes;
+};
+
 struct Profiler {
   std::mutex mu;
   bool on = false;
   std::vector<ProfRec> recs;
+  std::vector<DoneRec> done;  // resolved launches of the last profiled interval
   std::vector<cudaEvent_t> pool;
   double ms[CLS_COUNT] = {0}, flops[CLS_COUNT] = {0}, bytes[CLS_COUNT] = {0};
   int64_t n[CLS_COUNT] = {0};
@@ -737,6 +743,7 @@ vt_status vt_profile_begin(void* stream) {
     g_prof.pool.push_back(r.b);
   }
   g_prof.recs.clear();
+  g_prof.done.clear();
   for (int c = 0; c < CLS_COUNT; ++c) {
     g_prof.ms[c] = g_prof.flops[c] = g_prof.bytes[c] = 0;
     g_prof.n[c] = 0;
@@ -752,9 +759,9 @@ vt_status vt_profile_end(void* stream) {
   return VT_OK;
 }
 
-vt_status vt_profile_read(int cls, double* ms, int64_t* launches, double* flops, double* bytes) {
-  if (cls < 0 || cls >= CLS_COUNT) return fail(VT_ERR_INVALID_ARG, "class out of range");
-  std::lock_guard<std::mutex> l(g_prof.mu);
+namespace {
+// Resolves the pending event pairs into per-launch records and class totals.
+vt_status resolve_profile() {
   for (auto& r : g_prof.recs) {
     cudaError_t e = cudaEventSynchronize(r.b);
     if (e != cudaSuccess) return cuda_fail(e, "profile event");
@@ -764,14 +771,44 @@ vt_status vt_profile_read(int cls, double* ms, int64_t* launches, double* flops,
     g_prof.flops[r.cls] += r.flops;
     g_prof.bytes[r.cls] += r.bytes;
     g_prof.n[r.cls] += 1;
+    g_prof.done.push_back({r.cls, static_cast<double>(t), r.flops, r.bytes});
     g_prof.pool.push_back(r.a);
     g_prof.pool.push_back(r.b);
   }
   g_prof.recs.clear();
+  return VT_OK;
+}
+}  // namespace
+
+vt_status vt_profile_read(int cls, double* ms, int64_t* launches, double* flops, double* bytes) {
+  if (cls < 0 || cls >= CLS_COUNT) return fail(VT_ERR_INVALID_ARG, "class out of range");
+  std::lock_guard<std::mutex> l(g_prof.mu);
+  vt_status s = resolve_profile();
+  if (s) return s;
   if (ms) *ms = g_prof.ms[cls];
   if (launches) *launches = g_prof.n[cls];
   if (flops) *flops = g_prof.flops[cls];
   if (bytes) *bytes = g_prof.bytes[cls];
+  return VT_OK;
+}
+
+vt_status vt_profile_launches(int64_t* count) {
+  if (!count) return fail(VT_ERR_INVALID_ARG, "count is NULL");
+  std::lock_guard<std::mutex> l(g_prof.mu);
+  vt_status s = resolve_profile();
+  if (s) return s;
+  *count = static_cast<int64_t>(g_prof.done.size());
+  return VT_OK;
+}
+
+vt_status vt_profile_launch(int64_t i, int* cls, double* ms, double* flops, double* bytes) {
+  std::lock_guard<std::mutex> l(g_prof.mu);
+  if (i < 0 || i >= static_cast<int64_t>(g_prof.done.size())) return fail(VT_ERR_INVALID_ARG, "launch index out of range");
+  const DoneRec& d = g_prof.done[static_cast<size_t>(i)];
+  if (cls) *cls = d.cls;
+  if (ms) *ms = d.ms;
+  if (flops) *flops = d.flops;
+  if (bytes) *bytes = d.bytes;
   return VT_OK;
 }
 

@@ -80,6 +80,9 @@ _SIGS = {
     "vt_profile_end": ([_vp]),
     "vt_profile_read": ([_i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                          ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
+    "vt_profile_launches": ([ctypes.POINTER(ctypes.c_int64)]),
+    "vt_profile_launch": ([ctypes.c_int64, ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_double),
+                           ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -284,6 +287,19 @@ def vt_profile_read() -> dict:
         _check(lib.vt_profile_read(cls, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(fl), ctypes.byref(by)),
                "vt_profile_read")
         out[name] = dict(ms=ms.value, launches=n.value, flops=fl.value, bytes=by.value)
+    return out
+
+
+def vt_profile_launches() -> list[dict]:
+    """Every launch of the last profiled interval: class name, ms, flops, bytes."""
+    n = ctypes.c_int64()
+    _check(lib.vt_profile_launches(ctypes.byref(n)), "vt_profile_launches")
+    out = []
+    for i in range(n.value):
+        c, ms, fl, by = _i(), ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+        _check(lib.vt_profile_launch(i, ctypes.byref(c), ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(by)),
+               "vt_profile_launch")
+        out.append(dict(cls=PROFILE_CLASSES[c.value], ms=ms.value, flops=fl.value, bytes=by.value))
     return out
 
 
