@@ -1,6 +1,6 @@
 // Bidirectional (non-causal) multi-head attention for sm_100a, flash style:
-// O_h = softmax(q_h k_h^T * scale) v_h per image and head, computed one 128-row
-// query tile per CTA while 128-key tiles stream through a TMA ring.  No [N, N]
+// O_h = softmax(q_h k_h^T * scale) v_h per image and head, computed for two 128-row
+// query tiles per CTA while 128-key tiles stream through a TMA ring.  No [N, N]
 // buffer exists anywhere; memory traffic is q, k, v in and o out.
 //
 // The operation is the ViT self-attention of the "MiniMax-M3 Vision" model card
@@ -9,14 +9,17 @@
 // comment of CEILING_MAX_PATCHES) builds the full [seq, seq] score matrix per head and
 // notes that larger images need tiled attention; this kernel is that tiled form.
 //
-// CTA = 6 warps.  Warp 0 issues TMA loads (Q once, then K and V^T tiles).  Warp 1
-// allocates TMEM and issues the MMAs from one thread:
-//     S_j = Q K_j^T          -> TMEM columns [128 * (j & 1), +128)   (fp32)
-//     O  += P_j V_j          -> TMEM columns [256, 256 + D)          (fp32)
-// Warps 2..5 (one thread per query row) run the online softmax: load S_j from TMEM,
-// exponentiate with a lazily updated running maximum, write P_j (bf16) into a
-// 128-byte-swizzled shared tile for the next MMA, rescale O in TMEM only when the
-// maximum grows by more than 2^8, and finally write O / l.
+// CTA = 10 warps.  Warp 0 issues TMA loads (both Q tiles once, then K and V^T tiles
+// shared by the two query tiles).  Warp 1 allocates TMEM and issues the MMAs from one
+// thread; for key tile j and query tile t in {0, 1}:
+//     S_t = Q_t K_j^T         -> TMEM columns [256 t, 256 t + 128)        (fp32)
+//     O_t += P_t V_j          -> TMEM columns [256 t + 128, 256 t + 128 + D)
+// Warps 2..5 run the online softmax of query tile 0 and warps 6..9 that of query tile
+// 1 (one thread per query row): load S_t from TMEM, exponentiate against a lazily
+// updated running maximum, write P_t (bf16) into a 128-byte-swizzled shared tile for
+// the next MMA, rescale O_t in TMEM only when the maximum grows by more than 2^8, and
+// finally write O_t / l.  Two softmax warps per SM sub-partition hide each other's
+// latencies, and each K/V tile feeds twice the MMA work of a one-tile CTA.
 //
 // Operand layouts: q, k are [B, H, N, D] (D contiguous), used K-major; v is given
 // transposed, vt [B, H, D, ld_vt], so that V_j^T is K-major too.  A head of 80
@@ -32,7 +35,7 @@ namespace {
 
 __device__ unsigned int g_attn_err;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 
 __host__ __device__ constexpr uint32_t layout_code(int swizzle_bytes) {
   return swizzle_bytes == 128 ? 2u : swizzle_bytes == 64 ? 4u : 6u;
@@ -40,14 +43,14 @@ __host__ __device__ constexpr uint32_t layout_code(int swizzle_bytes) {
 
 template <int D>
 struct AttnShape {
-  static constexpr int BM = 128;  // query rows per CTA
+  static constexpr int BM = 128;  // query rows per tile (two tiles per CTA)
   static constexpr int BN = 128;  // keys per tile
   static constexpr int C0 = D >= 64 ? 64 : D;  // channels of chunk 0
   static constexpr int C1 = D - C0;            // channels of chunk 1 (0 if none)
   static constexpr int SW0 = C0 * 2, SW1 = C1 * 2;  // row bytes = swizzle span
   static constexpr uint32_t LAY0 = layout_code(SW0), LAY1 = layout_code(SW1);
   static constexpr int SBO0 = 8 * SW0, SBO1 = 8 * SW1;
-  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int Q_BYTES = BM * D * 2;  // one query tile
   static constexpr int Q1_OFF = BM * C0 * 2;
   static constexpr int K_BYTES = BN * D * 2;
   static constexpr int K1_OFF = BN * C0 * 2;
@@ -56,14 +59,15 @@ struct AttnShape {
   static constexpr int KV_BYTES = K_BYTES + V_BYTES;
   static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int AVAIL = 227 * 1024 - 1024 - BAR_BYTES - Q_BYTES - 2 * P_BYTES;
+  static constexpr int AVAIL = 232448 - 1024 - BAR_BYTES - 2 * Q_BYTES - 2 * P_BYTES;
   static constexpr int STAGES = AVAIL / KV_BYTES > 4 ? 4 : AVAIL / KV_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_BYTES + 2 * P_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_BYTES + STAGES * KV_BYTES + 2 * P_BYTES + BAR_BYTES;
   static constexpr int TMEM_COLS = 512;
   static_assert(C0 == 16 || C0 == 32 || C0 == 64, "chunk 0 width");
   static_assert(C1 == 0 || C1 == 16 || C1 == 32 || C1 == 64, "chunk 1 width");
   static_assert(D % 16 == 0 && D <= 128, "head_dim");
   static_assert(STAGES >= 2, "shared memory");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(Q1_OFF % 1024 == 0 && K1_OFF % 1024 == 0 && V1_OFF % 1024 == 0 && KV_BYTES % 1024 == 0 &&
                     Q_BYTES % 1024 == 0,
                 "1024-byte alignment of swizzled tiles");
@@ -95,25 +99,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   using S = AttnShape<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + S::Q_BYTES;                  // per stage: K tile then V^T tile
-  uint8_t* sP = sKV + S::STAGES * S::KV_BYTES;     // two P tiles
+  uint8_t* sQ = smem;                               // two query tiles
+  uint8_t* sKV = sQ + 2 * S::Q_BYTES;               // per stage: K tile then V^T tile
+  uint8_t* sP = sKV + S::STAGES * S::KV_BYTES;      // one P tile per query tile
   uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * S::P_BYTES);
   uint64_t* q_full = bar;
   uint64_t* kv_full = bar + 1;
   uint64_t* kv_empty = kv_full + S::STAGES;
-  uint64_t* s_full = kv_empty + S::STAGES;
+  uint64_t* s_full = kv_empty + S::STAGES;  // [2], per query tile
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 1;
+  uint64_t* drain = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* armed = const_cast<int*>(abort_flag + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int qp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // qp: pair of query tiles
   const int N = p.N;
   const int nkv = (N + S::BN - 1) / S::BN;
   const int bh = b * p.H + h;
@@ -129,10 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
       mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    armed[S::STAGES] = -1;  // q tile
+    armed[S::STAGES] = -1;  // query tiles
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_attn_err) != 0) ? 1 : 0;
     fence_barrier_init();
   }
@@ -152,10 +156,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ0);
       tma_prefetch_desc(&tmK0);
       tma_prefetch_desc(&tmV);
-      const int qrow = bh * N + qt * S::BM;
-      mbar_arrive_expect_tx(q_full, S::Q_BYTES);
-      tma_load_2d(sQ, &tmQ0, q_full, 0, qrow);
-      if (S::C1) tma_load_2d(sQ + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow);
+      const int qrow = bh * N + qp * 2 * S::BM;
+      mbar_arrive_expect_tx(q_full, 2 * S::Q_BYTES);
+      for (int t = 0; t < 2; ++t) {
+        tma_load_2d(sQ + t * S::Q_BYTES, &tmQ0, q_full, 0, qrow + t * S::BM);
+        if (S::C1) tma_load_2d(sQ + t * S::Q_BYTES + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow + t * S::BM);
+      }
       armed[S::STAGES] = 0;
       const int krow = bh * N;
       const int vrow = bh * D;
@@ -183,23 +189,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- MMA
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BN);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D);
-      const uint32_t tO = tmem + 256;
-      const uint32_t q_addr = smem_u32(sQ);
       bool issued = false;
       bool ok = mbar_wait(q_full, 0, abort_flag, &g_attn_err);
-      auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort_flag, &g_attn_err)) return false;
+      // O_t += P_t V_i for query tile t and key tile i.
+      auto issue_pv = [&](int t, int i) -> bool {
+        if (!mbar_wait(&p_full[t], i & 1, abort_flag, &g_attn_err)) return false;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sP + (i & 1) * S::P_BYTES);
+        const uint32_t p_addr = smem_u32(sP + t * S::P_BYTES);
         const uint32_t v_addr = smem_u32(sKV + (i % S::STAGES) * S::KV_BYTES + S::K_BYTES);
+        const uint32_t tO = tmem + t * 256 + 128;
 #pragma unroll
         for (int ks = 0; ks < S::BN / 16; ++ks) {
           const uint64_t ad = smem_desc(p_addr + (ks >> 2) * (S::BM * 128) + (ks & 3) * 32, 1024, 2);
           const uint64_t bd = smem_desc(v_addr + (ks >> 2) * S::V1_OFF + (ks & 3) * 32, 1024, 2);
           umma_bf16(tO, ad, bd, idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(&kv_empty[i % S::STAGES]);
-        umma_commit(o_done);
+        umma_commit(&o_done[t]);
         return true;
       };
       for (int j = 0; ok && j < nkv; ++j) {
@@ -208,24 +213,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        if (j >= 2 && !mbar_wait(&s_free[j & 1], ((j >> 1) - 1) & 1, abort_flag, &g_attn_err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         const uint32_t k_addr = smem_u32(sKV + s * S::KV_BYTES);
-        const uint32_t tS = tmem + (j & 1) * 128;
+        for (int t = 0; t < 2 && ok; ++t) {
+          // S_t is single-buffered: the softmax must have read S_t of tile j-1.
+          if (j >= 1 && !mbar_wait(&s_free[t], (j - 1) & 1, abort_flag, &g_attn_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t q_addr = smem_u32(sQ + t * S::Q_BYTES);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(tS, qk_desc<D>(q_addr, ks), qk_desc<D>(k_addr, ks), idesc_s, ks > 0 ? 1u : 0u);
-        issued = true;
-        umma_commit(&s_full[j & 1]);
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
+          for (int ks = 0; ks < D / 16; ++ks)
+            umma_bf16(tmem + t * 256, qk_desc<D>(q_addr, ks), qk_desc<D>(k_addr, ks), idesc_s, ks > 0 ? 1u : 0u);
+          issued = true;
+          umma_commit(&s_full[t]);
+        }
+        if (ok && j >= 1) {
+          ok = issue_pv(0, j - 1) && issue_pv(1, j - 1);
+          if (ok) umma_commit(&kv_empty[(j - 1) % S::STAGES]);
         }
       }
-      if (ok) issue_pv(nkv - 1);
+      if (ok) ok = issue_pv(0, nkv - 1) && issue_pv(1, nkv - 1);
       if (*abort_flag && issued) {
         umma_commit(drain);
         drain_wait(drain, 0);
@@ -233,17 +241,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (!skip) {
     // ------------------------------------------------------------- softmax
-    const int quad = warp & 3;
+    const int t = (warp - 2) >> 2;   // query tile of this warpgroup
+    const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tO = tmem + 256 + lane_off;
+    const uint32_t tS = tmem + t * 256 + lane_off;
+    const uint32_t tO = tS + 128;
     const float sl2 = p.scale * 1.4426950408889634f;  // scale * log2(e)
+    uint8_t* pbuf = sP + t * S::P_BYTES;
     float m_ref = -INFINITY;  // running maximum of s * sl2 used as the exponent origin
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int buf = j & 1;
-      if (!mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, &g_attn_err)) {
+      if (!mbar_wait(&s_full[t], j & 1, abort_flag, &g_attn_err)) {
         ok = false;
         break;
       }
@@ -251,13 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float s[S::BN];
       {
         uint32_t raw[S::BN];
-        tmem_ld128(tmem + buf * 128 + lane_off, raw);
+        tmem_ld128(tS, raw);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < S::BN; ++c) s[c] = __uint_as_float(raw[c]);
       }
       tc_fence_before();
-      mbar_arrive(&s_free[buf]);
+      mbar_arrive(&s_free[t]);
       const int valid = N - j * S::BN;
       if (valid < S::BN) {
 #pragma unroll
@@ -280,19 +290,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_new;
       } else {
         need = m_new > m_ref + 8.0f;
-      }
-      if (__any_sync(0xffffffffu, need)) {
-        // O must be scaled before P_j V_j accumulates: wait for P_{j-1} V_{j-1}.
-        if (!mbar_wait(o_done, (j - 1) & 1, abort_flag, &g_attn_err)) {
+        // P_t V_{j-1} must be complete before P_t is overwritten and before O_t is
+        // rescaled.
+        if (!mbar_wait(&o_done[t], (j - 1) & 1, abort_flag, &g_attn_err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
-        if (need) {
-          m_ref = m_new;
-          l *= alpha;
+      }
+      const bool any_need = __any_sync(0xffffffffu, need);
+      const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+      if (need) {
+        m_ref = m_new;
+        l *= alpha;
+      }
+      // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
+      const float neg = -m_ref;
+      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c16 = 0; c16 < S::BN / 8; ++c16) {
+        float e[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          e[i] = fast_exp2(fmaf(s[c16 * 8 + i], sl2, neg));
+          l8[i] += e[i];
         }
+        const int blk = c16 >> 3, cc = c16 & 7;
+        uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+        *dst = pack_bf16x8(e);
+      }
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      if (any_need) {
+        // Scale O_t to the new exponent origin before P_t V_j accumulates into it (the
+        // wait on P_t V_{j-1} above made O_t stable).
 #pragma unroll
         for (int c = 0; c < D; c += 16) {
           uint32_t o[16];
@@ -304,39 +334,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
       }
-      // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
-      uint8_t* pbuf = sP + buf * S::P_BYTES;
-      const float neg = -m_ref;
-      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c16 = 0; c16 < S::BN / 8; ++c16) {
-        float e[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          // a quarter of the exponentials on the FMA pipe, the rest on MUFU
-          const float x = fmaf(s[c16 * 8 + i], sl2, neg);
-          e[i] = (i >= 6) ? soft_exp2(x) : fast_exp2(x);
-          l8[i] += e[i];
-        }
-        const int blk = c16 >> 3, cc = c16 & 7;
-        uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
-        *dst = pack_bf16x8(e);
-      }
-      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[buf]);
+      mbar_arrive(&p_full[t]);
     }
-    if (ok) {
-      // wait for the last two P V products (phases are checked in order)
-      if (nkv >= 2) ok = mbar_wait(o_done, (nkv - 2) & 1, abort_flag, &g_attn_err);
-      if (ok) ok = mbar_wait(o_done, (nkv - 1) & 1, abort_flag, &g_attn_err);
-    }
+    if (ok) ok = mbar_wait(&o_done[t], (nkv - 1) & 1, abort_flag, &g_attn_err);
     if (ok) {
       tc_fence_after();
       float o[D];
       load_cols<D>(tO, o);
-      const int n = qt * S::BM + r;
+      const int n = (qp * 2 + t) * S::BM + r;
       if (n < N) {
         const float inv = 1.0f / l;
 #pragma unroll
@@ -380,7 +387,7 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
   }
   if (!make_tmap_2d(&v, p.vt, static_cast<uint64_t>(p.B) * p.H * D, p.N, p.ld_vt, D, 64, 128))
     return cudaErrorInvalidValue;
-  dim3 grid((p.N + S::BM - 1) / S::BM, p.H, p.B);
+  dim3 grid((p.N + 2 * S::BM - 1) / (2 * S::BM), p.H, p.B);
   attn_fwd_tcgen05<D><<<grid, kThreads, S::SMEM_BYTES, stream>>>(q0, q1, k0, k1, v, p);
   return cudaGetLastError();
 }
