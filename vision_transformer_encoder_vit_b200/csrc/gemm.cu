@@ -8,15 +8,20 @@
 // with GELU, projector Linear(1280,6144), GELU, Linear(6144,6144), Linear(24576,6144),
 // GELU, Linear(6144,6144)).
 //
+// Two kernels share one epilogue:
+//  * gemm_bf16_tcgen05: one CTA per 128 x BN tile.
+//  * gemm_bf16_tcgen05_pair: a cluster of two CTAs (the two SMs of a TPC) per
+//    256 x BN tile with tcgen05.mma.cta_group::2.  Each CTA stages its own 128 rows of A
+//    and BN/2 rows of B, so an SM streams 32 KB of operands per 64-deep K step instead
+//    of 48 KB, and six stages fit in shared memory.  The even CTA issues the MMAs and
+//    both CTAs drain their own 128 accumulator rows.  No load uses multicast.
 // CTA = 6 warps: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the MMAs
 // (one thread), warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
-// Tiles are 128 x BN with a 64-deep K step (one 128-byte swizzle atom), a
-// STAGES-deep ring of operand tiles, and two TMEM accumulators so that the epilogue
-// of one tile overlaps the main loop of the next.  Tiles are walked m-fastest by a
-// persistent grid (one CTA per SM), so concurrently running CTAs share the same
-// weight tile through L2.
-#include "ptx.cuh"
+// K steps are 64 deep (one 128-byte swizzle atom); two TMEM accumulators let the
+// epilogue of one tile overlap the main loop of the next.  Tiles are walked m-fastest
+// by a persistent grid, so concurrently running CTAs share each weight tile via L2.
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace vt {
 namespace {
@@ -27,10 +32,11 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 192;
 
-template <int BN>
+template <int BN, bool PAIR>
 struct GemmShape {
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA stages
   static constexpr int A_BYTES = kBM * kBK * 2;
-  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int B_BYTES = B_ROWS * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
@@ -39,7 +45,8 @@ struct GemmShape {
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tiles must keep 1024-byte alignment");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
+  static_assert(!PAIR || (BN / 2) % 8 == 0, "half of B must be whole 8-row groups");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -71,11 +78,131 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = global_ns();
+  while (global_ns() - t0 < ns) {
+  }
+}
+
+// Drains one accumulator: this thread's row `row`, columns [col0, col0 + BN), the
+// warp's TMEM lane quadrant at t_row.  Waits for the accumulator (tfull, phase
+// `parity`) itself, after issuing the loads it can issue early.  Returns false on abort.
+template <int BN, class RL, bool PAIR>
+__device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int col0, uint32_t t_row, uint64_t* tfull,
+                                              uint32_t parity, volatile int* abort_flag) {
+  auto wait_acc = [&]() -> bool {
+    const bool ok = PAIR ? mbar_wait_cluster(tfull, parity, abort_flag, &g_gemm_err)
+                         : mbar_wait(tfull, parity, abort_flag, &g_gemm_err);
+    if (ok) tc_fence_after();
+    return ok;
+  };
+  if constexpr (RL::D == 0) {
+    const bf16* bias = static_cast<const bf16*>(p.bias);
+    const bf16* resid = static_cast<const bf16*>(p.resid);
+    bf16* out = static_cast<bf16*>(p.out);
+    // Bias and residual of a 32-column chunk are loaded one chunk ahead (the first
+    // chunk before waiting for the accumulator) so that no global-load latency sits
+    // between the TMEM read and the store.
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    auto prefetch = [&](int col, uint4* bq, uint4* rq) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int cg = col + 8 * g;
+        bq[g] = (bias && cg < p.N) ? __ldg(reinterpret_cast<const uint4*>(bias + cg)) : zero;
+        rq[g] = (resid && cg < p.N && row < p.M)
+                    ? *reinterpret_cast<const uint4*>(resid + static_cast<size_t>(row) * p.ldr + cg)
+                    : zero;
+      }
+    };
+    uint4 bq[4], rq[4];
+    prefetch(col0, bq, rq);
+    if (!wait_acc()) return false;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      const int col = col0 + c0;
+      if (col >= p.N) break;
+      uint4 bn_[4] = {zero, zero, zero, zero}, rn_[4] = {zero, zero, zero, zero};
+      if (c0 + 32 < BN) prefetch(col + 32, bn_, rn_);
+      float v[32];
+      load_cols<32>(t_row + c0, v);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int cg = col + 8 * g;
+        if (cg < p.N) {
+          if (bias) add_bf16x8(v + 8 * g, bq[g]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float x = v[8 * g + i];
+            if (p.act == ACT_GELU_TANH) x = gelu_tanh(x);
+            else if (p.act == ACT_GELU_ERF) x = gelu_erf(x);
+            v[8 * g + i] = x;
+          }
+          if (row < p.M) {
+            if (resid) add_bf16x8(v + 8 * g, rq[g]);
+            *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.ldo + cg) = pack_bf16x8(v + 8 * g);
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        bq[g] = bn_[g];
+        rq[g] = rn_[g];
+      }
+    }
+  } else {
+    if (!wait_acc()) return false;
+    constexpr int D = RL::D;
+    constexpr int HPT = BN / D;
+    const bf16* bias = static_cast<const bf16*>(p.bias);
+    const int width = p.heads * D;
+    int b = 0, n = 0, tp = 0, hp = 0, wp = 0;
+    if (row < p.M) {
+      b = row / p.ntok;
+      n = row - b * p.ntok;
+      token_position(n, p.gh, p.gw, p.order, &tp, &hp, &wp);
+    }
+#pragma unroll 1
+    for (int hh = 0; hh < HPT; ++hh) {
+      const int col = col0 + hh * D;
+      if (col >= p.N) break;
+      float v[D];
+      load_cols<D>(t_row + hh * D, v);
+      if (bias) {
+#pragma unroll
+        for (int g = 0; g < D / 8; ++g) add_bf16x8(v + 8 * g, *reinterpret_cast<const uint4*>(bias + col + 8 * g));
+      }
+      const int which = col / width;
+      const int head = (col - which * width) / D;
+      if (row < p.M) {
+        if (which < 2) {
+          if (p.rope) {
+            const float2* tab = p.rope_tab;
+            rope_block<0, RL::S0>(v, tab + (static_cast<size_t>(0 * kRopeMaxPos + tp) * kRopePairs));
+            rope_block<RL::S0, RL::S1>(v, tab + (static_cast<size_t>(1 * kRopeMaxPos + hp) * kRopePairs));
+            rope_block<RL::S0 + RL::S1, RL::S2>(v, tab + (static_cast<size_t>(2 * kRopeMaxPos + wp) * kRopePairs));
+          }
+          bf16* dst = static_cast<bf16*>(which == 0 ? p.q : p.k) +
+                      ((static_cast<size_t>(b) * p.heads + head) * p.ntok + n) * D;
+#pragma unroll
+          for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(v + 8 * g);
+        } else {
+          bf16* dst = static_cast<bf16*>(p.vt) + (static_cast<size_t>(b) * p.heads + head) * D * p.ld_vt + n;
+#pragma unroll
+          for (int d = 0; d < D; ++d) dst[static_cast<size_t>(d) * p.ld_vt] = __float2bfloat16_rn(v[d]);
+        }
+      }
+    }
+  }
+  return true;
+}
+
+// ------------------------------------------------------------ one CTA per tile
+
 template <int BN, class RL>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmParams p) {
-  using S = GemmShape<BN>;
+  using S = GemmShape<BN, false>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -151,6 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag) {  // let every load already issued land before the CTA exits
         for (int s = 0; s < S::STAGES; ++s)
           if (armed[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(armed[s]));
+      } else {
+        // Wait until the MMAs released every stage (their commits arrive asynchronously).
+        for (int i = 0; i < S::STAGES; ++i) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) break;
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
       }
     }
   } else if (!skip && warp == 1) {
@@ -204,105 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-      if constexpr (RL::D == 0) {
-        const bf16* bias = static_cast<const bf16*>(p.bias);
-        const bf16* resid = static_cast<const bf16*>(p.resid);
-        bf16* out = static_cast<bf16*>(p.out);
-        // Bias and residual of a 32-column chunk are loaded one chunk ahead (the first
-        // chunk before waiting for the accumulator) so that no global-load latency sits
-        // between the TMEM read and the store.
-        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-        auto prefetch = [&](int col, uint4* bq, uint4* rq) {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int cg = col + 8 * g;
-            bq[g] = (bias && cg < p.N) ? __ldg(reinterpret_cast<const uint4*>(bias + cg)) : zero;
-            rq[g] = (resid && cg < p.N && row < p.M)
-                        ? *reinterpret_cast<const uint4*>(resid + static_cast<size_t>(row) * p.ldr + cg)
-                        : zero;
-          }
-        };
-        uint4 bq[4], rq[4];
-        prefetch(nb * BN, bq, rq);
-        if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          const int col = nb * BN + c0;
-          if (col >= p.N) break;
-          uint4 bn_[4] = {zero, zero, zero, zero}, rn_[4] = {zero, zero, zero, zero};
-          if (c0 + 32 < BN) prefetch(col + 32, bn_, rn_);
-          float v[32];
-          load_cols<32>(t_row + c0, v);
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int cg = col + 8 * g;
-            if (cg < p.N) {
-              if (bias) add_bf16x8(v + 8 * g, bq[g]);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                float x = v[8 * g + i];
-                if (p.act == ACT_GELU_TANH) x = gelu_tanh(x);
-                else if (p.act == ACT_GELU_ERF) x = gelu_erf(x);
-                v[8 * g + i] = x;
-              }
-              if (row < p.M) {
-                if (resid) add_bf16x8(v + 8 * g, rq[g]);
-                *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.ldo + cg) = pack_bf16x8(v + 8 * g);
-              }
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            bq[g] = bn_[g];
-            rq[g] = rn_[g];
-          }
-        }
-      } else {
-        if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
-        tc_fence_after();
-        constexpr int D = RL::D;
-        constexpr int HPT = BN / D;
-        const bf16* bias = static_cast<const bf16*>(p.bias);
-        const int width = p.heads * D;
-        int b = 0, n = 0, tp = 0, hp = 0, wp = 0;
-        if (row < p.M) {
-          b = row / p.ntok;
-          n = row - b * p.ntok;
-          token_position(n, p.gh, p.gw, p.order, &tp, &hp, &wp);
-        }
-#pragma unroll 1
-        for (int hh = 0; hh < HPT; ++hh) {
-          const int col = nb * BN + hh * D;
-          if (col >= p.N) break;
-          float v[D];
-          load_cols<D>(t_row + hh * D, v);
-          if (bias) {
-#pragma unroll
-            for (int g = 0; g < D / 8; ++g) add_bf16x8(v + 8 * g, *reinterpret_cast<const uint4*>(bias + col + 8 * g));
-          }
-          const int which = col / width;
-          const int head = (col - which * width) / D;
-          if (row < p.M) {
-            if (which < 2) {
-              if (p.rope) {
-                const float2* tab = p.rope_tab;
-                rope_block<0, RL::S0>(v, tab + (static_cast<size_t>(0 * kRopeMaxPos + tp) * kRopePairs));
-                rope_block<RL::S0, RL::S1>(v, tab + (static_cast<size_t>(1 * kRopeMaxPos + hp) * kRopePairs));
-                rope_block<RL::S0 + RL::S1, RL::S2>(v, tab + (static_cast<size_t>(2 * kRopeMaxPos + wp) * kRopePairs));
-              }
-              bf16* dst = static_cast<bf16*>(which == 0 ? p.q : p.k) +
-                          ((static_cast<size_t>(b) * p.heads + head) * p.ntok + n) * D;
-#pragma unroll
-              for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(v + 8 * g);
-            } else {
-              bf16* dst = static_cast<bf16*>(p.vt) + (static_cast<size_t>(b) * p.heads + head) * D * p.ld_vt + n;
-#pragma unroll
-              for (int d = 0; d < D; ++d) dst[static_cast<size_t>(d) * p.ld_vt] = __float2bfloat16_rn(v[d]);
-            }
-          }
-        }
-      }
+      if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag)) break;
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -317,9 +355,190 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------- two CTAs per 256-row tile
+
+template <int BN, class RL>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const GemmParams p) {
+  using S = GemmShape<BN, true>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S::STAGES * S::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);  // used in the even CTA
+  uint64_t* empty = full + S::STAGES;                                          // both CTAs
+  uint64_t* tfull = empty + S::STAGES;                                         // both CTAs
+  uint64_t* tempty = tfull + 2;                                                // even CTA
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* armed = const_cast<int*>(abort_flag + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int m_tiles = (p.M + 2 * kBM - 1) / (2 * kBM);
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int nk = (p.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      armed[s] = -1;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_gemm_err) != 0) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();  // barrier inits and TMEM allocation visible to both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // Both CTAs must take the same path: skip only if either saw an earlier error.
+  const bool skip = *abort_flag != 0;
+
+  if (!skip && warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      // Both CTAs load their own halves; completion is counted on the even CTA's
+      // full[stage], armed by the even CTA for the bytes of both.
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+        const int mb = tile % m_tiles, nb = tile / m_tiles;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE_BYTES);
+          tma_load_2d_pair(sA + stage * S::A_BYTES, &tmA, full_leader, kb * kBK, mb * 2 * kBM + rank * kBM);
+          tma_load_2d_pair(sB + stage * S::B_BYTES, &tmB, full_leader, kb * kBK, nb * BN + rank * (BN / 2));
+          armed[stage] = static_cast<int>(phase);
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        if (rank == 0)
+          for (int s = 0; s < S::STAGES; ++s)
+            if (armed[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(armed[s]));
+      } else {
+        // Wait until the MMAs released every stage, so that no arrival from the even
+        // CTA's commits is still on its way to this CTA's barriers when it exits.
+        for (int i = 0; i < S::STAGES; ++i) {
+          if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) break;
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (!skip && warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // -------------------------------------------------------- MMA (even CTA)
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool issued_any = false;
+      for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+        const int acc = it & 1;
+        if (!mbar_wait_cluster(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, &g_gemm_err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_cluster(&full[stage], phase, abort_flag, &g_gemm_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * S::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * S::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            umma_bf16_pair(d_tmem, smem_desc(a_addr + kk * 32, 1024, 2), smem_desc(b_addr + kk * 32, 1024, 2),
+                           idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          const uint32_t e_local = smem_u32(&empty[stage]);
+          umma_commit_pair(mapa_shared(e_local, 0));
+          umma_commit_pair(mapa_shared(e_local, 1));
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        const uint32_t t_local = smem_u32(&tfull[acc]);
+        umma_commit_pair(mapa_shared(t_local, 0));
+        umma_commit_pair(mapa_shared(t_local, 1));
+      }
+      if (*abort_flag && issued_any) {
+        umma_commit_pair(mapa_shared(smem_u32(drain), 0));
+        drain_wait(drain, 0);
+      }
+    }
+  } else if (!skip) {
+    // ------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+      const int acc = it & 1;
+      const int mb = tile % m_tiles, nb = tile / m_tiles;
+      const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
+      const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
+      if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag)) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
+    }
+  }
+
+  // Neither CTA may leave while the pair's MMAs, loads or arrivals can still touch it.
+  if (*abort_flag) spin_ns(20000);
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------- launch
+
 template <int BN, class RL>
 cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
-  using S = GemmShape<BN>;
+  using S = GemmShape<BN, false>;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05<BN, RL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -336,17 +555,53 @@ cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int BN, class RL>
+cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
+  using S = GemmShape<BN, true>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_pair<BN, RL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, p.A, p.M, p.K, p.lda, kBM, kBK, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN / 2, kBK, 128)) return cudaErrorInvalidValue;
+  const int tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
+  const int max_pairs = device_sm_count() / 2;
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return cudaSuccess;
+  // Pairs of CTAs (256-row tiles) once there are enough rows to keep them busy.
+  const bool pair = p.M >= 1024;
   if (qkv_mode) {
     if (p.head_dim == 80 && p.sections[0] == 16 && p.sections[1] == 32 && p.sections[2] == 32)
-      return launch_one<240, Rope80>(p, stream);
+      return pair ? launch_pair<240, Rope80>(p, stream) : launch_one<240, Rope80>(p, stream);
     if (p.head_dim == 32 && p.sections[0] == 8 && p.sections[1] == 12 && p.sections[2] == 12)
       return launch_one<256, Rope32>(p, stream);
     return cudaErrorNotSupported;
   }
+  if (pair) return launch_pair<256, Rope0>(p, stream);
   // Wide tiles when they still fill the SMs; narrower ones for small problems.
   const int sms = device_sm_count();
   const long tiles256 = static_cast<long>((p.M + kBM - 1) / kBM) * ((p.N + 255) / 256);
