@@ -43,6 +43,27 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+KERNEL_SOURCES = {"gemm": "gemm.cu", "attention": "attention.cu"}
+
+
+def recorded_traffic(cls: str, workload_name: str):
+    """Per-launch DRAM bytes of a kernel class from the committed ncu capture
+    (profiles/traffic_<workload>.txt), or None if there is none for this workload or
+    the kernel's sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
+    if not os.path.exists(path):
+        return None
+    csrc = os.path.join(ROOT, "vision_transformer_encoder_vit_b200", "csrc")
+    data = open(os.path.join(csrc, KERNEL_SOURCES[cls]), "rb").read() + open(os.path.join(csrc, "ptx.cuh"), "rb").read()
+    sha = hashlib.sha1(data).hexdigest()
+    for line in open(path):
+        f = line.split()
+        if len(f) >= 8 and f[0] == "kernel_class" and f[1] == cls:
+            return float(f[7]) if f[3] == sha else None
+    return None
+
+
 def workload(name: str) -> dict:
     """Shape of the benchmarked step."""
     if name in ("tower448", "tower2016"):
@@ -366,7 +387,9 @@ def run_gpu(args, wl):
         roofline = dict(bound="tensor", kernel=("gemm_bf16_tcgen05 (all linear layers)" if dom == "gemm"
                                                  else "attn_fwd_tcgen05"),
                         achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
-                        peak_source=f"{peaks_kind} bf16 sustained", traffic=None,
+                        peak_source=f"{peaks_kind} bf16 sustained",
+                        traffic=recorded_traffic(dom, {"tower448": "tower448_b8"}.get(wl["name"], wl["name"])),
+                        traffic_unit="bytes per launch (ncu dram read + write)",
                         per_launch_flops=p["flops"] / max(p["launches"], 1),
                         avg_launch_us=1000.0 * p["ms"] / max(p["launches"], 1))
         classes = {k: dict(ms_per_step=v["ms"] / args.profile_steps,
