@@ -601,7 +601,23 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) 
       return launch_one<256, Rope32>(p, stream);
     return cudaErrorNotSupported;
   }
-  if (pair) return launch_pair<256, Rope0>(p, stream);
+  if (pair) {
+    // 224-wide tiles when they fill the last wave of CTA pairs clearly better than
+    // 256-wide ones (measured on B200 for short-K, 1280-wide outputs such as the
+    // attention output projection of 8 images at 448x448).
+    if (p.K <= 2048) {
+      const int pairs = device_sm_count() / 2;
+      const int mt = (p.M + 2 * kBM - 1) / (2 * kBM);
+      auto eff = [&](int bn) {
+        const int nt = (p.N + bn - 1) / bn;
+        const long tiles = static_cast<long>(mt) * nt;
+        const long waves = (tiles + pairs - 1) / pairs;
+        return (static_cast<double>(tiles) / (waves * pairs)) * (static_cast<double>(p.N) / (nt * bn));
+      };
+      if (eff(224) * 0.93 > eff(256)) return launch_pair<224, Rope0>(p, stream);
+    }
+    return launch_pair<256, Rope0>(p, stream);
+  }
   // Wide tiles when they still fill the SMs; narrower ones for small problems.
   const int sms = device_sm_count();
   const long tiles256 = static_cast<long>((p.M + kBM - 1) / kBM) * ((p.N + 255) / 256);
