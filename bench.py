@@ -29,6 +29,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from vision_transformer_encoder_vit_b200 import replicas as REP  # noqa: E402
 from vision_transformer_encoder_vit_b200 import synthetic as S  # noqa: E402
 
 METRIC = "ViT tower images/s & tokens/s at 448²/2016²; attention+GEMM TFLOP/s vs BF16 peak"
@@ -201,7 +202,7 @@ def oracle_attention(wl: dict, budget_s: float = 15.0) -> dict:
 # --------------------------------------------------------------- reference
 
 def run_reference(args, wl):
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = REP.rank_env()
     if rank != 0:
         return
     steps = []
@@ -232,9 +233,7 @@ def run_gpu(args, wl):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = REP.rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
@@ -251,7 +250,7 @@ def run_gpu(args, wl):
     if wl["kind"] == "tower":
         cfg = wl["cfg"]
         tower = V.Tower(cfg, S.make_weights(cfg))
-        px_host = torch.from_numpy(S.make_pixels(cfg, batch=B, seed=cfg["seed"] + rank)).pin_memory()
+        px_host = torch.from_numpy(S.make_pixels(cfg, batch=B, seed=REP.replica_seed(cfg["seed"], rank))).pin_memory()
         px = px_host.to(dev)
         ws = tower.workspace(B, grid)
         out = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16, device=dev)
@@ -336,12 +335,9 @@ def run_gpu(args, wl):
     clk = clocks.stop()
     V.vt_check(stream)
     ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = REP.max_over_ranks(ms, dev)
     ms_per_step = ms / args.steps
-    value = world * units_per_step * args.steps / (ms / 1000.0)
+    value = REP.job_throughput(units_per_step, args.steps, ms, world)
 
     # ---------------- per-kernel-class times of one profiled step (events around each launch)
     V.vt_profile_begin(stream)
@@ -369,11 +365,8 @@ def run_gpu(args, wl):
         e_e.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_s.elapsed_time(e_e)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = dict(value=world * B * args.steps / (e2e_ms / 1000.0), unit=unit,
+        e2e_ms = REP.max_over_ranks(e2e_ms, dev)
+        e2e = dict(value=REP.job_throughput(B, args.steps, e2e_ms, world), unit=unit,
                    h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h.numel() * 2),
                    api="vt_forward_host")
         del ws_h

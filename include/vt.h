@@ -236,6 +236,13 @@ VT_API vt_status vt_index_maps(const int32_t* grid_thw, int32_t* token_order, in
  * (VT_ERR_TIMEOUT), clearing them, and pending launch errors (VT_ERR_CUDA). */
 VT_API vt_status vt_check(void* stream);
 
+/* Diagnostic of the failure-detection path.  Launches one CTA whose only waiting
+ * thread waits on an mbarrier that nothing arrives on; the wait is bounded like every
+ * wait in the library's kernels, gives up after 1 s, records a device timeout and
+ * returns.  The following vt_check() then returns VT_ERR_TIMEOUT (and clears it);
+ * the CUDA context stays usable.  Nothing faults, traps or hangs. */
+VT_API vt_status vt_selftest_wait_timeout(void* stream);
+
 /* Message of the calling thread's last failed call ("" if none). */
 VT_API const char* vt_last_error(void);
 

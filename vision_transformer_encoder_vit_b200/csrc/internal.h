@@ -108,6 +108,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
 
 int device_sm_count();
 
+unsigned int selftest_read_clear_error(cudaStream_t stream);
+
 // Sets the calling thread's message returned by vt_last_error().
 void set_error_message(const char* msg);
 

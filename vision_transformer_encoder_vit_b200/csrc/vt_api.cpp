@@ -731,7 +731,10 @@ vt_status vt_check(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "pending launch error");
   const unsigned int ge = gemm_read_clear_error(st);
   const unsigned int ae = attention_read_clear_error(st);
-  if (ge || ae) return fail(VT_ERR_TIMEOUT, "kernel wait limit reached (gemm flags %u, attention flags %u)", ge, ae);
+  const unsigned int se = selftest_read_clear_error(st);
+  if (ge || ae || se)
+    return fail(VT_ERR_TIMEOUT, "kernel wait limit reached (gemm flags %u, attention flags %u, self-test flags %u)",
+                ge, ae, se);
   return VT_OK;
 }
 

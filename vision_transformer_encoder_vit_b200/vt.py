@@ -76,6 +76,7 @@ _SIGS = {
     "vt_patch_unfold": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "vt_index_maps": ([_i32p, _i32p, _i32p, _i32p]),
     "vt_check": ([_vp]),
+    "vt_selftest_wait_timeout": ([_vp]),
     "vt_profile_begin": ([_vp]),
     "vt_profile_end": ([_vp]),
     "vt_profile_read": ([_i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
@@ -269,6 +270,10 @@ def vt_index_maps(grid_thw):
 
 def vt_check(stream=None) -> None:
     _check(lib.vt_check(_stream(stream)), "vt_check")
+
+
+def vt_selftest_wait_timeout(stream=None) -> None:
+    _check(lib.vt_selftest_wait_timeout(_stream(stream)), "vt_selftest_wait_timeout")
 
 
 def vt_profile_begin(stream=None) -> None:
