@@ -74,6 +74,14 @@ def workload(name: str) -> dict:
         return dict(kind="tower", name=name, cfg=cfg, batch=cfg["batch"], grid=(t, gh, gw), tokens=N,
                     desc=f"full tower (32 layers) + 2x2 merge + projector, {cfg['batch']} image(s) of "
                          f"{cfg['image'][0]}x{cfg['image'][1]}")
+    if name == "varlen_mix":
+        cfg = S.get_config("tower448")
+        images = [(448, 448), (336, 448), (224, 224), (672, 672), (448, 224), (560, 560), (280, 392), (448, 448)]
+        grids = [(1, h // cfg["patch"], w // cfg["patch"]) for h, w in images]
+        return dict(kind="varlen", name=name, cfg=cfg, batch=len(images), images=images, grids=grids,
+                    tokens=sum(g[1] * g[2] for g in grids),
+                    desc="full tower + 2x2 merge + projector on one packed batch of 8 images of mixed sizes "
+                         + ", ".join(f"{h}x{w}" for h, w in images))
     if name.startswith("attn"):
         n = int(name[4:])
         side = int(round(n ** 0.5))
@@ -244,7 +252,7 @@ def run_gpu(args, wl):
     stream = torch.cuda.current_stream()
     peaks, peaks_kind = load_peaks()
     B = wl["batch"]
-    grid = wl["grid"]
+    grid = wl.get("grid")
     N = wl["tokens"]
 
     if wl["kind"] == "tower":
@@ -255,11 +263,29 @@ def run_gpu(args, wl):
         ws = tower.workspace(B, grid)
         out = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16, device=dev)
 
-        def step():
-            V.vt_forward(tower.h, px, grid, B, out, None, ws, ws.numel(), stream)
+        def launch(s_):
+            V.vt_forward(tower.h, px, grid, B, out, None, ws, ws.numel(), s_)
 
         flops = tower_flops(cfg, N)
         step_flops = B * flops["total"]
+        units_per_step = B
+        unit = "images/s"
+    elif wl["kind"] == "varlen":
+        cfg = wl["cfg"]
+        tower = V.Tower(cfg, S.make_weights(cfg))
+        pix = [S.make_pixels(dict(cfg, image=hw), batch=1, seed=REP.replica_seed(cfg["seed"], rank) + i)[0]
+               for i, hw in enumerate(wl["images"])]
+        px_host = torch.from_numpy(np.concatenate([a.ravel() for a in pix])).pin_memory()
+        px = px_host.to(dev)
+        grids = wl["grids"]
+        ws_bytes = V.vt_workspace_bytes_varlen(tower.h, grids)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        out = torch.empty((N // 4, cfg["proj_out"]), dtype=torch.bfloat16, device=dev)
+
+        def launch(s_):
+            V.vt_forward_varlen(tower.h, px, grids, out, None, ws, ws_bytes, s_)
+
+        step_flops = sum(tower_flops(cfg, g[1] * g[2])["total"] for g in grids)
         units_per_step = B
         unit = "images/s"
     else:
@@ -273,12 +299,15 @@ def run_gpu(args, wl):
         ws_bytes = V.vt_attention_workspace_bytes(1, H, N, D)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
-        def step():
-            V.vt_attention(q, k, v, o, 1, H, N, D, pos, (16, 32, 32), 10000.0, D ** -0.5, ws, ws_bytes, stream)
+        def launch(s_):
+            V.vt_attention(q, k, v, o, 1, H, N, D, pos, (16, 32, 32), 10000.0, D ** -0.5, ws, ws_bytes, s_)
 
         step_flops = 4.0 * H * N * N * D
         units_per_step = 1
         unit = "calls/s"
+
+    def step():
+        launch(stream)
 
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
@@ -296,11 +325,7 @@ def run_gpu(args, wl):
             s2.wait_stream(stream)
             with torch.cuda.stream(s2):
                 with torch.cuda.graph(g, stream=s2):
-                    if wl["kind"] == "tower":
-                        V.vt_forward(tower.h, px, grid, B, out, None, ws, ws.numel(), s2)
-                    else:
-                        V.vt_attention(q, k, v, o, 1, H, N, D, pos, (16, 32, 32), 10000.0, D ** -0.5, ws,
-                                       ws_bytes, s2)
+                    launch(s2)
             stream.wait_stream(s2)
             g.replay()
             torch.cuda.synchronize()
@@ -392,7 +417,7 @@ def run_gpu(args, wl):
                            not v["flops"] else None)
                    for k, v in prof.items() if v["launches"]}
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and wl["kind"] in ("tower", "attn"):
             cpu = (oracle_images_per_s(wl["cfg"], args.cpu_budget) if wl["kind"] == "tower"
                    else oracle_attention(wl, args.cpu_budget))
             cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
@@ -401,11 +426,11 @@ def run_gpu(args, wl):
             ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
             data="synthetic: seeded N(0,0.02) bf16 weights, U[0,1] ImageNet-normalised pixels",
             config=dict(workload=wl["name"], description=wl["desc"], per_gpu_batch=B, global_batch=B * world,
-                        tokens_per_image=N, merged_tokens_per_image=N // 4,
+                        tokens_per_image=N / B, merged_tokens_per_image=(N // 4) / B,
                         l2="flushed (512 MB write) between timed steps", launch="cuda graph" if graph else "eager",
                         parallelism=f"replicas x{world}"),
-            tokens_per_s=value * N if wl["kind"] == "tower" else None,
-            output_tokens_per_s=value * N // 4 if wl["kind"] == "tower" else None,
+            tokens_per_s=value * N / B if wl["kind"] in ("tower", "varlen") else None,
+            output_tokens_per_s=value * (N // 4) / B if wl["kind"] in ("tower", "varlen") else None,
             tflops=world * step_flops * args.steps / (ms / 1000.0) / 1e12,
             roofline=roofline, kernel_classes=classes,
             cpu_baseline=cpu, e2e=e2e,

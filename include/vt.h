@@ -146,6 +146,22 @@ VT_API vt_status vt_forward_host(vt_handle* h, const float* pixels_host, const i
                           void* out_host, void* ws, size_t ws_bytes, void* stream);
 VT_API vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out);
 
+/* Variable-resolution batch: B images (1 <= B <= 64) of different patch grids in one
+ * call, their tokens packed into one sequence; attention stays within each image.
+ *   pixels  device fp32, the images' [3, H_b, W_b] arrays concatenated in order
+ *           (H_b = grids[3b+1]*patch, W_b = grids[3b+2]*patch)
+ *   grids   host int32 [B, 3] (t, h, w) per image; t = 1, h and w even, <= 4096
+ *   out     device bf16 [sum_b N_b/4, proj_out]: image b's merged tokens (raster order)
+ *           follow image b-1's
+ *   tower_out  device bf16 [sum_b N_b, hidden] (raster order per image) or NULL
+ *   ws      device workspace of vt_workspace_bytes_varlen(h, B, grids) bytes
+ * Each image's result equals vt_forward on that image alone.  Source: the capacity
+ * discussion of "spark_model/layers/vision_encoder/enc_impl/init.rs" (images of any
+ * size up to a per-call bound share the encoder). */
+VT_API vt_status vt_workspace_bytes_varlen(const vt_handle* h, int B, const int32_t* grids, size_t* out);
+VT_API vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int32_t* grids, int B, void* out,
+                                   void* tower_out, void* ws, size_t ws_bytes, void* stream);
+
 /* One pre-LN tower layer i on raster-ordered tokens: x_out = layer_i(x_in), both
  * device bf16 [B, t*h*w, hidden]; x_in may equal x_out.  Source: ViTBlock of
  * "metrale_model_arch/weight_loader/qwen3_vl.rs" (norm1, qkv, proj, norm2, fc1, fc2);

@@ -130,6 +130,26 @@ def test_workspace_is_affine_in_tokens():
     V.vt_destroy(h)
 
 
+def test_varlen_workspace_and_argument_checks():
+    cfg = S.get_config("tower448")
+    h = V.vt_create(cfg)
+    one = V.vt_workspace_bytes(h, 1, (1, 32, 32))
+    assert V.vt_workspace_bytes_varlen(h, [(1, 32, 32)]) == one
+    mixed = V.vt_workspace_bytes_varlen(h, [(1, 32, 32), (1, 16, 24), (1, 2, 2)])
+    tokens = 1024 + 384 + 4
+    assert one < mixed <= 30208 * tokens + 64 * 256  # affine in the packed token count
+    with pytest.raises(V.VtError) as e:
+        V.vt_workspace_bytes_varlen(h, [(1, 32, 32), (1, 15, 24)])
+    assert _status(e) == "VT_ERR_SHAPE"
+    with pytest.raises(V.VtError) as e:
+        V.vt_workspace_bytes_varlen(h, [(1, 2, 2)] * 65)
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    with pytest.raises(V.VtError) as e:
+        V.vt_forward_varlen(h, 16, [(1, 2, 2)], 16, None, 16, 1 << 20)
+    assert _status(e) == "VT_ERR_NOT_LOADED"
+    V.vt_destroy(h)
+
+
 def test_attention_workspace_linear():
     s1 = V.vt_attention_workspace_bytes(1, 16, 6400, 80)
     s2 = V.vt_attention_workspace_bytes(1, 16, 65536, 80)

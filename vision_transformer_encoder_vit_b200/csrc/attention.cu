@@ -118,7 +118,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int qp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // qp: pair of query tiles
-  const int N = p.N;
+  // Tokens of this image and the packed token where they start.
+  const int N = p.varlen ? p.vl.tok_off[b + 1] - p.vl.tok_off[b] : p.N;
+  const int tok0 = p.varlen ? p.vl.tok_off[b] : b * p.N;
+  if (qp * 2 * S::BM >= N) return;  // a smaller image of a packed batch: nothing here
   const int nkv = (N + S::BN - 1) / S::BN;
   const int bh = b * p.H + h;
 
@@ -156,14 +159,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ0);
       tma_prefetch_desc(&tmK0);
       tma_prefetch_desc(&tmV);
-      const int qrow = bh * N + qp * 2 * S::BM;
+      const int qrow = tok0 * p.H + h * N + qp * 2 * S::BM;
       mbar_arrive_expect_tx(q_full, 2 * S::Q_BYTES);
       for (int t = 0; t < 2; ++t) {
         tma_load_2d(sQ + t * S::Q_BYTES, &tmQ0, q_full, 0, qrow + t * S::BM);
         if (S::C1) tma_load_2d(sQ + t * S::Q_BYTES + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow + t * S::BM);
       }
       armed[S::STAGES] = 0;
-      const int krow = bh * N;
+      const int krow = tok0 * p.H + h * N;
       const int vrow = bh * D;
       for (int j = 0; j < nkv; ++j) {
         const int s = j % S::STAGES;
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv = 1.0f / l;
 #pragma unroll
         for (int i = 0; i < D; ++i) o[i] *= inv;
-        bf16* dst = static_cast<bf16*>(p.o) + (static_cast<size_t>(b) * N + n) * (p.H * D) + h * D;
+        bf16* dst = static_cast<bf16*>(p.o) + (static_cast<size_t>(tok0) + n) * (p.H * D) + h * D;
 #pragma unroll
         for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(o + 8 * g);
       }
@@ -374,7 +377,7 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const uint64_t rows = static_cast<uint64_t>(p.B) * p.H * p.N;
+  const uint64_t rows = static_cast<uint64_t>(p.varlen ? p.vl.tok_off[p.vl.count] : p.B * p.N) * p.H;
   CUtensorMap q0, q1, k0, k1, v;
   if (!make_tmap_2d(&q0, p.q, rows, D, D, S::BM, S::C0, S::SW0)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&k0, p.k, rows, D, D, S::BN, S::C0, S::SW0)) return cudaErrorInvalidValue;
@@ -385,7 +388,7 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
     q1 = q0;
     k1 = k0;
   }
-  if (!make_tmap_2d(&v, p.vt, static_cast<uint64_t>(p.B) * p.H * D, p.N, p.ld_vt, D, 64, 128))
+  if (!make_tmap_2d(&v, p.vt, static_cast<uint64_t>(p.B) * p.H * D, p.varlen ? p.ld_vt : p.N, p.ld_vt, D, 64, 128))
     return cudaErrorInvalidValue;
   dim3 grid((p.N + 2 * S::BM - 1) / (2 * S::BM), p.H, p.B);
   attn_fwd_tcgen05<D><<<grid, kThreads, S::SMEM_BYTES, stream>>>(q0, q1, k0, k1, v, p);

@@ -171,6 +171,29 @@ __global__ void __launch_bounds__(256) patch_unfold_kernel(const float* __restri
   }
 }
 
+// Variable-resolution form: one block per packed token; the image comes from the table.
+__global__ void __launch_bounds__(256) patch_unfold_varlen_kernel(const float* __restrict__ px,
+                                                                  bf16* __restrict__ out, const VarlenTable vl,
+                                                                  int patch, int tp) {
+  const int row = blockIdx.x;
+  const int b = varlen_image(vl, row);
+  const int n = row - vl.tok_off[b];
+  const int gh = vl.gh[b], gw = vl.gw[b];
+  const int H = gh * patch, W = gw * patch;
+  int t, hh, ww;
+  token_position(n, gh, gw, ORDER_BLOCK, &t, &hh, &ww);
+  const int pp = patch * patch;
+  const int K = 3 * tp * pp;
+  bf16* dst = out + static_cast<size_t>(row) * K;
+  const float* img = px + vl.pix_off[b];
+  for (int e = threadIdx.x; e < 3 * pp; e += blockDim.x) {
+    const int c = e / pp, rem = e - c * pp;
+    const int kh = rem / patch, kw = rem - kh * patch;
+    const bf16 v = __float2bfloat16_rn(img[(static_cast<size_t>(c) * H + hh * patch + kh) * W + ww * patch + kw]);
+    for (int f = 0; f < tp; ++f) dst[c * tp * pp + f * pp + rem] = v;
+  }
+}
+
 // ------------------------------------------------------------------ reorder
 // Moves whole rows between raster order and 2x2-block order (the 2x2 merge of the
 // "MiniMax-M3 Vision" model card groups each block's four tokens).
@@ -284,6 +307,14 @@ cudaError_t launch_patch_unfold(const float* pixels, void* out, int B, int H, in
   if (rows <= 0) return cudaSuccess;
   patch_unfold_kernel<<<static_cast<unsigned>(rows), 256, 0, stream>>>(pixels, static_cast<bf16*>(out), H, W, patch,
                                                                        tp, gh, gw, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_patch_unfold_varlen(const float* pixels, void* out, const VarlenTable& vl, int patch, int tp,
+                                       cudaStream_t stream) {
+  const int rows = vl.tok_off[vl.count];
+  if (rows <= 0) return cudaSuccess;
+  patch_unfold_varlen_kernel<<<rows, 256, 0, stream>>>(pixels, static_cast<bf16*>(out), vl, patch, tp);
   return cudaGetLastError();
 }
 

@@ -155,11 +155,25 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
     constexpr int HPT = BN / D;
     const bf16* bias = static_cast<const bf16*>(p.bias);
     const int width = p.heads * D;
-    int b = 0, n = 0, tp = 0, hp = 0, wp = 0;
+    // Token n of image b, whose tokens start at packed row tok0 and number ntok.
+    int n = 0, tp = 0, hp = 0, wp = 0, ntok = p.ntok, ld_vt = p.ld_vt;
+    size_t tok0 = 0, vt0 = 0;
     if (row < p.M) {
-      b = row / p.ntok;
-      n = row - b * p.ntok;
-      token_position(n, p.gh, p.gw, p.order, &tp, &hp, &wp);
+      if (p.varlen) {
+        const int b = varlen_image(p.vl, row);
+        tok0 = static_cast<size_t>(p.vl.tok_off[b]);
+        ntok = p.vl.tok_off[b + 1] - p.vl.tok_off[b];
+        n = row - p.vl.tok_off[b];
+        ld_vt = p.vl.ld_vt[b];
+        vt0 = static_cast<size_t>(p.vl.vt_off[b]);
+        token_position(n, p.vl.gh[b], p.vl.gw[b], p.order, &tp, &hp, &wp);
+      } else {
+        const int b = row / p.ntok;
+        n = row - b * p.ntok;
+        tok0 = static_cast<size_t>(b) * p.ntok;
+        vt0 = static_cast<size_t>(b) * p.heads * D * p.ld_vt;
+        token_position(n, p.gh, p.gw, p.order, &tp, &hp, &wp);
+      }
     }
 #pragma unroll 1
     for (int hh = 0; hh < HPT; ++hh) {
@@ -181,14 +195,16 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
             rope_block<RL::S0, RL::S1>(v, tab + (static_cast<size_t>(1 * kRopeMaxPos + hp) * kRopePairs));
             rope_block<RL::S0 + RL::S1, RL::S2>(v, tab + (static_cast<size_t>(2 * kRopeMaxPos + wp) * kRopePairs));
           }
+          // [heads, ntok, D] block of this image, which starts at token tok0
           bf16* dst = static_cast<bf16*>(which == 0 ? p.q : p.k) +
-                      ((static_cast<size_t>(b) * p.heads + head) * p.ntok + n) * D;
+                      (tok0 * p.heads + static_cast<size_t>(head) * ntok + n) * D;
 #pragma unroll
           for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(v + 8 * g);
         } else {
-          bf16* dst = static_cast<bf16*>(p.vt) + (static_cast<size_t>(b) * p.heads + head) * D * p.ld_vt + n;
+          // [heads, D, ld_vt] block of this image at vt0
+          bf16* dst = static_cast<bf16*>(p.vt) + vt0 + static_cast<size_t>(head) * D * ld_vt + n;
 #pragma unroll
-          for (int d = 0; d < D; ++d) dst[static_cast<size_t>(d) * p.ld_vt] = __float2bfloat16_rn(v[d]);
+          for (int d = 0; d < D; ++d) dst[static_cast<size_t>(d) * ld_vt] = __float2bfloat16_rn(v[d]);
         }
       }
     }

@@ -34,6 +34,32 @@ __host__ __device__ inline void token_position(int n, int gh, int gw, int order,
   }
 }
 
+// --------------------------------------------------- variable-resolution batches
+
+// Images of different grids packed into one token sequence.  Passed by value as a
+// kernel parameter (so launches stay capturable in CUDA graphs).
+constexpr int kMaxVarlenImages = 64;
+struct VarlenTable {
+  int count;                              // images in the batch
+  int tok_off[kMaxVarlenImages + 1];      // first token of each image; tok_off[count] = total
+  int gh[kMaxVarlenImages];               // patch grid of each image (t = 1)
+  int gw[kMaxVarlenImages];
+  long long vt_off[kMaxVarlenImages];     // element offset of each image's v^T block
+  int ld_vt[kMaxVarlenImages];            // its row stride (tokens rounded up to 8)
+  long long pix_off[kMaxVarlenImages];    // float offset of each image's [3, H, W] pixels
+};
+
+// Image of packed token `row` (binary search over tok_off).
+__host__ __device__ inline int varlen_image(const VarlenTable& t, int row) {
+  int lo = 0, hi = t.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (t.tok_off[mid] <= row) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 // ------------------------------------------------------------------ GEMM
 
 enum GemmAct : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2 };
@@ -62,6 +88,11 @@ struct GemmParams {
   int rope;                 // 0: no rotation
   int sections[3];
   const float2* rope_tab;   // [3][kRopeMaxPos][kRopePairs] (cos, sin)
+  // Variable-resolution batch: rows are packed tokens of images of different grids.
+  // q and k of image b are [heads, N_b, head_dim] blocks starting at token tok_off[b];
+  // v^T of image b is [heads, head_dim, ld_vt[b]] at vt_off[b].
+  int varlen;
+  VarlenTable vl;
 };
 
 // Returns a CUDA error code (cudaSuccess on success); host-side shape checks are the
@@ -78,6 +109,12 @@ struct AttnParams {
   void* o;         // [B, N, H * D] bf16
   int B, H, N, D, ld_vt;
   float scale;
+  // Variable-resolution batch (varlen != 0): image b has vl.tok_off[b+1] - tok_off[b]
+  // tokens; q and k hold [H, N_b, D] blocks at token tok_off[b]; vt is [B, H, D, ld_vt]
+  // with one common ld_vt >= every N_b and zeros beyond N_b; o rows are packed tokens.
+  // N is then the largest N_b (it sizes the grid).
+  int varlen;
+  VarlenTable vl;
 };
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream);
 unsigned int attention_read_clear_error(cudaStream_t stream);
@@ -89,6 +126,10 @@ cudaError_t launch_layernorm(const void* x, const void* gamma, const void* beta,
 // pixels [B, 3, H, W] fp32 -> patch vectors [B * gh * gw, 3 * tp * p * p] bf16 in `order`.
 cudaError_t launch_patch_unfold(const float* pixels, void* out, int B, int H, int W, int patch, int tp,
                                 int order, cudaStream_t stream);
+// Packed images of different sizes (vl.pix_off, vl.gh, vl.gw) -> packed patch vectors
+// in 2x2-block order per image.
+cudaError_t launch_patch_unfold_varlen(const float* pixels, void* out, const VarlenTable& vl, int patch, int tp,
+                                       cudaStream_t stream);
 // Row gather: out[r] = in[src(r)] where src maps between raster and block order.
 // to_block != 0: out is block order, in is raster.  Rows of `cols` bf16 each.
 cudaError_t launch_reorder_rows(const void* in, void* out, int B, int gt, int gh, int gw, int cols, int to_block,

@@ -137,8 +137,16 @@ vt_status run_layernorm(const void* x, const void* g, const void* b, void* y, in
 }
 
 vt_status run_attention(const AttnParams& p, cudaStream_t st) {
-  const double flops = 4.0 * p.B * p.H * static_cast<double>(p.N) * p.N * p.D;
-  ProfScope ps(CLS_ATTN, flops, 8.0 * p.B * p.H * static_cast<double>(p.N) * p.D, st);
+  double n2 = static_cast<double>(p.B) * p.N * p.N, n1 = static_cast<double>(p.B) * p.N;
+  if (p.varlen) {  // per-image token counts of a packed batch
+    n2 = n1 = 0;
+    for (int b = 0; b < p.vl.count; ++b) {
+      const double n = p.vl.tok_off[b + 1] - p.vl.tok_off[b];
+      n2 += n * n;
+      n1 += n;
+    }
+  }
+  ProfScope ps(CLS_ATTN, 4.0 * p.H * n2 * p.D, 8.0 * p.H * n1 * p.D, st);
   cudaError_t e = launch_attention(p, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return VT_OK;
@@ -176,13 +184,14 @@ struct Plan {
   size_t x, xn, q, k, vt, o, hmid, unfold, y1, y2, z1, total;
 };
 
-Plan make_plan(const vt_config& c, int B, int t, int h, int w) {
+// Workspace layout for M packed tokens whose transposed v blocks take vt_elems elements.
+Plan make_plan_core(const vt_config& c, int M_, size_t vt_elems) {
   Plan p;
-  p.N = t * h * w;
-  p.M = B * p.N;
-  p.Mm = p.M / 4;
-  p.ld_vt = round8(p.N);
-  const size_t d = c.hidden, M = p.M;
+  p.N = 0;
+  p.ld_vt = 0;
+  p.M = M_;
+  p.Mm = M_ / 4;
+  const size_t d = c.hidden, M = static_cast<size_t>(M_);
   const size_t K0 = 3ull * c.temporal_patch * c.patch * c.patch;
   size_t off = 0;
   p.x = off;
@@ -197,7 +206,7 @@ Plan make_plan(const vt_config& c, int B, int t, int h, int w) {
   p.k = o2;
   o2 += align256(M * d * 2);
   p.vt = o2;
-  o2 += align256(static_cast<size_t>(B) * c.heads * c.head_dim * p.ld_vt * 2);
+  o2 += align256(vt_elems * 2);
   p.o = o2;
   o2 += align256(M * d * 2);
   p.hmid = o2;
@@ -212,6 +221,15 @@ Plan make_plan(const vt_config& c, int B, int t, int h, int w) {
   p.z1 = o3;
   o3 += align256(static_cast<size_t>(p.Mm) * c.proj_hidden * 2);
   p.total = std::max(o2, o3);
+  return p;
+}
+
+Plan make_plan(const vt_config& c, int B, int t, int h, int w) {
+  const int N = t * h * w;
+  const int ld = round8(N);
+  Plan p = make_plan_core(c, B * N, static_cast<size_t>(B) * c.heads * c.head_dim * ld);
+  p.N = N;
+  p.ld_vt = ld;
   return p;
 }
 
@@ -233,8 +251,10 @@ vt_status check_grid(const vt_handle* h, int B, const int32_t* g, int* t, int* g
 }
 
 // One pre-LN layer over M tokens stored at x (in place).
+// One pre-LN layer over the M tokens at x_in (written to x, which may equal x_in).  With
+// vl non-null the tokens are a packed batch of images of different grids.
 vt_status run_layer(vt_handle* h, int i, const void* x_in, void* x, int B, int gt, int gh, int gw, int order,
-                    char* ws, const Plan& pl, cudaStream_t st) {
+                    char* ws, const Plan& pl, cudaStream_t st, const VarlenTable* vl = nullptr) {
   const vt_config& c = h->cfg;
   const vt_handle::Layer& L = h->layers[i];
   const int d = c.hidden, M = pl.M;
@@ -259,12 +279,16 @@ vt_status run_layer(vt_handle* h, int i, const void* x_in, void* x, int B, int g
     p.sections[1] = c.rope_sections[1];
     p.sections[2] = c.rope_sections[2];
     p.rope_tab = h->rope_tab;
+    if (vl) {
+      p.varlen = 1;
+      p.vl = *vl;
+    }
     ProfScope ps(CLS_GEMM, 2.0 * M * 3.0 * d * d, 0, st);
     cudaError_t e = launch_gemm(p, st, 1);
     if (e != cudaSuccess) return cuda_fail(e, "qkv gemm launch");
   }
   {
-    AttnParams a;
+    AttnParams a{};
     a.q = ws + pl.q;
     a.k = ws + pl.k;
     a.vt = ws + pl.vt;
@@ -275,6 +299,17 @@ vt_status run_layer(vt_handle* h, int i, const void* x_in, void* x, int B, int g
     a.D = c.head_dim;
     a.ld_vt = pl.ld_vt;
     a.scale = 1.0f / std::sqrt(static_cast<float>(c.head_dim));
+    if (vl) {
+      // one launch for the whole packed batch: per-image token counts come from the
+      // table; v^T blocks share the stride ld_vt[0] (>= every image's tokens)
+      a.varlen = 1;
+      a.vl = *vl;
+      a.B = vl->count;
+      int nmax = 0;
+      for (int b = 0; b < vl->count; ++b) nmax = std::max(nmax, vl->tok_off[b + 1] - vl->tok_off[b]);
+      a.N = nmax;
+      a.ld_vt = vl->ld_vt[0];
+    }
     if ((s = run_attention(a, st))) return s;
   }
   if ((s = run_gemm(gemm_params(ws + pl.o, d, L.o_w, d, L.o_b, x_in, d, x, d, M, d, d, ACT_NONE), st))) return s;
@@ -500,6 +535,111 @@ vt_status vt_forward(vt_handle* h, const float* pixels, const int32_t* grid_thw,
     cudaError_t e = launch_reorder_rows(x, tower_out, B, t, gh, gw, c.hidden, 0, st);
     if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
   }
+  return run_projector(h, x, out, w, pl, st);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validates the grids of a variable-resolution batch and builds its table and plan.
+vt_status build_varlen(const vt_handle* h, int B, const int32_t* grids, VarlenTable* vl, Plan* pl) {
+  if (!grids) return fail(VT_ERR_INVALID_ARG, "grids is NULL");
+  if (B <= 0 || B > kMaxVarlenImages)
+    return fail(VT_ERR_INVALID_ARG, "a variable-resolution batch holds 1 to %d images (got %d)", kMaxVarlenImages, B);
+  const vt_config& c = h->cfg;
+  std::memset(vl, 0, sizeof(*vl));
+  vl->count = B;
+  long long tok = 0, pix = 0;
+  int nmax = 0;
+  for (int b = 0; b < B; ++b) {
+    int t, gh, gw;
+    vt_status s = check_grid(h, 1, grids + 3 * b, &t, &gh, &gw);
+    if (s) return s;
+    const long long n = static_cast<long long>(gh) * gw;
+    vl->tok_off[b] = static_cast<int>(tok);
+    vl->gh[b] = gh;
+    vl->gw[b] = gw;
+    vl->pix_off[b] = pix;
+    nmax = std::max(nmax, static_cast<int>(n));
+    tok += n;
+    pix += 3 * n * c.patch * c.patch;
+    if (tok * c.heads > (1ll << 30)) return fail(VT_ERR_SHAPE, "too many tokens in one call");
+  }
+  vl->tok_off[B] = static_cast<int>(tok);
+  // v^T of every image uses one stride (the largest image's tokens, rounded up to 8) so
+  // that a single attention launch covers the batch; the padding is zeroed per forward.
+  const int ld = round8(nmax);
+  long long vt_elems = 0;
+  for (int b = 0; b < B; ++b) {
+    vl->ld_vt[b] = ld;
+    vl->vt_off[b] = vt_elems;
+    vt_elems += static_cast<long long>(c.heads) * c.head_dim * ld;
+  }
+  *pl = make_plan_core(c, static_cast<int>(tok), static_cast<size_t>(vt_elems));
+  return VT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+vt_status vt_workspace_bytes_varlen(const vt_handle* h, int B, const int32_t* grids, size_t* out) {
+  if (!h || !out) return fail(VT_ERR_INVALID_ARG, "handle and out must not be NULL");
+  VarlenTable vl;
+  Plan pl;
+  vt_status s = build_varlen(h, B, grids, &vl, &pl);
+  if (s) return s;
+  *out = pl.total;
+  return VT_OK;
+}
+
+vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int32_t* grids, int B, void* out,
+                            void* tower_out, void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!pixels || !out || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, out and ws must not be NULL");
+  if (!aligned16(pixels) || !aligned16(out) || !aligned16(ws) || (tower_out && !aligned16(tower_out)))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  VarlenTable vl;
+  Plan pl;
+  if ((s = build_varlen(h, B, grids, &vl, &pl))) return s;
+  if (ws_bytes < pl.total)
+    return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, pl.total);
+  const vt_config& c = h->cfg;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  void* x = w + pl.x;
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  {
+    ProfScope ps(CLS_UNFOLD, 0, pl.M * (4.0 * 3 * c.patch * c.patch + 2.0 * K0), st);
+    cudaError_t e = launch_patch_unfold_varlen(pixels, w + pl.unfold, vl, c.patch, c.temporal_patch, st);
+    if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
+  }
+  if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0,
+                                ACT_NONE),
+                    st)))
+    return s;
+  // The QKV epilogue writes only each image's own v^T columns; the rest of the common
+  // stride must read as zeros in the attention's P.V (P is zero there).
+  {
+    const size_t vt_bytes = static_cast<size_t>(B) * c.heads * c.head_dim * vl.ld_vt[0] * 2;
+    cudaError_t e = cudaMemsetAsync(w + pl.vt, 0, vt_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing v^T padding");
+  }
+  for (int i = 0; i < c.layers; ++i)
+    if ((s = run_layer(h, i, x, x, B, 1, 0, 0, ORDER_BLOCK, w, pl, st, &vl))) return s;
+  if (tower_out) {
+    for (int b = 0; b < B; ++b) {
+      ProfScope ps(CLS_REORDER, 0, 4.0 * (vl.tok_off[b + 1] - vl.tok_off[b]) * c.hidden, st);
+      const size_t off = static_cast<size_t>(vl.tok_off[b]) * c.hidden * 2;
+      cudaError_t e = launch_reorder_rows(static_cast<char*>(x) + off, static_cast<char*>(tower_out) + off, 1, 1,
+                                          vl.gh[b], vl.gw[b], c.hidden, 0, st);
+      if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+    }
+  }
+  // Each image's tokens start at a multiple of 4 and keep their 2x2 groups together,
+  // so the merged [tokens/4, 4P] view spans the whole packed batch.
   return run_projector(h, x, out, w, pl, st);
 }
 

@@ -63,6 +63,8 @@ _SIGS = {
     "vt_forward": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_forward_host": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_forward_host_workspace_bytes": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
+    "vt_workspace_bytes_varlen": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
+    "vt_forward_varlen": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_tower_layer": ([_vp, _i, _vp, _vp, _i32p, _i, _vp, _sz, _vp]),
     "vt_patch_embed": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_merge_project": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
@@ -181,6 +183,25 @@ def vt_workspace_bytes(h: int, B: int, grid_thw) -> int:
 def vt_forward(h, pixels, grid_thw, B, out, tower_out, ws, ws_bytes, stream=None) -> None:
     _check(lib.vt_forward(h, _ptr(pixels), _grid(grid_thw), B, _ptr(out), _ptr(tower_out), _ptr(ws),
                           ws_bytes, _stream(stream)), "vt_forward")
+
+
+def _grids(grids) -> ctypes.Array:
+    flat = [int(v) for g in grids for v in g]
+    return (ctypes.c_int32 * len(flat))(*flat)
+
+
+def vt_workspace_bytes_varlen(h: int, grids) -> int:
+    out = _sz()
+    _check(lib.vt_workspace_bytes_varlen(h, len(grids), _grids(grids), ctypes.byref(out)),
+           "vt_workspace_bytes_varlen")
+    return out.value
+
+
+def vt_forward_varlen(h, pixels, grids, out, tower_out, ws, ws_bytes, stream=None) -> None:
+    """grids: list of (t, h, w) per image; pixels: the images' [3, H, W] fp32 arrays
+    concatenated on the device."""
+    _check(lib.vt_forward_varlen(h, _ptr(pixels), _grids(grids), len(grids), _ptr(out), _ptr(tower_out), _ptr(ws),
+                                 ws_bytes, _stream(stream)), "vt_forward_varlen")
 
 
 def vt_forward_host_workspace_bytes(h: int, B: int, grid_thw) -> int:
