@@ -50,6 +50,7 @@ __all__ = [
     "token_grid", "patch_unfold", "patch_embed", "layer_norm", "gelu",
     "rope_inv_freq", "positions_raster", "apply_rope_3d", "attention",
     "attention_probs", "tower_layer", "tower_layer_rows", "merge_2x2", "projector",
+    "patch_unfold_video", "forward_video",
     "projector_rows", "forward",
     "block_order", "merge_source_map",
 ]
@@ -91,6 +92,27 @@ def patch_unfold(image: np.ndarray, patch: int = 14, temporal_patch: int = 2) ->
             block = image[:, h * patch:(h + 1) * patch, w * patch:(w + 1) * patch]
             clip = np.stack([block] * temporal_patch, axis=1)  # [C, tp, p, p]
             out[h * gw + w] = clip.reshape(-1)
+    return out
+
+
+def patch_unfold_video(frames: np.ndarray, patch: int = 14, temporal_patch: int = 2) -> np.ndarray:
+    """A clip [F, 3, H, W] -> patch vectors [T*gh*gw, 3*tp*patch*patch], raster (t, h, w).
+
+    Temporal patch t covers frames t*tp .. t*tp + tp - 1 (model card, Architecture:
+    temporal patch size 2); a clip whose frame count is not a multiple of tp repeats
+    its last frame, the same rule that makes one image a clip of tp copies of its frame
+    (v2_loaders FINDINGS, section 3).  T = ceil(F / tp).
+    """
+    F, C, H, W = frames.shape
+    T = -(-F // temporal_patch)
+    gh, gw = H // patch, W // patch
+    out = np.empty((T * gh * gw, C * temporal_patch * patch * patch), dtype=np.float64)
+    for t in range(T):
+        idx = [min(t * temporal_patch + tt, F - 1) for tt in range(temporal_patch)]
+        for h in range(gh):
+            for w in range(gw):
+                block = frames[idx][:, :, h * patch:(h + 1) * patch, w * patch:(w + 1) * patch]  # [tp, C, p, p]
+                out[(t * gh + h) * gw + w] = block.transpose(1, 0, 2, 3).reshape(-1)  # (c, t, kh, kw)
     return out
 
 
@@ -324,6 +346,26 @@ def forward(pixels: np.ndarray, w: dict, cfg: dict, keep_layers: bool = False,
         res["layer_in"] = [np.stack(a) for a in lin]
         res["layer_out"] = [np.stack(a) for a in lout]
     return res
+
+
+def forward_video(clips: np.ndarray, w: dict, cfg: dict, layers: int | None = None) -> dict:
+    """Tower + merge + projector for clips [B, F, 3, H, W]: T = ceil(F/tp) temporal
+    patches, all T*gh*gw tokens of a clip attend to each other, RoPE positions
+    (t, h, w), the 2x2 merge within each temporal slice."""
+    p, tp = cfg["patch"], cfg["temporal_patch"]
+    L = cfg["layers"] if layers is None else layers
+    tows, outs = [], []
+    for b in range(clips.shape[0]):
+        clip = clips[b].astype(np.float64)
+        T = -(-clip.shape[0] // tp)
+        gh, gw = clip.shape[2] // p, clip.shape[3] // p
+        pos = positions_raster(T, gh, gw) if cfg.get("use_rope", True) else None
+        x = patch_embed(patch_unfold_video(clip, p, tp), w["embeddings.proj.weight"], w["embeddings.proj.bias"])
+        for i in range(L):
+            x = tower_layer(x, w, i, cfg, pos)
+        tows.append(x)
+        outs.append(projector(x, w, cfg, T, gh, gw))
+    return dict(tower=np.stack(tows), out=np.stack(outs))
 
 
 # ----------------------------------------------------------------- index maps

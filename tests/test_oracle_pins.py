@@ -221,6 +221,50 @@ def test_patch_embed_equals_conv3d(H, W):
     np.testing.assert_allclose(got, ref, atol=1e-12)
 
 
+@pytest.mark.parametrize("F", [1, 2, 3, 4])
+def test_video_patch_embed_equals_conv3d(F):
+    # A clip of F frames: Conv3d with temporal stride 2 over the frames, the last frame
+    # repeated when F is odd (one image = a clip of one frame = its frame twice).
+    r = _rng(40 + F)
+    clip = r.standard_normal((F, 3, 28, 42))
+    wt = r.standard_normal((12, 3, 2, 14, 14)) * 0.02
+    bias = r.standard_normal(12)
+    got = R.patch_embed(R.patch_unfold_video(clip, 14, 2), wt, bias)
+    T = -(-F // 2)
+    padded = np.concatenate([clip, np.repeat(clip[-1:], 2 * T - F, axis=0)], axis=0)  # [2T, 3, H, W]
+    ref = F_conv3d(padded, wt, bias)  # [12, T, gh, gw]
+    np.testing.assert_allclose(got, ref.reshape(12, -1).T, atol=1e-12)
+    if F == 1:
+        np.testing.assert_array_equal(R.patch_unfold_video(clip, 14, 2), R.patch_unfold(clip[0], 14, 2))
+
+
+def F_conv3d(clip, wt, bias):
+    x = torch.tensor(clip).permute(1, 0, 2, 3)[None]  # [1, 3, F, H, W]
+    return F.conv3d(x, torch.tensor(wt), torch.tensor(bias), stride=(2, 14, 14))[0].numpy()
+
+
+def test_video_forward_one_frame_equals_image_forward():
+    cfg = S.get_config("tiny")
+    w = S.weights_f64(S.make_weights(cfg, affine=True))
+    px = S.make_pixels(cfg, batch=1).astype(np.float64)
+    img = R.forward(px, w, cfg)
+    vid = R.forward_video(px[:, None], w, cfg)
+    np.testing.assert_allclose(vid["out"], img["out"], atol=1e-12)
+
+
+def test_video_time_axis_matters_and_merges_within_slices():
+    cfg = S.get_config("tiny", layers=1)
+    w = S.weights_f64(S.make_weights(cfg, affine=True, layers=1))
+    r = _rng(50)
+    clip = r.standard_normal((1, 4, 3, 56, 56))
+    res = R.forward_video(clip, w, cfg)
+    assert res["tower"].shape == (1, 2 * 16, 128) and res["out"].shape == (1, 2 * 4, 256)
+    # swapping the two temporal patches changes the result (RoPE's t block, attention
+    # across time), so the time axis is not ignored
+    swapped = np.concatenate([clip[:, 2:], clip[:, :2]], axis=1)
+    assert abs(R.forward_video(swapped, w, cfg)["out"] - res["out"]).max() > 1e-6
+
+
 def test_patch_unfold_layout():
     img = np.arange(3 * 28 * 42, dtype=np.float64).reshape(3, 28, 42)
     u = R.patch_unfold(img, 14, 2)
