@@ -82,6 +82,13 @@ def workload(name: str) -> dict:
                     tokens=sum(g[1] * g[2] for g in grids),
                     desc="full tower + 2x2 merge + projector on one packed batch of 8 images of mixed sizes "
                          + ", ".join(f"{h}x{w}" for h, w in images))
+    if name.startswith("video"):  # video<side>_f<frames>: 2 clips of that many square frames
+        side, frames = (int(v) for v in name[5:].split("_f"))
+        cfg = dict(S.get_config("tower448"), image=(side, side), batch=2)
+        t, gh, gw = -(-frames // cfg["temporal_patch"]), side // cfg["patch"], side // cfg["patch"]
+        return dict(kind="video", name=name, cfg=cfg, batch=2, frames=frames, grid=(t, gh, gw), tokens=t * gh * gw,
+                    desc=f"full tower + 2x2 merge + projector, 2 clips of {frames} frames of {side}x{side} "
+                         f"({t} temporal patches, {t * gh * gw} tokens per clip)")
     if name.startswith("attn"):
         n = int(name[4:])
         side = int(round(n ** 0.5))
@@ -288,6 +295,20 @@ def run_gpu(args, wl):
         step_flops = sum(tower_flops(cfg, g[1] * g[2])["total"] for g in grids)
         units_per_step = B
         unit = "images/s"
+    elif wl["kind"] == "video":
+        cfg = wl["cfg"]
+        tower = V.Tower(cfg, S.make_weights(cfg))
+        F = wl["frames"]
+        px = torch.from_numpy(S.make_clips(cfg, F, batch=B, seed=REP.replica_seed(cfg["seed"], rank))).to(dev)
+        ws = tower.workspace(B, grid)
+        out = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16, device=dev)
+
+        def launch(s_):
+            V.vt_forward_video(tower.h, px, F, grid, B, out, None, ws, ws.numel(), s_)
+
+        step_flops = B * tower_flops(cfg, N)["total"]
+        units_per_step = B
+        unit = "clips/s"
     else:
         H, D = wl["heads"], wl["D"]
         q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -421,16 +442,18 @@ def run_gpu(args, wl):
             cpu = (oracle_images_per_s(wl["cfg"], args.cpu_budget) if wl["kind"] == "tower"
                    else oracle_attention(wl, args.cpu_budget))
             cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        # tokens of one image (clip); a packed varlen batch reports its mean image
+        per_unit = N / B if wl["kind"] == "varlen" else N
         line = dict(
             metric=METRIC, value=value, unit=unit, n_gpus=world, steps=args.steps, warmup=max(args.warmup, 3),
             ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
             data="synthetic: seeded N(0,0.02) bf16 weights, U[0,1] ImageNet-normalised pixels",
             config=dict(workload=wl["name"], description=wl["desc"], per_gpu_batch=B, global_batch=B * world,
-                        tokens_per_image=N / B, merged_tokens_per_image=(N // 4) / B,
+                        tokens_per_image=per_unit, merged_tokens_per_image=per_unit / 4,
                         l2="flushed (512 MB write) between timed steps", launch="cuda graph" if graph else "eager",
                         parallelism=f"replicas x{world}"),
-            tokens_per_s=value * N / B if wl["kind"] in ("tower", "varlen") else None,
-            output_tokens_per_s=value * (N // 4) / B if wl["kind"] in ("tower", "varlen") else None,
+            tokens_per_s=value * per_unit if wl["kind"] != "attn" else None,
+            output_tokens_per_s=value * per_unit / 4 if wl["kind"] != "attn" else None,
             tflops=world * step_flops * args.steps / (ms / 1000.0) / 1e12,
             roofline=roofline, kernel_classes=classes,
             cpu_baseline=cpu, e2e=e2e,

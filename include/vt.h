@@ -50,7 +50,7 @@ extern "C" {
 typedef enum vt_status {
   VT_OK = 0,
   VT_ERR_INVALID_ARG = 1, /* null pointer, non-positive or inconsistent size, misalignment */
-  VT_ERR_SHAPE = 2,       /* image side not a multiple of patch*merge, t != 1, grid too large */
+  VT_ERR_SHAPE = 2,       /* image side not a multiple of patch*merge, wrong t, grid too large */
   VT_ERR_NOT_LOADED = 3,  /* forward before a complete vt_load_weights */
   VT_ERR_WEIGHT = 4,      /* missing, duplicate, unknown or wrong-shape weight */
   VT_ERR_WORKSPACE = 5,   /* workspace smaller than vt_workspace_bytes() */
@@ -121,14 +121,15 @@ VT_API vt_status vt_destroy(vt_handle* h);
  * Synchronous.  Errors: VT_ERR_WEIGHT names the offending tensor in vt_last_error(). */
 VT_API vt_status vt_load_weights(vt_handle* h, const vt_weight* w, int n);
 
-/* Bytes of caller workspace vt_forward / vt_tower_layer / vt_merge_project need for B
- * images of grid grid_thw (host int32[3] = t, h, w in patches).  Affine in B*t*h*w:
- * no term grows with the square of the sequence.  Host only. */
+/* Bytes of caller workspace vt_forward / vt_forward_video / vt_tower_layer /
+ * vt_merge_project need for B images or clips of grid grid_thw (host int32[3] = t, h, w
+ * in patches, t <= 4096).  Affine in B*t*h*w: no term grows with the square of the
+ * sequence.  Host only. */
 VT_API vt_status vt_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out);
 
 /* Full forward: patch unfold -> patch embedding -> layers -> 2x2 merge -> projector.
  *   pixels    device fp32 [B, 3, H, W], already normalised, H = grid_h*patch, W = grid_w*patch
- *   grid_thw  host int32[3]; t must be 1; h and w even and at most 4096
+ *   grid_thw  host int32[3]; t must be 1 (clips: vt_forward_video); h and w even, <= 4096
  *   out       device bf16 [B, t*h*w/4, proj_out], merged tokens in raster (i, j) order
  *   tower_out device bf16 [B, t*h*w, hidden] in raster order, or NULL
  *   ws        device workspace of at least vt_workspace_bytes(h, B, grid_thw) bytes
@@ -145,6 +146,23 @@ VT_API vt_status vt_forward(vt_handle* h, const float* pixels, const int32_t* gr
 VT_API vt_status vt_forward_host(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B,
                           void* out_host, void* ws, size_t ws_bytes, void* stream);
 VT_API vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out);
+
+/* Video: B clips of `frames` frames each, all frames of one size.
+ *   clips     device fp32 [B, frames, 3, H, W], already normalised
+ *   frames    >= 1; temporal patch t takes frames t*tp .. t*tp+tp-1 (tp = the config's
+ *             temporal_patch), the last frame repeated when frames is not a multiple of
+ *             tp, so frames = 1 is vt_forward's still image
+ *   grid_thw  host int32[3]; t must equal ceil(frames / tp); h and w as for vt_forward
+ *   out       device bf16 [B, t*h*w/4, proj_out]: merged tokens in (t, i, j) raster order,
+ *             the 2x2 merge within each temporal slice
+ *   tower_out device bf16 [B, t*h*w, hidden] in (t, h, w) raster order, or NULL
+ *   ws        device workspace of at least vt_workspace_bytes(h, B, grid_thw) bytes
+ * All t*h*w tokens of a clip attend to each other; RoPE rotates by (t, h, w).  Errors:
+ * VT_ERR_SHAPE when t does not match frames, as for vt_forward otherwise.  Source:
+ * "MiniMax-M3 Vision" model card, Architecture table (Conv3d patch embed, temporal patch
+ * size 2, 3D RoPE); the frame-repeat rule of the "v2_loaders" findings, section 3. */
+VT_API vt_status vt_forward_video(vt_handle* h, const float* clips, int frames, const int32_t* grid_thw, int B,
+                                  void* out, void* tower_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Variable-resolution batch: B images (1 <= B <= 64) of different patch grids in one
  * call, their tokens packed into one sequence; attention stays within each image.
@@ -169,7 +187,8 @@ VT_API vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int3
 VT_API vt_status vt_tower_layer(vt_handle* h, int layer, const void* x_in, void* x_out, const int32_t* grid_thw,
                          int B, void* ws, size_t ws_bytes, void* stream);
 
-/* Patch embedding alone: x = Conv3d(pixels) as [B, t*h*w, hidden] bf16, raster order. */
+/* Patch embedding alone for still images (t = 1): x = Conv3d(pixels) as [B, h*w, hidden]
+ * bf16, raster order. */
 VT_API vt_status vt_patch_embed(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* x_out,
                          void* ws, size_t ws_bytes, void* stream);
 

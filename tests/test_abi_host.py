@@ -58,7 +58,7 @@ def test_forward_before_load_and_grid_errors():
     with pytest.raises(V.VtError) as e:
         V.vt_forward(h, 16, (1, 8, 8), 1, 16, None, 16, 1 << 20)
     assert _status(e) == "VT_ERR_NOT_LOADED"
-    for grid, code in [((1, 7, 8), "VT_ERR_SHAPE"), ((2, 8, 8), "VT_ERR_SHAPE"),
+    for grid, code in [((1, 7, 8), "VT_ERR_SHAPE"), ((4097, 8, 8), "VT_ERR_SHAPE"),
                        ((1, 8, 8194), "VT_ERR_SHAPE"), ((0, 8, 8), "VT_ERR_INVALID_ARG")]:
         with pytest.raises(V.VtError) as e:
             V.vt_workspace_bytes(h, 1, grid)
@@ -141,11 +141,29 @@ def test_varlen_workspace_and_argument_checks():
     with pytest.raises(V.VtError) as e:
         V.vt_workspace_bytes_varlen(h, [(1, 32, 32), (1, 15, 24)])
     assert _status(e) == "VT_ERR_SHAPE"
+    with pytest.raises(V.VtError) as e:  # clips go through vt_forward_video
+        V.vt_workspace_bytes_varlen(h, [(1, 32, 32), (2, 16, 24)])
+    assert _status(e) == "VT_ERR_SHAPE"
     with pytest.raises(V.VtError) as e:
         V.vt_workspace_bytes_varlen(h, [(1, 2, 2)] * 65)
     assert _status(e) == "VT_ERR_INVALID_ARG"
     with pytest.raises(V.VtError) as e:
         V.vt_forward_varlen(h, 16, [(1, 2, 2)], 16, None, 16, 1 << 20)
+    assert _status(e) == "VT_ERR_NOT_LOADED"
+    V.vt_destroy(h)
+
+
+def test_video_workspace_counts_every_temporal_patch():
+    """A clip of grid (t, h, w) is one sequence of t*h*w tokens: its plan equals a still
+    image of the same token count, and the still-image entry points refuse t > 1."""
+    h = V.vt_create(S.get_config("tower448"))
+    for t, gh, gw in [(2, 8, 8), (3, 16, 24), (8, 32, 32)]:
+        assert V.vt_workspace_bytes(h, 2, (t, gh, gw)) == V.vt_workspace_bytes(h, 2, (1, gh, t * gw))
+    with pytest.raises(V.VtError) as e:
+        V.vt_forward_host_workspace_bytes(h, 1, (2, 8, 8))
+    assert _status(e) == "VT_ERR_SHAPE"
+    with pytest.raises(V.VtError) as e:
+        V.vt_forward_video(h, 16, 4, (2, 8, 8), 1, 16, None, 16, 1 << 20)
     assert _status(e) == "VT_ERR_NOT_LOADED"
     V.vt_destroy(h)
 

@@ -147,14 +147,16 @@ __global__ void __launch_bounds__(256) layernorm_block(const bf16* __restrict__ 
 }
 
 // -------------------------------------------------------------- patch unfold
-// One image's 14x14 patches, the frame repeated tp times ("v2_loaders" findings,
-// section 3: temporal dimension padded to 2 by repeating the frame), flattened in
-// (c, t, kh, kw) order to match a Conv3d weight [hidden, 3, tp, p, p].  One block per
-// token; the fp32 pixel is rounded to bf16 (nearest even).
+// Patch vectors of clips of F frames [B, F, 3, H, W], flattened in (c, t, kh, kw) order
+// to match a Conv3d weight [hidden, 3, tp, p, p].  Temporal patch t covers frames
+// t*tp .. t*tp+tp-1, the last frame repeated when F is not a multiple of tp; a still
+// image is the clip F = 1, its frame repeated tp times ("v2_loaders" findings, section 3:
+// temporal dimension padded to 2 by repeating the frame).  One block per token; the
+// fp32 pixel is rounded to bf16 (nearest even).
 __global__ void __launch_bounds__(256) patch_unfold_kernel(const float* __restrict__ px, bf16* __restrict__ out,
-                                                           int H, int W, int patch, int tp, int gh, int gw,
-                                                           int order) {
-  const int ntok = gh * gw;
+                                                           int F, int H, int W, int patch, int tp, int gt, int gh,
+                                                           int gw, int order) {
+  const int ntok = gt * gh * gw;
   const int row = blockIdx.x;
   const int b = row / ntok, n = row - (row / ntok) * ntok;
   int t, hh, ww;
@@ -162,12 +164,15 @@ __global__ void __launch_bounds__(256) patch_unfold_kernel(const float* __restri
   const int pp = patch * patch;
   const int K = 3 * tp * pp;
   bf16* dst = out + static_cast<size_t>(row) * K;
-  const float* img = px + static_cast<size_t>(b) * 3 * H * W;
+  const float* clip = px + static_cast<size_t>(b) * F * 3 * H * W;
   for (int e = threadIdx.x; e < 3 * pp; e += blockDim.x) {
     const int c = e / pp, rem = e - c * pp;
     const int kh = rem / patch, kw = rem - kh * patch;
-    const bf16 v = __float2bfloat16_rn(img[(static_cast<size_t>(c) * H + hh * patch + kh) * W + ww * patch + kw]);
-    for (int f = 0; f < tp; ++f) dst[c * tp * pp + f * pp + rem] = v;
+    const size_t pix = (static_cast<size_t>(c) * H + hh * patch + kh) * W + ww * patch + kw;
+    for (int f = 0; f < tp; ++f) {
+      const int frame = min(t * tp + f, F - 1);
+      dst[c * tp * pp + f * pp + rem] = __float2bfloat16_rn(clip[static_cast<size_t>(frame) * 3 * H * W + pix]);
+    }
   }
 }
 
@@ -302,11 +307,16 @@ cudaError_t launch_layernorm(const void* x, const void* gamma, const void* beta,
 
 cudaError_t launch_patch_unfold(const float* pixels, void* out, int B, int H, int W, int patch, int tp, int order,
                                 cudaStream_t stream) {
-  const int gh = H / patch, gw = W / patch;
-  const long rows = static_cast<long>(B) * gh * gw;
+  return launch_patch_unfold_frames(pixels, out, B, 1, H, W, patch, tp, order, stream);
+}
+
+cudaError_t launch_patch_unfold_frames(const float* pixels, void* out, int B, int F, int H, int W, int patch, int tp,
+                                       int order, cudaStream_t stream) {
+  const int gh = H / patch, gw = W / patch, gt = (F + tp - 1) / tp;
+  const long rows = static_cast<long>(B) * gt * gh * gw;
   if (rows <= 0) return cudaSuccess;
-  patch_unfold_kernel<<<static_cast<unsigned>(rows), 256, 0, stream>>>(pixels, static_cast<bf16*>(out), H, W, patch,
-                                                                       tp, gh, gw, order);
+  patch_unfold_kernel<<<static_cast<unsigned>(rows), 256, 0, stream>>>(pixels, static_cast<bf16*>(out), F, H, W,
+                                                                       patch, tp, gt, gh, gw, order);
   return cudaGetLastError();
 }
 

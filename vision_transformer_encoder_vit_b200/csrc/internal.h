@@ -126,6 +126,10 @@ cudaError_t launch_layernorm(const void* x, const void* gamma, const void* beta,
 // pixels [B, 3, H, W] fp32 -> patch vectors [B * gh * gw, 3 * tp * p * p] bf16 in `order`.
 cudaError_t launch_patch_unfold(const float* pixels, void* out, int B, int H, int W, int patch, int tp,
                                 int order, cudaStream_t stream);
+// Clips [B, F, 3, H, W] -> [B * ceil(F/tp) * gh * gw, 3 * tp * p * p]; temporal patch t
+// takes frames t*tp .. t*tp+tp-1, the last frame repeated past the end of the clip.
+cudaError_t launch_patch_unfold_frames(const float* pixels, void* out, int B, int F, int H, int W, int patch,
+                                       int tp, int order, cudaStream_t stream);
 // Packed images of different sizes (vl.pix_off, vl.gh, vl.gw) -> packed patch vectors
 // in 2x2-block order per image.
 cudaError_t launch_patch_unfold_varlen(const float* pixels, void* out, const VarlenTable& vl, int patch, int tp,

@@ -240,13 +240,20 @@ vt_status check_grid(const vt_handle* h, int B, const int32_t* g, int* t, int* g
   *gh = g[1];
   *gw = g[2];
   if (*t <= 0 || *gh <= 0 || *gw <= 0) return fail(VT_ERR_INVALID_ARG, "grid_thw must be positive");
-  if (*t != 1) return fail(VT_ERR_SHAPE, "only t = 1 (still images) is supported, got t = %d", *t);
+  if (*t > kRopeMaxPos) return fail(VT_ERR_SHAPE, "t = %d above %d temporal patches", *t, kRopeMaxPos);
   if ((*gh % h->cfg.merge) || (*gw % h->cfg.merge))
     return fail(VT_ERR_SHAPE, "grid %dx%d is not a multiple of the %dx%d merge", *gh, *gw, h->cfg.merge, h->cfg.merge);
   if (*gh > kRopeMaxPos || *gw > kRopeMaxPos)
     return fail(VT_ERR_SHAPE, "grid side above %d patches", kRopeMaxPos);
   const long long M = static_cast<long long>(B) * (*t) * (*gh) * (*gw);
   if (M > (1ll << 30)) return fail(VT_ERR_SHAPE, "too many tokens in one call (%lld)", M);
+  return VT_OK;
+}
+
+// Entry points whose pixels are still images [B, 3, H, W] take grids with t = 1 only.
+vt_status check_still(int t, const char* entry) {
+  if (t != 1)
+    return fail(VT_ERR_SHAPE, "%s takes still images (t = 1), got t = %d; clips go through vt_forward_video", entry, t);
   return VT_OK;
 }
 
@@ -501,27 +508,23 @@ vt_status vt_load_weights(vt_handle* h, const vt_weight* w, int n) {
   return VT_OK;
 }
 
-vt_status vt_forward(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* out, void* tower_out,
-                     void* ws, size_t ws_bytes, void* stream) {
-  vt_status s = check_loaded(h);
-  if (s) return s;
-  if (!pixels || !out || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, out and ws must not be NULL");
-  if (!aligned16(pixels) || !aligned16(out) || !aligned16(ws) || (tower_out && !aligned16(tower_out)))
-    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
-  int t, gh, gw;
-  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+// Forward of B clips of F frames [B, F, 3, H, W] with grid (t, gh, gw), t = ceil(F / tp)
+// (a still image is F = 1, t = 1).  Arguments are checked by the callers.
+static vt_status forward_clips(vt_handle* h, const float* pixels, int F, int B, int t, int gh, int gw, void* out,
+                               void* tower_out, void* ws, size_t ws_bytes, cudaStream_t st) {
   const vt_config& c = h->cfg;
   const Plan pl = make_plan(c, B, t, gh, gw);
   if (ws_bytes < pl.total)
     return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, pl.total);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  vt_status s;
   char* w = static_cast<char*>(ws);
   void* x = w + pl.x;
   const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
   {
-    ProfScope ps(CLS_UNFOLD, 0, pl.M * (4.0 * 3 * c.patch * c.patch + 2.0 * K0), st);
-    cudaError_t e = launch_patch_unfold(pixels, w + pl.unfold, B, gh * c.patch, gw * c.patch, c.patch,
-                                        c.temporal_patch, ORDER_BLOCK, st);
+    const double px_bytes = 4.0 * B * F * 3.0 * (gh * c.patch) * (gw * c.patch);
+    ProfScope ps(CLS_UNFOLD, 0, px_bytes + 2.0 * pl.M * K0, st);
+    cudaError_t e = launch_patch_unfold_frames(pixels, w + pl.unfold, B, F, gh * c.patch, gw * c.patch, c.patch,
+                                               c.temporal_patch, ORDER_BLOCK, st);
     if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
   }
   if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0,
@@ -536,6 +539,40 @@ vt_status vt_forward(vt_handle* h, const float* pixels, const int32_t* grid_thw,
     if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
   }
   return run_projector(h, x, out, w, pl, st);
+}
+
+static vt_status check_forward_ptrs(const float* pixels, const void* out, const void* tower_out, const void* ws) {
+  if (!pixels || !out || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, out and ws must not be NULL");
+  if (!aligned16(pixels) || !aligned16(out) || !aligned16(ws) || (tower_out && !aligned16(tower_out)))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return VT_OK;
+}
+
+vt_status vt_forward(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* out, void* tower_out,
+                     void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if ((s = check_forward_ptrs(pixels, out, tower_out, ws))) return s;
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  if ((s = check_still(t, "vt_forward"))) return s;
+  return forward_clips(h, pixels, 1, B, t, gh, gw, out, tower_out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+vt_status vt_forward_video(vt_handle* h, const float* clips, int frames, const int32_t* grid_thw, int B, void* out,
+                           void* tower_out, void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if ((s = check_forward_ptrs(clips, out, tower_out, ws))) return s;
+  if (frames <= 0) return fail(VT_ERR_INVALID_ARG, "a clip needs at least one frame (got %d)", frames);
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  const int tp = h->cfg.temporal_patch;
+  if (t != (frames + tp - 1) / tp)
+    return fail(VT_ERR_SHAPE, "grid t = %d does not match %d frames at temporal patch %d (expected %d)", t, frames,
+                tp, (frames + tp - 1) / tp);
+  return forward_clips(h, clips, frames, B, t, gh, gw, out, tower_out, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -556,6 +593,7 @@ vt_status build_varlen(const vt_handle* h, int B, const int32_t* grids, VarlenTa
     int t, gh, gw;
     vt_status s = check_grid(h, 1, grids + 3 * b, &t, &gh, &gw);
     if (s) return s;
+    if ((s = check_still(t, "vt_forward_varlen"))) return s;
     const long long n = static_cast<long long>(gh) * gw;
     vl->tok_off[b] = static_cast<int>(tok);
     vl->gh[b] = gh;
@@ -647,6 +685,7 @@ vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, const int32
   size_t base;
   vt_status s = vt_workspace_bytes(h, B, grid_thw, &base);
   if (s) return s;
+  if ((s = check_still(grid_thw[0], "vt_forward_host"))) return s;
   const vt_config& c = h->cfg;
   const size_t N = static_cast<size_t>(grid_thw[0]) * grid_thw[1] * grid_thw[2];
   const size_t px = static_cast<size_t>(B) * 3 * N * c.patch * c.patch * 4;
@@ -704,6 +743,7 @@ vt_status vt_patch_embed(vt_handle* h, const float* pixels, const int32_t* grid_
   if (!pixels || !x_out || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, x_out and ws must not be NULL");
   int t, gh, gw;
   if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  if ((s = check_still(t, "vt_patch_embed"))) return s;
   const vt_config& c = h->cfg;
   const Plan pl = make_plan(c, B, t, gh, gw);
   if (ws_bytes < pl.total) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, pl.total);

@@ -171,6 +171,15 @@ def make_pixels(cfg: dict, batch: int | None = None, seed: int | None = None,
     return np.ascontiguousarray(x, dtype=np.float32)
 
 
+def make_clips(cfg: dict, frames: int, batch: int | None = None, seed: int | None = None) -> np.ndarray:
+    """Clips of ``frames`` ImageNet-normalised U[0,1] frames, float32 [B, F, 3, H, W];
+    the frames are independent draws (no motion model: every frame differs)."""
+    seed = cfg["seed"] if seed is None else seed
+    B = cfg["batch"] if batch is None else batch
+    flat = make_pixels(cfg, batch=B * frames, seed=seed)
+    return np.ascontiguousarray(flat.reshape(B, frames, *flat.shape[1:]))
+
+
 def make_activations(rows: int, cols: int, seed: int) -> np.ndarray:
     """bf16 bits of N(0,1) activations [rows, cols]."""
     rng = np.random.default_rng(seed + 2000)

@@ -65,6 +65,7 @@ _SIGS = {
     "vt_forward_host_workspace_bytes": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
     "vt_workspace_bytes_varlen": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
     "vt_forward_varlen": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
+    "vt_forward_video": ([_vp, _vp, _i, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_tower_layer": ([_vp, _i, _vp, _vp, _i32p, _i, _vp, _sz, _vp]),
     "vt_patch_embed": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_merge_project": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
@@ -183,6 +184,12 @@ def vt_workspace_bytes(h: int, B: int, grid_thw) -> int:
 def vt_forward(h, pixels, grid_thw, B, out, tower_out, ws, ws_bytes, stream=None) -> None:
     _check(lib.vt_forward(h, _ptr(pixels), _grid(grid_thw), B, _ptr(out), _ptr(tower_out), _ptr(ws),
                           ws_bytes, _stream(stream)), "vt_forward")
+
+
+def vt_forward_video(h, clips, frames, grid_thw, B, out, tower_out, ws, ws_bytes, stream=None) -> None:
+    """clips: device fp32 [B, frames, 3, H, W]; grid_thw = (ceil(frames / tp), H/p, W/p)."""
+    _check(lib.vt_forward_video(h, _ptr(clips), frames, _grid(grid_thw), B, _ptr(out), _ptr(tower_out), _ptr(ws),
+                                ws_bytes, _stream(stream)), "vt_forward_video")
 
 
 def _grids(grids) -> ctypes.Array:
