@@ -37,6 +37,12 @@ tests/test_oracle_pins.py):
   * 2x2 merge: merged token (i, j) concatenates tokens (2i,2j), (2i,2j+1), (2i+1,2j),
     (2i+1,2j+1) in that order; merged tokens are in raster (i, j) order.
   * Images of a batch are independent (attention never crosses images).
+  * Preprocessing ("bicubic resize to 672x672, OpenAI CLIP mean/std", findings section
+    3): the resize is separable cubic-convolution resampling with the Keys kernel at
+    a = -0.5, output pixel centres mapped onto input pixel centres, the kernel widened
+    by the scale factor when shrinking, taps outside the image dropped and the weights
+    renormalised; resized values stay real numbers (no clamping or rounding to 8 bits)
+    before scaling by 1/255 and normalising per channel.
 
 Parity with the real MiniMax-M3 weights is not checked here (no trained weights or
 reference outputs exist on the pages); every function below is pinned against
@@ -51,6 +57,7 @@ __all__ = [
     "rope_inv_freq", "positions_raster", "apply_rope_3d", "attention",
     "attention_probs", "tower_layer", "tower_layer_rows", "merge_2x2", "projector",
     "patch_unfold_video", "forward_video",
+    "cubic_kernel", "resize_taps", "resize_bicubic", "preprocess",
     "projector_rows", "forward",
     "block_order", "merge_source_map",
 ]
@@ -120,6 +127,64 @@ def patch_embed(patches: np.ndarray, weight: np.ndarray, bias: np.ndarray) -> np
     """Conv3d with kernel = stride = (tp, p, p) as a matrix product (model card,
     Architecture: Conv3d patch embed).  weight is [hidden, 3, tp, p, p]."""
     return patches @ weight.reshape(weight.shape[0], -1).T + bias
+
+
+# -------------------------------------------------------------- preprocessing
+
+def cubic_kernel(x: float, a: float = -0.5) -> float:
+    """Keys' cubic convolution kernel: 1 at 0, 0 at every other integer, support |x| < 2
+    (findings section 3 names a bicubic resize; a = -0.5 is the reading)."""
+    x = abs(x)
+    if x <= 1.0:
+        return ((a + 2.0) * x - (a + 3.0)) * x * x + 1.0
+    if x < 2.0:
+        return (((x - 5.0) * x + 8.0) * x - 4.0) * a
+    return 0.0
+
+
+def resize_taps(n_in: int, n_out: int) -> list[tuple[int, np.ndarray]]:
+    """For each output index i along one axis: (first input index, weights summing to 1).
+
+    Output pixel i has its centre at input coordinate c = (i + 1/2) * n_in / n_out (pixel
+    centres at half-integers).  When shrinking (n_in > n_out) the kernel is stretched by
+    the scale so every input pixel contributes (antialiasing); input pixels j with
+    |j + 1/2 - c| inside the support get weight cubic_kernel((j + 1/2 - c) / stretch),
+    pixels outside the image are left out and the weights are divided by their sum.
+    """
+    scale = n_in / n_out
+    stretch = max(scale, 1.0)
+    support = 2.0 * stretch
+    taps = []
+    for i in range(n_out):
+        c = (i + 0.5) * scale
+        lo = max(int(c - support + 0.5), 0)
+        hi = min(int(c + support + 0.5), n_in)
+        w = np.array([cubic_kernel((j + 0.5 - c) / stretch) for j in range(lo, hi)], dtype=np.float64)
+        taps.append((lo, w / w.sum()))
+    return taps
+
+
+def resize_bicubic(img: np.ndarray, out_h: int, out_w: int) -> np.ndarray:
+    """An image [H, W, C] resampled to [out_h, out_w, C]: the 1D resampling of
+    resize_taps along the width, then along the height (the two commute)."""
+    H, W, C = img.shape
+    src = img.astype(np.float64)
+    tmp = np.empty((H, out_w, C), dtype=np.float64)
+    for i, (lo, w) in enumerate(resize_taps(W, out_w)):
+        tmp[:, i, :] = np.tensordot(w, src[:, lo:lo + len(w), :], axes=([0], [1]))
+    out = np.empty((out_h, out_w, C), dtype=np.float64)
+    for i, (lo, w) in enumerate(resize_taps(H, out_h)):
+        out[i] = np.tensordot(w, tmp[lo:lo + len(w)], axes=([0], [0]))
+    return out
+
+
+def preprocess(img_u8: np.ndarray, out_h: int, out_w: int, mean, std) -> np.ndarray:
+    """A decoded RGB image [H, W, 3] of 8-bit values -> model pixels [3, out_h, out_w]:
+    bicubic resize, scale by 1/255, subtract the channel mean, divide by the channel
+    standard deviation (findings section 3: bicubic resize, CLIP mean/std)."""
+    x = resize_bicubic(img_u8, out_h, out_w) / 255.0
+    x = (x - np.asarray(mean, np.float64)) / np.asarray(std, np.float64)
+    return np.ascontiguousarray(x.transpose(2, 0, 1))
 
 
 # ------------------------------------------------------- normalisation, GELU

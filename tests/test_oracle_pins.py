@@ -437,3 +437,59 @@ def test_row_sampled_layer_and_projector_equal_full():
     mrows = np.array([0, 5, 15])
     np.testing.assert_allclose(R.projector_rows(x, w, cfg, 1, 8, 8, mrows),
                                R.projector(x, w, cfg, 1, 8, 8)[mrows], atol=1e-12)
+
+
+# -------------------------------------------------------------- preprocessing
+
+def test_cubic_kernel_values_and_partition_of_unity():
+    # Keys' kernel at a = -0.5, by hand: (a+2)|x|^3 - (a+3)|x|^2 + 1 on [0, 1],
+    # a|x|^3 - 5a|x|^2 + 8a|x| - 4a on [1, 2)
+    assert R.cubic_kernel(0.0) == 1.0
+    for x in (1.0, -1.0, 2.0, -2.0, 2.5):
+        assert R.cubic_kernel(x) == 0.0
+    assert R.cubic_kernel(0.5) == pytest.approx(0.5625, abs=1e-15)
+    assert R.cubic_kernel(-1.5) == pytest.approx(-0.0625, abs=1e-15)
+    assert R.cubic_kernel(0.25) == pytest.approx(1.5 * 0.25 ** 3 - 2.5 * 0.25 ** 2 + 1, abs=1e-15)
+    for x in _rng(40).uniform(0, 1, 7):  # the four taps around any point sum to 1
+        assert sum(R.cubic_kernel(x + k) for k in (-2, -1, 0, 1)) == pytest.approx(1.0, abs=1e-14)
+
+
+@pytest.mark.parametrize("src,dst", [((20, 30), (28, 42)), ((97, 61), (28, 28)), ((40, 13), (14, 56)),
+                                     ((448, 336), (112, 84)), ((28, 28), (28, 28)), ((9, 300), (42, 14))])
+def test_resize_equals_torch_antialiased_bicubic(src, dst):
+    # torch's antialiased bicubic is an independent implementation of the same
+    # resampling (a = -0.5, stretched kernel when shrinking, renormalised edge taps)
+    img = _rng(41).uniform(0, 255, size=(*src, 3))
+    got = R.resize_bicubic(img, *dst)
+    ref = F.interpolate(torch.tensor(img).permute(2, 0, 1)[None], size=dst, mode="bicubic", antialias=True,
+                        align_corners=False)[0].permute(1, 2, 0).numpy()
+    np.testing.assert_allclose(got, ref, atol=1e-10)
+
+
+def test_resize_identity_constant_and_linear():
+    r = _rng(42)
+    img = r.uniform(0, 255, size=(17, 23, 3))
+    np.testing.assert_array_equal(R.resize_bicubic(img, 17, 23), img)  # same size: exact copy
+    flat = np.full((31, 19, 3), 77.0)
+    np.testing.assert_allclose(R.resize_bicubic(flat, 14, 42), 77.0, atol=1e-12)
+    # upscaling reproduces a linear ramp away from the borders (cubic convolution is exact
+    # on polynomials of degree < 3 when no tap is dropped)
+    ramp = np.broadcast_to(np.arange(40.0)[None, :, None] * 3.0 + 5.0, (6, 40, 3)).copy()
+    out = R.resize_bicubic(ramp, 6, 100)
+    centres = (np.arange(100) + 0.5) * 40 / 100 - 0.5
+    np.testing.assert_allclose(out[:, 5:-5, 0], np.broadcast_to(centres[5:-5] * 3.0 + 5.0, (6, 90)), atol=1e-10)
+
+
+def test_preprocess_channel_order_and_statistics():
+    img = np.zeros((14, 28, 3), dtype=np.uint8)
+    img[..., 0], img[..., 1], img[..., 2] = 10, 128, 250
+    out = R.preprocess(img, 28, 14, S.CLIP_MEAN, S.CLIP_STD)
+    assert out.shape == (3, 28, 14)
+    for c, v in enumerate((10, 128, 250)):
+        np.testing.assert_allclose(out[c], (v / 255 - S.CLIP_MEAN[c]) / S.CLIP_STD[c], atol=1e-12)
+    # a non-constant image: preprocess = normalise(torch resize) channel by channel
+    img = S.make_images_u8([(50, 70)], seed=1)[0]
+    ref = F.interpolate(torch.tensor(img, dtype=torch.float64).permute(2, 0, 1)[None], size=(28, 42),
+                        mode="bicubic", antialias=True, align_corners=False)[0].numpy()
+    ref = (ref / 255 - np.asarray(S.CLIP_MEAN)[:, None, None]) / np.asarray(S.CLIP_STD)[:, None, None]
+    np.testing.assert_allclose(R.preprocess(img, 28, 42, S.CLIP_MEAN, S.CLIP_STD), ref, atol=1e-10)

@@ -19,6 +19,9 @@ import numpy as np
 # values the tower consumes.
 IMAGENET_MEAN = (0.485, 0.456, 0.406)
 IMAGENET_STD = (0.229, 0.224, 0.225)
+# OpenAI CLIP image statistics (the "OpenAI CLIP mean/std" the preprocessing names).
+CLIP_MEAN = (0.48145466, 0.4578275, 0.40821073)
+CLIP_STD = (0.26862954, 0.26130258, 0.27577711)
 
 _TOWER_BASE = dict(
     patch=14, temporal_patch=2, merge=2, rope_theta=10000.0, ln_eps=1e-6,
@@ -169,6 +172,25 @@ def make_pixels(cfg: dict, batch: int | None = None, seed: int | None = None,
         std = np.asarray(IMAGENET_STD, np.float32)[None, :, None, None]
         x = (x - mean) / std
     return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def make_images_u8(sizes, seed: int = 0) -> list[np.ndarray]:
+    """Decoded RGB images of the given (H, W) sizes as uint8 [H, W, 3]: a smooth random
+    field (sum of low-frequency waves) plus uniform noise, clipped to 0..255, so both
+    flat areas and edges occur."""
+    rng = np.random.default_rng(seed + 2000)
+    out = []
+    for H, W in sizes:
+        y = np.linspace(0.0, 1.0, H)[:, None, None]
+        x = np.linspace(0.0, 1.0, W)[None, :, None]
+        img = np.full((H, W, 3), 128.0)
+        for _ in range(4):
+            fy, fx = rng.uniform(0.5, 6.0, size=2)
+            ph = rng.uniform(0, 2 * np.pi, size=3)[None, None, :]
+            img += rng.uniform(20, 50) * np.sin(2 * np.pi * (fy * y + fx * x) + ph)
+        img += rng.uniform(-40, 40, size=(H, W, 3))
+        out.append(np.clip(np.rint(img), 0, 255).astype(np.uint8))
+    return out
 
 
 def make_clips(cfg: dict, frames: int, batch: int | None = None, seed: int | None = None) -> np.ndarray:
