@@ -82,6 +82,14 @@ def workload(name: str) -> dict:
                     tokens=sum(g[1] * g[2] for g in grids),
                     desc="full tower + 2x2 merge + projector on one packed batch of 8 images of mixed sizes "
                          + ", ".join(f"{h}x{w}" for h, w in images))
+    if name == "u8_672":
+        cfg = dict(S.get_config("tower448"), image=(672, 672))
+        sizes = [(1080, 1920), (768, 1024), (480, 640), (3024, 4032), (1200, 1600), (720, 1280), (2000, 3000),
+                 (512, 512)]
+        return dict(kind="u8", name=name, cfg=cfg, batch=len(sizes), sizes=sizes, grid=(1, 48, 48), tokens=48 * 48,
+                    desc="decoded 8-bit images of 8 photo sizes (" + ", ".join(f"{h}x{w}" for h, w in sizes)
+                         + ") resized on the GPU to 672x672 (bicubic, CLIP normalisation) + full tower + 2x2 merge"
+                         " + projector")
     if name.startswith("video"):  # video<side>_f<frames>: 2 clips of that many square frames
         side, frames = (int(v) for v in name[5:].split("_f"))
         cfg = dict(S.get_config("tower448"), image=(side, side), batch=2)
@@ -295,6 +303,22 @@ def run_gpu(args, wl):
         step_flops = sum(tower_flops(cfg, g[1] * g[2])["total"] for g in grids)
         units_per_step = B
         unit = "images/s"
+    elif wl["kind"] == "u8":
+        cfg = wl["cfg"]
+        tower = V.Tower(cfg, S.make_weights(cfg))
+        images = S.make_images_u8(wl["sizes"], seed=REP.replica_seed(cfg["seed"], rank))
+        img_host = torch.from_numpy(np.concatenate([im.ravel() for im in images])).pin_memory()
+        img = img_host.to(dev)
+        sizes = wl["sizes"]
+        ws = tower.workspace(B, grid)
+        out = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16, device=dev)
+
+        def launch(s_):
+            V.vt_forward_u8(tower.h, img, sizes, grid, out, None, ws, ws.numel(), stream=s_)
+
+        step_flops = B * tower_flops(cfg, N)["total"]
+        units_per_step = B
+        unit = "images/s"
     elif wl["kind"] == "video":
         cfg = wl["cfg"]
         tower = V.Tower(cfg, S.make_weights(cfg))
@@ -416,6 +440,30 @@ def run_gpu(args, wl):
                    h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h.numel() * 2),
                    api="vt_forward_host")
         del ws_h
+    elif wl["kind"] == "u8":
+        # decoded images from pinned host memory -> device, forward, projected tokens back
+        out_h = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            img.copy_(img_host, non_blocking=True)
+            launch(stream)
+            out_h.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        e_s.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = REP.max_over_ranks(e_s.elapsed_time(e_e), dev)
+        e2e = dict(value=REP.job_throughput(B, args.steps, e2e_ms, world), unit=unit,
+                   h2d_bytes_per_step=int(img_host.numel()), d2h_bytes_per_step=int(out_h.numel() * 2),
+                   api="vt_forward_u8 (+ host copies)")
 
     if rank == 0:
         # dominant kernel class by device time

@@ -164,6 +164,35 @@ VT_API vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, cons
 VT_API vt_status vt_forward_video(vt_handle* h, const float* clips, int frames, const int32_t* grid_thw, int B,
                                   void* out, void* tower_out, void* ws, size_t ws_bytes, void* stream);
 
+/* GPU preprocessing of decoded images: bicubic resize to the grid's size, scaling by
+ * 1/255 and per-channel normalisation, x = (v/255 - mean[c]) / std[c].
+ *   images    device uint8, the B images [H0_b, W0_b, 3] (RGB, rows of interleaved
+ *             pixels, as decoded) concatenated in order; no alignment needed
+ *   src_hw    host int32 [B, 2] = (H0_b, W0_b); each side at most 16x the target side
+ *   grid_thw  host int32[3] = (1, h, w): every image is resized to h*patch x w*patch
+ *   mean, std host float[3] each, or NULL for the OpenAI CLIP statistics
+ *             (0.48145466, 0.4578275, 0.40821073) / (0.26862954, 0.26130258, 0.27577711)
+ *   pixels    device fp32 [B, 3, h*patch, w*patch], the input vt_forward takes
+ * The resize is cubic convolution with Keys' kernel (a = -0.5): output pixel centres map
+ * onto input pixel centres, the kernel is stretched by the scale factor when shrinking
+ * (every source pixel contributes), taps outside the image are dropped and the weights
+ * renormalised; resized values are not clamped or rounded to 8 bits.  Needs no weights
+ * (h may be unloaded).  Errors: VT_ERR_SHAPE for a grid t != 1 or a source side above 16x
+ * the target, VT_ERR_INVALID_ARG for empty images or std <= 0.  Source: "v2_loaders"
+ * findings, section 3 (bicubic resize to 672x672, OpenAI CLIP mean/std, patchify). */
+VT_API vt_status vt_preprocess(const vt_handle* h, const uint8_t* images, const int32_t* src_hw, int B,
+                               const int32_t* grid_thw, const float* mean, const float* std, float* pixels,
+                               void* stream);
+
+/* Full forward from decoded images: the preprocessing of vt_preprocess writes the patch
+ * vectors of the patch-embedding GEMM directly (no fp32 pixel array), then the forward
+ * of vt_forward.  Arguments as vt_preprocess and vt_forward; ws of at least
+ * vt_workspace_bytes(h, B, grid_thw) bytes.  The result equals vt_forward applied to
+ * vt_preprocess's pixels, bit for bit. */
+VT_API vt_status vt_forward_u8(vt_handle* h, const uint8_t* images, const int32_t* src_hw, int B,
+                               const int32_t* grid_thw, const float* mean, const float* std, void* out,
+                               void* tower_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Variable-resolution batch: B images (1 <= B <= 64) of different patch grids in one
  * call, their tokens packed into one sequence; attention stays within each image.
  *   pixels  device fp32, the images' [3, H_b, W_b] arrays concatenated in order

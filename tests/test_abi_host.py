@@ -180,3 +180,24 @@ def test_last_error_message_is_thread_local_string():
     with pytest.raises(V.VtError):
         V.vt_linear(None, 16, None, None, 16, 4, 16, 16, 0)
     assert "NULL" in V.vt_last_error()
+
+
+def test_preprocess_argument_checks_need_no_device():
+    h = V.vt_create(S.get_config("tiny"))
+    grid = (1, 4, 4)  # 56 x 56 target
+    for src, code in [([(900, 56)], "VT_ERR_SHAPE"),       # more than 16x the target height
+                      ([(56, 897)], "VT_ERR_SHAPE"),
+                      ([(0, 56)], "VT_ERR_INVALID_ARG")]:
+        with pytest.raises(V.VtError) as e:
+            V.vt_preprocess(h, 16, src, grid, 16)
+        assert _status(e) == code, src
+    with pytest.raises(V.VtError) as e:
+        V.vt_preprocess(h, 16, [(56, 56)], grid, 16, mean=(0.5, 0.5, 0.5), std=(0.2, 0.0, 0.2))
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    with pytest.raises(V.VtError) as e:
+        V.vt_preprocess(h, 16, [(56, 56)], (2, 4, 4), 16)
+    assert _status(e) == "VT_ERR_SHAPE"
+    with pytest.raises(V.VtError) as e:
+        V.vt_forward_u8(h, 16, [(56, 56)], grid, 16, None, 16, 1 << 20)
+    assert _status(e) == "VT_ERR_NOT_LOADED"
+    V.vt_destroy(h)

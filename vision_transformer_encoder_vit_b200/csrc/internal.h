@@ -134,6 +134,23 @@ cudaError_t launch_patch_unfold_frames(const float* pixels, void* out, int B, in
 // in 2x2-block order per image.
 cudaError_t launch_patch_unfold_varlen(const float* pixels, void* out, const VarlenTable& vl, int patch, int tp,
                                        cudaStream_t stream);
+// Decoded 8-bit RGB images [H0_b, W0_b, 3] resized to one patch grid.  Passed by value.
+constexpr int kMaxShrink = 16;  // a source side may be at most 16x the target side
+struct PreprocTable {
+  int count;                            // images in this launch (<= kMaxVarlenImages)
+  long long src_off[kMaxVarlenImages];  // byte offset of each image
+  int src_h[kMaxVarlenImages];
+  int src_w[kMaxVarlenImages];
+  float mean[3], std[3];                // per channel, applied after scaling by 1/255
+};
+// Upper bound on the source rows under one output patch (sizes the shared staging).
+size_t preprocess_rows_bound(int src, int dst, int patch);
+// Bicubic resize + normalisation of tab.count images to grid (gh, gw): to_patches = 0
+// writes pixels fp32 [count, 3, gh*p, gw*p]; to_patches = 1 writes patch vectors bf16
+// [count*gh*gw, 3*tp*p*p] in `order`.  rows_cap >= preprocess_rows_bound of every image.
+cudaError_t launch_preprocess(const uint8_t* images, const PreprocTable& tab, void* out, int gh, int gw,
+                              int patch, int tp, int order, int to_patches, int rows_cap, cudaStream_t stream);
+unsigned int preprocess_read_clear_error(cudaStream_t stream);
 // Row gather: out[r] = in[src(r)] where src maps between raster and block order.
 // to_block != 0: out is block order, in is raster.  Rows of `cols` bf16 each.
 cudaError_t launch_reorder_rows(const void* in, void* out, int B, int gt, int gh, int gw, int cols, int to_block,

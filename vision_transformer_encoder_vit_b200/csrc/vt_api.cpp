@@ -508,25 +508,15 @@ vt_status vt_load_weights(vt_handle* h, const vt_weight* w, int n) {
   return VT_OK;
 }
 
-// Forward of B clips of F frames [B, F, 3, H, W] with grid (t, gh, gw), t = ceil(F / tp)
-// (a still image is F = 1, t = 1).  Arguments are checked by the callers.
-static vt_status forward_clips(vt_handle* h, const float* pixels, int F, int B, int t, int gh, int gw, void* out,
-                               void* tower_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+// Everything after the patch vectors: patch-embed GEMM on the block-ordered patch
+// vectors at ws + pl.unfold, the layers, the optional raster copy of the tower, the
+// merge and projector.
+static vt_status forward_embedded(vt_handle* h, int B, int t, int gh, int gw, void* out, void* tower_out, char* w,
+                                  const Plan& pl, cudaStream_t st) {
   const vt_config& c = h->cfg;
-  const Plan pl = make_plan(c, B, t, gh, gw);
-  if (ws_bytes < pl.total)
-    return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, pl.total);
-  vt_status s;
-  char* w = static_cast<char*>(ws);
   void* x = w + pl.x;
   const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
-  {
-    const double px_bytes = 4.0 * B * F * 3.0 * (gh * c.patch) * (gw * c.patch);
-    ProfScope ps(CLS_UNFOLD, 0, px_bytes + 2.0 * pl.M * K0, st);
-    cudaError_t e = launch_patch_unfold_frames(pixels, w + pl.unfold, B, F, gh * c.patch, gw * c.patch, c.patch,
-                                               c.temporal_patch, ORDER_BLOCK, st);
-    if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
-  }
+  vt_status s;
   if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0,
                                 ACT_NONE),
                     st)))
@@ -539,6 +529,26 @@ static vt_status forward_clips(vt_handle* h, const float* pixels, int F, int B, 
     if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
   }
   return run_projector(h, x, out, w, pl, st);
+}
+
+// Forward of B clips of F frames [B, F, 3, H, W] with grid (t, gh, gw), t = ceil(F / tp)
+// (a still image is F = 1, t = 1).  Arguments are checked by the callers.
+static vt_status forward_clips(vt_handle* h, const float* pixels, int F, int B, int t, int gh, int gw, void* out,
+                               void* tower_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const vt_config& c = h->cfg;
+  const Plan pl = make_plan(c, B, t, gh, gw);
+  if (ws_bytes < pl.total)
+    return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, pl.total);
+  char* w = static_cast<char*>(ws);
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  {
+    const double px_bytes = 4.0 * B * F * 3.0 * (gh * c.patch) * (gw * c.patch);
+    ProfScope ps(CLS_UNFOLD, 0, px_bytes + 2.0 * pl.M * K0, st);
+    cudaError_t e = launch_patch_unfold_frames(pixels, w + pl.unfold, B, F, gh * c.patch, gw * c.patch, c.patch,
+                                               c.temporal_patch, ORDER_BLOCK, st);
+    if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
+  }
+  return forward_embedded(h, B, t, gh, gw, out, tower_out, w, pl, st);
 }
 
 static vt_status check_forward_ptrs(const float* pixels, const void* out, const void* tower_out, const void* ws) {
@@ -573,6 +583,122 @@ vt_status vt_forward_video(vt_handle* h, const float* clips, int frames, const i
                 tp, (frames + tp - 1) / tp);
   return forward_clips(h, clips, frames, B, t, gh, gw, out, tower_out, ws, ws_bytes,
                        static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+// OpenAI CLIP image statistics, used when the caller passes no mean / std.
+const float kClipMean[3] = {0.48145466f, 0.4578275f, 0.40821073f};
+const float kClipStd[3] = {0.26862954f, 0.26130258f, 0.27577711f};
+
+// Checks decoded-image sizes against the target grid and splits the batch into
+// launch tables of at most kMaxVarlenImages images.
+vt_status build_preproc(const vt_config& c, const int32_t* src_hw, int B, int gh, int gw, const float* mean,
+                        const float* std_, std::vector<PreprocTable>* tabs, int* rows_cap, double* src_bytes) {
+  if (!src_hw) return fail(VT_ERR_INVALID_ARG, "src_hw is NULL");
+  const float* m = mean ? mean : kClipMean;
+  const float* sd = std_ ? std_ : kClipStd;
+  for (int ch = 0; ch < 3; ++ch)
+    if (!(sd[ch] > 0.f) || !std::isfinite(m[ch]))
+      return fail(VT_ERR_INVALID_ARG, "channel %d: std must be positive and mean finite", ch);
+  const int H1 = gh * c.patch, W1 = gw * c.patch;
+  tabs->clear();
+  long long off = 0;
+  size_t cap = 1;
+  for (int b = 0; b < B; ++b) {
+    const int H0 = src_hw[2 * b], W0 = src_hw[2 * b + 1];
+    if (H0 <= 0 || W0 <= 0) return fail(VT_ERR_INVALID_ARG, "image %d has size %dx%d", b, H0, W0);
+    if (H0 > kMaxShrink * H1 || W0 > kMaxShrink * W1)
+      return fail(VT_ERR_SHAPE, "image %d (%dx%d) is more than %dx the %dx%d target", b, H0, W0, kMaxShrink, H1, W1);
+    if (b % kMaxVarlenImages == 0) {
+      tabs->emplace_back();
+      PreprocTable& t = tabs->back();
+      std::memset(&t, 0, sizeof(t));
+      for (int ch = 0; ch < 3; ++ch) {
+        t.mean[ch] = m[ch];
+        t.std[ch] = sd[ch];
+      }
+      off = 0;  // offsets are relative to the table's first image
+    }
+    PreprocTable& t = tabs->back();
+    t.src_off[t.count] = off;
+    t.src_h[t.count] = H0;
+    t.src_w[t.count] = W0;
+    ++t.count;
+    off += 3ll * H0 * W0;
+    *src_bytes += 3.0 * H0 * W0;
+    cap = std::max(cap, preprocess_rows_bound(H0, H1, c.patch));
+  }
+  *rows_cap = static_cast<int>(cap);
+  return VT_OK;
+}
+
+// Launches the tables one after the other; images and out advance per table.
+vt_status run_preproc(const vt_config& c, const uint8_t* images, const std::vector<PreprocTable>& tabs, void* out,
+                      int gh, int gw, int to_patches, int rows_cap, cudaStream_t st) {
+  const size_t per_image = to_patches ? static_cast<size_t>(gh) * gw * 3 * c.temporal_patch * c.patch * c.patch * 2
+                                      : static_cast<size_t>(3) * gh * c.patch * gw * c.patch * 4;
+  char* o = static_cast<char*>(out);
+  for (const PreprocTable& t : tabs) {
+    cudaError_t e = launch_preprocess(images, t, o, gh, gw, c.patch, c.temporal_patch, ORDER_BLOCK, to_patches,
+                                      rows_cap, st);
+    if (e != cudaSuccess) return cuda_fail(e, "preprocess launch");
+    images += t.src_off[t.count - 1] + 3ll * t.src_h[t.count - 1] * t.src_w[t.count - 1];
+    o += per_image * t.count;
+  }
+  return VT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+vt_status vt_preprocess(const vt_handle* h, const uint8_t* images, const int32_t* src_hw, int B,
+                        const int32_t* grid_thw, const float* mean, const float* std_, float* pixels, void* stream) {
+  if (!h) return fail(VT_ERR_INVALID_ARG, "handle is NULL");
+  if (!images || !pixels) return fail(VT_ERR_INVALID_ARG, "images and pixels must not be NULL");
+  if (!aligned16(pixels)) return fail(VT_ERR_INVALID_ARG, "pixels must be 16-byte aligned");
+  int t, gh, gw;
+  vt_status s = check_grid(h, B, grid_thw, &t, &gh, &gw);
+  if (s) return s;
+  if ((s = check_still(t, "vt_preprocess"))) return s;
+  std::vector<PreprocTable> tabs;
+  int cap;
+  double src_bytes = 0;
+  if ((s = build_preproc(h->cfg, src_hw, B, gh, gw, mean, std_, &tabs, &cap, &src_bytes))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope ps(CLS_UNFOLD, 0, src_bytes + 4.0 * B * 3.0 * gh * gw * h->cfg.patch * h->cfg.patch, st);
+  return run_preproc(h->cfg, images, tabs, pixels, gh, gw, 0, cap, st);
+}
+
+vt_status vt_forward_u8(vt_handle* h, const uint8_t* images, const int32_t* src_hw, int B, const int32_t* grid_thw,
+                        const float* mean, const float* std_, void* out, void* tower_out, void* ws, size_t ws_bytes,
+                        void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!images || !out || !ws) return fail(VT_ERR_INVALID_ARG, "images, out and ws must not be NULL");
+  if (!aligned16(out) || !aligned16(ws) || (tower_out && !aligned16(tower_out)))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int t, gh, gw;
+  if ((s = check_grid(h, B, grid_thw, &t, &gh, &gw))) return s;
+  if ((s = check_still(t, "vt_forward_u8"))) return s;
+  const vt_config& c = h->cfg;
+  const Plan pl = make_plan(c, B, t, gh, gw);
+  if (ws_bytes < pl.total)
+    return fail(VT_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, pl.total);
+  std::vector<PreprocTable> tabs;
+  int cap;
+  double src_bytes = 0;
+  if ((s = build_preproc(c, src_hw, B, gh, gw, mean, std_, &tabs, &cap, &src_bytes))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  {
+    ProfScope ps(CLS_UNFOLD, 0, src_bytes + 2.0 * pl.M * 3 * c.temporal_patch * c.patch * c.patch, st);
+    if ((s = run_preproc(c, images, tabs, w + pl.unfold, gh, gw, 1, cap, st))) return s;
+  }
+  return forward_embedded(h, B, t, gh, gw, out, tower_out, w, pl, st);
 }
 
 }  // extern "C"
@@ -912,9 +1038,11 @@ vt_status vt_check(void* stream) {
   const unsigned int ge = gemm_read_clear_error(st);
   const unsigned int ae = attention_read_clear_error(st);
   const unsigned int se = selftest_read_clear_error(st);
+  const unsigned int pe = preprocess_read_clear_error(st);
   if (ge || ae || se)
     return fail(VT_ERR_TIMEOUT, "kernel wait limit reached (gemm flags %u, attention flags %u, self-test flags %u)",
                 ge, ae, se);
+  if (pe) return fail(VT_ERR_CUDA, "preprocess tap window above its bound (flags %u): results are wrong", pe);
   return VT_OK;
 }
 

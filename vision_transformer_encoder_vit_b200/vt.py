@@ -54,6 +54,7 @@ _i = ctypes.c_int
 _f = ctypes.c_float
 _sz = ctypes.c_size_t
 _i32p = ctypes.POINTER(ctypes.c_int32)
+_fp = ctypes.POINTER(ctypes.c_float)
 
 _SIGS = {
     "vt_create": ([ctypes.POINTER(vt_config), ctypes.POINTER(_vp)]),
@@ -66,6 +67,8 @@ _SIGS = {
     "vt_workspace_bytes_varlen": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
     "vt_forward_varlen": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_forward_video": ([_vp, _vp, _i, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
+    "vt_preprocess": ([_vp, _vp, _i32p, _i, _i32p, _fp, _fp, _vp, _vp]),
+    "vt_forward_u8": ([_vp, _vp, _i32p, _i, _i32p, _fp, _fp, _vp, _vp, _vp, _sz, _vp]),
     "vt_tower_layer": ([_vp, _i, _vp, _vp, _i32p, _i, _vp, _sz, _vp]),
     "vt_patch_embed": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_merge_project": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
@@ -190,6 +193,29 @@ def vt_forward_video(h, clips, frames, grid_thw, B, out, tower_out, ws, ws_bytes
     """clips: device fp32 [B, frames, 3, H, W]; grid_thw = (ceil(frames / tp), H/p, W/p)."""
     _check(lib.vt_forward_video(h, _ptr(clips), frames, _grid(grid_thw), B, _ptr(out), _ptr(tower_out), _ptr(ws),
                                 ws_bytes, _stream(stream)), "vt_forward_video")
+
+
+def _stats(v) -> ctypes.Array | None:
+    return None if v is None else (ctypes.c_float * 3)(*[float(x) for x in v])
+
+
+def _sizes(src_hw) -> ctypes.Array:
+    flat = [int(v) for hw in src_hw for v in hw]
+    return (ctypes.c_int32 * len(flat))(*flat)
+
+
+def vt_preprocess(h, images, src_hw, grid_thw, pixels, mean=None, std=None, stream=None) -> None:
+    """images: device uint8, the images' [H0, W0, 3] arrays concatenated; src_hw: list of
+    (H0, W0); pixels: device fp32 [B, 3, h*p, w*p].  mean/std None: CLIP statistics."""
+    _check(lib.vt_preprocess(h, _ptr(images), _sizes(src_hw), len(src_hw), _grid(grid_thw), _stats(mean),
+                             _stats(std), _ptr(pixels), _stream(stream)), "vt_preprocess")
+
+
+def vt_forward_u8(h, images, src_hw, grid_thw, out, tower_out, ws, ws_bytes, mean=None, std=None,
+                  stream=None) -> None:
+    _check(lib.vt_forward_u8(h, _ptr(images), _sizes(src_hw), len(src_hw), _grid(grid_thw), _stats(mean),
+                             _stats(std), _ptr(out), _ptr(tower_out), _ptr(ws), ws_bytes, _stream(stream)),
+           "vt_forward_u8")
 
 
 def _grids(grids) -> ctypes.Array:
