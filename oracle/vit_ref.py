@@ -37,6 +37,11 @@ tests/test_oracle_pins.py):
   * 2x2 merge: merged token (i, j) concatenates tokens (2i,2j), (2i,2j+1), (2i+1,2j),
     (2i+1,2j+1) in that order; merged tokens are in raster (i, j) order.
   * Images of a batch are independent (attention never crosses images).
+  * Backward ("differentiable" loaders whose probe backpropagates the pooled tower
+    feature, findings summary and section 3): the gradient of a scalar loss with respect
+    to the model pixels, given its gradient with respect to the tower output, through
+    every layer and the patch embedding (the chain rule applied to the forward above;
+    weights are constants).
   * Preprocessing ("bicubic resize to 672x672, OpenAI CLIP mean/std", findings section
     3): the resize is separable cubic-convolution resampling with the Keys kernel at
     a = -0.5, output pixel centres mapped onto input pixel centres, the kernel widened
@@ -58,6 +63,8 @@ __all__ = [
     "attention_probs", "tower_layer", "tower_layer_rows", "merge_2x2", "projector",
     "patch_unfold_video", "forward_video",
     "cubic_kernel", "resize_taps", "resize_bicubic", "preprocess",
+    "layer_norm_backward", "gelu_backward", "rope_3d_backward", "attention_backward",
+    "tower_layer_backward", "patch_fold", "tower_backward",
     "projector_rows", "forward",
     "block_order", "merge_source_map",
 ]
@@ -331,6 +338,131 @@ def tower_layer_rows(x: np.ndarray, w: dict, i: int, cfg: dict, pos: np.ndarray 
     xn = layer_norm(xr, w[p + "ln2.weight"], w[p + "ln2.bias"], cfg["ln_eps"])
     hmid = gelu(xn @ w[p + "mlp.fc1.weight"].T + w[p + "mlp.fc1.bias"], cfg["gelu_tanh"])
     return xr + hmid @ w[p + "mlp.fc2.weight"].T + w[p + "mlp.fc2.bias"]
+
+
+# ------------------------------------------------------------------ backward
+#
+# Reverse-mode derivatives of the forward functions above: each takes the forward's
+# inputs and the gradient dy of a scalar loss with respect to the forward's output, and
+# returns the gradient with respect to the chosen input (J^T dy).
+
+def layer_norm_backward(x: np.ndarray, gamma: np.ndarray, eps: float, dy: np.ndarray) -> np.ndarray:
+    """d loss / d x of layer_norm(x, gamma, beta, eps) over the last axis.
+    With xhat = (x - mu) / sigma and g = dy * gamma:
+        dx = (g - mean(g) - xhat * mean(g * xhat)) / sigma."""
+    mu = x.mean(axis=-1, keepdims=True)
+    sigma = np.sqrt(((x - mu) ** 2).mean(axis=-1, keepdims=True) + eps)
+    xhat = (x - mu) / sigma
+    g = dy * gamma
+    return (g - g.mean(axis=-1, keepdims=True) - xhat * (g * xhat).mean(axis=-1, keepdims=True)) / sigma
+
+
+def gelu_backward(z: np.ndarray, dy: np.ndarray, tanh_form: bool = True) -> np.ndarray:
+    """d loss / d z of gelu(z): dy * gelu'(z).  tanh form, u = c (z + 0.044715 z^3):
+    gelu' = 0.5 (1 + tanh u) + 0.5 z (1 - tanh^2 u) c (1 + 3 * 0.044715 z^2);
+    exact form: gelu' = Phi(z) + z phi(z)."""
+    if tanh_form:
+        c = np.sqrt(2.0 / np.pi)
+        th = np.tanh(c * (z + 0.044715 * z ** 3))
+        return dy * (0.5 * (1.0 + th) + 0.5 * z * (1.0 - th ** 2) * c * (1.0 + 3 * 0.044715 * z ** 2))
+    from math import erf, sqrt
+    cdf = 0.5 * (1.0 + np.vectorize(erf)(z / sqrt(2.0)))
+    pdf = np.exp(-0.5 * z ** 2) / np.sqrt(2.0 * np.pi)
+    return dy * (cdf + z * pdf)
+
+
+def rope_3d_backward(dy: np.ndarray, pos: np.ndarray, sections, theta: float) -> np.ndarray:
+    """d loss / d x of apply_rope_3d(x, pos): every pair is rotated by phi, a linear
+    map whose transpose is the rotation by -phi, i.e. the embedding at position -pos."""
+    return apply_rope_3d(dy, -pos, sections, theta)
+
+
+def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray, scale: float):
+    """Gradients of O = softmax(q k^T * scale) v for one head (q [n, D], k, v [N, D],
+    do = d loss / d O [n, D]).  With P the probabilities:
+        dv = P^T do,   dP = do v^T,   dS = P * (dP - rowsum(P * dP)),
+        dq = scale dS k,   dk = scale dS^T q."""
+    P = attention_probs(q, k, scale)
+    dv = P.T @ do
+    dP = do @ v.T
+    dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+    return scale * dS @ k, scale * dS.T @ q, dv
+
+
+def tower_layer_backward(x: np.ndarray, w: dict, i: int, cfg: dict, pos: np.ndarray | None,
+                         dy: np.ndarray) -> np.ndarray:
+    """d loss / d x of tower_layer(x, w, i, cfg, pos) for one image, given
+    dy = d loss / d (layer output).  Recomputes the forward's intermediates, then walks
+    the block backwards: MLP branch, LN2, output projection, attention, RoPE, qkv, LN1;
+    each residual connection passes its gradient through unchanged."""
+    p = f"layers.{i}."
+    N, d = x.shape
+    H, D = cfg["heads"], cfg["head_dim"]
+    # forward, keeping what the backward needs
+    xn1 = layer_norm(x, w[p + "ln1.weight"], w[p + "ln1.bias"], cfg["ln_eps"])
+    qkv = xn1 @ w[p + "attn.qkv.weight"].T + w[p + "attn.qkv.bias"]
+    q = qkv[:, 0 * d:1 * d].reshape(N, H, D)
+    k = qkv[:, 1 * d:2 * d].reshape(N, H, D)
+    v = qkv[:, 2 * d:3 * d].reshape(N, H, D)
+    if pos is not None:
+        q = apply_rope_3d(q, pos, cfg["rope_sections"], cfg["rope_theta"])
+        k = apply_rope_3d(k, pos, cfg["rope_sections"], cfg["rope_theta"])
+    o = attention(q.transpose(1, 0, 2), k.transpose(1, 0, 2), v.transpose(1, 0, 2),
+                  1.0 / np.sqrt(D)).reshape(N, d)
+    x1 = x + o @ w[p + "attn.o.weight"].T + w[p + "attn.o.bias"]
+    xn2 = layer_norm(x1, w[p + "ln2.weight"], w[p + "ln2.bias"], cfg["ln_eps"])
+    z = xn2 @ w[p + "mlp.fc1.weight"].T + w[p + "mlp.fc1.bias"]
+    # MLP branch: x2 = x1 + gelu(z) W2^T + b2
+    dz = gelu_backward(z, dy @ w[p + "mlp.fc2.weight"], cfg["gelu_tanh"])
+    dx1 = dy + layer_norm_backward(x1, w[p + "ln2.weight"], cfg["ln_eps"], dz @ w[p + "mlp.fc1.weight"])
+    # attention branch: x1 = x + o Wo^T + bo
+    do = (dx1 @ w[p + "attn.o.weight"]).reshape(N, H, D)
+    dq, dk, dv = (np.empty((N, H, D)) for _ in range(3))
+    for h in range(H):
+        dq[:, h], dk[:, h], dv[:, h] = attention_backward(q[:, h], k[:, h], v[:, h], do[:, h], 1.0 / np.sqrt(D))
+    if pos is not None:
+        dq = rope_3d_backward(dq, pos, cfg["rope_sections"], cfg["rope_theta"])
+        dk = rope_3d_backward(dk, pos, cfg["rope_sections"], cfg["rope_theta"])
+    dqkv = np.concatenate([dq.reshape(N, d), dk.reshape(N, d), dv.reshape(N, d)], axis=1)
+    return dx1 + layer_norm_backward(x, w[p + "ln1.weight"], cfg["ln_eps"], dqkv @ w[p + "attn.qkv.weight"])
+
+
+def patch_fold(du: np.ndarray, H: int, W: int, patch: int = 14, temporal_patch: int = 2) -> np.ndarray:
+    """Transpose of patch_unfold: gradients of the patch vectors [gh*gw, 3*tp*p*p]
+    (raster) -> gradient of the image [3, H, W].  Each pixel sits in one patch, once per
+    repeated frame, so its gradient is the sum over those tp copies."""
+    gh, gw = H // patch, W // patch
+    out = np.zeros((3, H, W), dtype=np.float64)
+    blocks = du.reshape(gh, gw, 3, temporal_patch, patch, patch).sum(axis=3)  # [gh, gw, 3, p, p]
+    for h in range(gh):
+        for w_ in range(gw):
+            out[:, h * patch:(h + 1) * patch, w_ * patch:(w_ + 1) * patch] = blocks[h, w_]
+    return out
+
+
+def tower_backward(pixels: np.ndarray, w: dict, cfg: dict, d_tower: np.ndarray,
+                   layers: int | None = None) -> dict:
+    """Gradient of a loss with respect to the pixels [B, 3, H, W], given its gradient
+    d_tower [B, N, hidden] with respect to the tower output (raster order).  Returns
+    dict(tower=the forward's tower output, d_pixels=[B, 3, H, W])."""
+    p, tp = cfg["patch"], cfg["temporal_patch"]
+    L = cfg["layers"] if layers is None else layers
+    tows, grads = [], []
+    for b in range(pixels.shape[0]):
+        img = pixels[b].astype(np.float64)
+        gh, gw = img.shape[1] // p, img.shape[2] // p
+        pos = positions_raster(1, gh, gw) if cfg.get("use_rope", True) else None
+        xs = [patch_embed(patch_unfold(img, p, tp), w["embeddings.proj.weight"], w["embeddings.proj.bias"])]
+        for i in range(L):
+            xs.append(tower_layer(xs[-1], w, i, cfg, pos))
+        dx = d_tower[b].astype(np.float64)
+        for i in reversed(range(L)):
+            dx = tower_layer_backward(xs[i], w, i, cfg, pos, dx)
+        wpe = w["embeddings.proj.weight"]
+        du = dx @ wpe.reshape(wpe.shape[0], -1)
+        tows.append(xs[-1])
+        grads.append(patch_fold(du, img.shape[1], img.shape[2], p, tp))
+    return dict(tower=np.stack(tows), d_pixels=np.stack(grads))
 
 
 # ------------------------------------------------------- merge and projector

@@ -493,3 +493,120 @@ def test_preprocess_channel_order_and_statistics():
                         mode="bicubic", antialias=True, align_corners=False)[0].numpy()
     ref = (ref / 255 - np.asarray(S.CLIP_MEAN)[:, None, None]) / np.asarray(S.CLIP_STD)[:, None, None]
     np.testing.assert_allclose(R.preprocess(img, 28, 42, S.CLIP_MEAN, S.CLIP_STD), ref, atol=1e-10)
+
+
+# ------------------------------------------------------------------ backward
+
+def _fd_directional(f, x, v, dy, eps=1e-5):
+    """<dy, (f(x + eps v) - f(x - eps v)) / (2 eps)>: the directional derivative of
+    the loss <dy, f(x)> along v, by central differences (error O(eps^2))."""
+    return float(np.sum(dy * (f(x + eps * v) - f(x - eps * v))) / (2 * eps))
+
+
+def test_layer_norm_and_gelu_backward_equal_autograd():
+    r = _rng(50)
+    x, dy, gamma = r.standard_normal((7, 40)), r.standard_normal((7, 40)), 1 + 0.1 * r.standard_normal(40)
+    xt = torch.tensor(x, requires_grad=True)
+    F.layer_norm(xt, (40,), torch.tensor(gamma), torch.tensor(0.1 * gamma), 1e-6).backward(torch.tensor(dy))
+    np.testing.assert_allclose(R.layer_norm_backward(x, gamma, 1e-6, dy), xt.grad.numpy(), atol=1e-12)
+    z = 3 * r.standard_normal((5, 33))
+    dz = r.standard_normal((5, 33))
+    for tanh_form, approx in ((True, "tanh"), (False, "none")):
+        zt = torch.tensor(z, requires_grad=True)
+        F.gelu(zt, approximate=approx).backward(torch.tensor(dz))
+        np.testing.assert_allclose(R.gelu_backward(z, dz, tanh_form), zt.grad.numpy(), atol=1e-12)
+
+
+def test_rope_backward_is_the_transpose():
+    r = _rng(51)
+    pos = R.positions_raster(2, 3, 5)
+    x, y = r.standard_normal((30, 2, 80)), r.standard_normal((30, 2, 80))
+    rx = R.apply_rope_3d(x, pos, (16, 32, 32), 1e4)
+    # <R x, y> = <x, R^T y> and R^T R = I
+    assert np.sum(rx * y) == pytest.approx(np.sum(x * R.rope_3d_backward(y, pos, (16, 32, 32), 1e4)), abs=1e-10)
+    np.testing.assert_allclose(R.rope_3d_backward(rx, pos, (16, 32, 32), 1e4), x, atol=1e-12)
+
+
+def test_attention_backward_equals_autograd_and_differences():
+    r = _rng(52)
+    n, N, D = 9, 13, 16
+    q, k, v, do = r.standard_normal((n, D)), r.standard_normal((N, D)), r.standard_normal((N, D)), \
+        r.standard_normal((n, D))
+    scale = D ** -0.5
+    dq, dk, dv = R.attention_backward(q, k, v, do, scale)
+    qt, kt, vt = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    (torch.softmax(qt @ kt.T * scale, dim=1) @ vt).backward(torch.tensor(do))
+    for got, ref in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), atol=1e-12)
+    # and against central differences of the oracle's own forward, input by input
+    f = lambda a, b, c: R.attention_probs(a, b, scale) @ c
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        vdir = r.standard_normal((q, k, v)[which].shape)
+        args = [q, k, v]
+        g = lambda z: f(*[z if i == which else args[i] for i in range(3)])
+        assert _fd_directional(g, args[which], vdir, do) == pytest.approx(np.sum(grad * vdir), rel=1e-7)
+
+
+def test_layer_backward_without_rope_equals_autograd_of_torch_modules():
+    cfg = S.get_config("tiny", use_rope=False)
+    w = _layer_weights(cfg, 53)
+    d, H = cfg["hidden"], cfg["heads"]
+    r = _rng(54)
+    x, dy = r.standard_normal((24, d)), r.standard_normal((24, d))
+    mha = torch.nn.MultiheadAttention(d, H, bias=True, batch_first=True)
+    ln1, ln2 = torch.nn.LayerNorm(d, eps=1e-6), torch.nn.LayerNorm(d, eps=1e-6)
+    fc1, fc2 = torch.nn.Linear(d, cfg["mlp"]), torch.nn.Linear(cfg["mlp"], d)
+    T = torch.tensor
+    with torch.no_grad():
+        mha.in_proj_weight.copy_(T(w["layers.0.attn.qkv.weight"]))
+        mha.in_proj_bias.copy_(T(w["layers.0.attn.qkv.bias"]))
+        mha.out_proj.weight.copy_(T(w["layers.0.attn.o.weight"]))
+        mha.out_proj.bias.copy_(T(w["layers.0.attn.o.bias"]))
+        for mod, nm in ((ln1, "ln1"), (ln2, "ln2")):
+            mod.weight.copy_(T(w[f"layers.0.{nm}.weight"]))
+            mod.bias.copy_(T(w[f"layers.0.{nm}.bias"]))
+        for mod, nm in ((fc1, "fc1"), (fc2, "fc2")):
+            mod.weight.copy_(T(w[f"layers.0.mlp.{nm}.weight"]))
+            mod.bias.copy_(T(w[f"layers.0.mlp.{nm}.bias"]))
+    xt = T(x)[None].requires_grad_(True)
+    a = ln1(xt)
+    y = xt + mha(a, a, a, need_weights=False)[0]
+    y = y + fc2(F.gelu(fc1(ln2(y)), approximate="tanh"))
+    y.backward(T(dy)[None])
+    np.testing.assert_allclose(R.tower_layer_backward(x, w, 0, cfg, None, dy), xt.grad[0].numpy(), atol=1e-11)
+
+
+def test_layer_backward_with_rope_equals_central_differences():
+    cfg = S.get_config("tiny")
+    w = _layer_weights(cfg, 55)
+    r = _rng(56)
+    pos = R.positions_raster(1, 4, 6)
+    x, dy = r.standard_normal((24, cfg["hidden"])), r.standard_normal((24, cfg["hidden"]))
+    dx = R.tower_layer_backward(x, w, 0, cfg, pos, dy)
+    for _ in range(3):
+        vdir = r.standard_normal(x.shape)
+        fd = _fd_directional(lambda z: R.tower_layer(z, w, 0, cfg, pos), x, vdir, dy)
+        assert fd == pytest.approx(np.sum(dx * vdir), rel=1e-7)
+    # the rotation matters: without it the gradient differs
+    assert np.abs(R.tower_layer_backward(x, w, 0, cfg, None, dy) - dx).max() > 1e-3
+
+
+def test_patch_fold_is_the_transpose_of_unfold():
+    r = _rng(57)
+    img, du = r.standard_normal((3, 28, 42)), r.standard_normal((6, 3 * 2 * 14 * 14))
+    assert np.sum(R.patch_unfold(img, 14, 2) * du) == pytest.approx(np.sum(img * R.patch_fold(du, 28, 42)),
+                                                                     abs=1e-10)
+
+
+def test_tower_backward_equals_central_differences_on_pixels():
+    cfg = dict(S.get_config("tiny"), image=(28, 56))
+    w = S.weights_f64(S.make_weights(cfg, affine=True))
+    r = _rng(58)
+    px = r.standard_normal((1, 3, 28, 56))
+    d_tower = r.standard_normal((1, 8, cfg["hidden"]))
+    res = R.tower_backward(px, w, cfg, d_tower)
+    np.testing.assert_allclose(res["tower"], R.forward(px, w, cfg)["tower"], atol=1e-12)
+    for _ in range(2):
+        vdir = r.standard_normal(px.shape)
+        fd = _fd_directional(lambda z: R.forward(z, w, cfg)["tower"], px, vdir, d_tower)
+        assert fd == pytest.approx(np.sum(res["d_pixels"] * vdir), rel=1e-6)
