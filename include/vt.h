@@ -209,6 +209,53 @@ VT_API vt_status vt_workspace_bytes_varlen(const vt_handle* h, int B, const int3
 VT_API vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int32_t* grids, int B, void* out,
                                    void* tower_out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- backward
+ * Gradient of a scalar loss with respect to the pixels, given its gradient with
+ * respect to the tower output: every layer backwards (recomputed from its saved input),
+ * then the patch embedding and the fold onto the image.  Weights are constants (no
+ * weight gradients).  Source: "v2_loaders - Differentiable Vision Tower Loaders
+ * (spark2)", summary and section 3 (the loaders are differentiable; the probe
+ * backpropagates the pooled tower feature to the image); the forward differentiated is
+ * that of the "MiniMax-M3 Vision" model card, Architecture table.  Still images only
+ * (grid t = 1); head_dim 80 (RoPE 16/32/32) or 32 (8/12/12). */
+
+/* Builds library-owned transposed copies of the tower weights (the size of the tower
+ * weights again), after vt_load_weights; a later vt_load_weights drops them.
+ * Synchronises the device.  VT_ERR_UNSUPPORTED for other head layouts. */
+VT_API vt_status vt_enable_backward(vt_handle* h);
+
+/* Bytes of the saved-activation buffer (every layer's input, L * B*N*hidden bf16) and of
+ * the workspace (covers both vt_forward_saved and vt_backward).  Host only. */
+VT_API vt_status vt_backward_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* saved_bytes,
+                                   size_t* ws_bytes);
+
+/* Forward of the tower that keeps every layer's input in `saved` (device, opaque layout)
+ * and writes the tower output tower_out (device bf16 [B, N, hidden], raster order).
+ * pixels as vt_forward. */
+VT_API vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* tower_out,
+                                  void* saved, size_t saved_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/* d_tower: device bf16 [B, N, hidden] (raster order), the loss gradient with respect to
+ * the tower output of the vt_forward_saved call that filled `saved`; d_pixels: device
+ * fp32 [B, 3, H, W], the loss gradient with respect to the pixels (the sum over the
+ * temporal patch's two copies of each frame).  VT_ERR_NOT_LOADED before
+ * vt_enable_backward. */
+VT_API vt_status vt_backward(vt_handle* h, const void* saved, const int32_t* grid_thw, int B, const void* d_tower,
+                             float* d_pixels, void* ws, size_t ws_bytes, void* stream);
+
+/* Attention backward alone, no rotary embedding: q, k, v device bf16 [B, H, N, D] (q, k
+ * as the scores use them), dO device bf16 [B*N, H*D] (gradient of the output
+ * [B, N, H, D]); writes dqkv device bf16 [B*N, 3*H*D] = [dq | dk | dv], each in the
+ * [B*N, H*D] layout.  Recomputes the forward; no [N, N] buffer.  D in {32, 80}. */
+VT_API vt_status vt_attention_backward_workspace_bytes(int B, int H, int N, int D, size_t* out);
+VT_API vt_status vt_attention_backward(const void* q, const void* k, const void* v, const void* dO, void* dqkv, int B,
+                                       int H, int N, int D, float scale, void* ws, size_t ws_bytes, void* stream);
+
+/* LayerNorm backward plus a residual gradient: dx = dres + J^T dy for y = LN(x) (gamma);
+ * all device bf16 [rows, cols] (gamma [cols]); dres may equal dx; cols a multiple of 8. */
+VT_API vt_status vt_layernorm_backward(const void* x, const void* gamma, const void* dy, const void* dres, void* dx,
+                                       int rows, int cols, float eps, void* stream);
+
 /* One pre-LN tower layer i on raster-ordered tokens: x_out = layer_i(x_in), both
  * device bf16 [B, t*h*w, hidden]; x_in may equal x_out.  Source: ViTBlock of
  * "metrale_model_arch/weight_loader/qwen3_vl.rs" (norm1, qkv, proj, norm2, fc1, fc2);

@@ -201,3 +201,27 @@ def test_preprocess_argument_checks_need_no_device():
         V.vt_forward_u8(h, 16, [(56, 56)], grid, 16, None, 16, 1 << 20)
     assert _status(e) == "VT_ERR_NOT_LOADED"
     V.vt_destroy(h)
+
+
+def test_backward_argument_checks_need_no_device():
+    assert V.vt_attention_backward_workspace_bytes(2, 16, 100, 80) == \
+        4 * ((2 * 16 * 80 * 104 * 2 + 255) // 256 * 256) + (2 * 100 * 16 * 80 * 2 + 255) // 256 * 256 + \
+        2 * ((2 * 16 * 128 * 4 + 255) // 256 * 256)
+    for D, code in ((64, "VT_ERR_UNSUPPORTED"), (80, "VT_ERR_WORKSPACE")):
+        with pytest.raises(V.VtError) as e:
+            V.vt_attention_backward(16, 16, 16, 16, 16, 1, 2, 100, D, 0.1, 16, 1024)
+        assert _status(e) == code
+    with pytest.raises(V.VtError) as e:
+        V.vt_layernorm_backward(16, 16, 16, 16, 16, 4, 1281, 1e-6)
+    assert _status(e) == "VT_ERR_INVALID_ARG"
+    h = V.vt_create(S.get_config("tower448"))
+    saved, ws = V.vt_backward_bytes(h, 2, (1, 32, 32))
+    assert saved == 32 * 2 * 1024 * 1280 * 2  # every layer's input
+    assert ws >= V.vt_workspace_bytes(h, 2, (1, 32, 32))
+    with pytest.raises(V.VtError) as e:
+        V.vt_backward_bytes(h, 1, (2, 8, 8))
+    assert _status(e) == "VT_ERR_SHAPE"
+    with pytest.raises(V.VtError) as e:
+        V.vt_enable_backward(h)
+    assert _status(e) == "VT_ERR_NOT_LOADED"
+    V.vt_destroy(h)

@@ -1,0 +1,123 @@
+"""The tower backward on the GPU against the fp64 oracle: LayerNorm backward, the
+attention backward (ragged sizes, both head layouts), and the pixel gradient of whole
+towers (tiny, and one and two full-width 1280 layers).  Gates as for the forward:
+relative L2 <= 1e-2 for single kernels, <= 2e-2 for gradients that crossed whole layers,
+plus the element-wise bound of tests/gpu_util.py."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vit_ref as R
+from vision_transformer_encoder_vit_b200 import synthetic as S
+from tests.gpu_util import REL_L2_FINAL, REL_L2_LAYER, assert_close, dev_bf16, dev_f32, empty_bf16, host_f64
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from vision_transformer_encoder_vit_b200 import vt as V
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 1280), (37, 1280), (1000, 128), (9, 200)])
+def test_layernorm_backward(rows, cols):
+    x = S.make_matrix((rows, cols), rows + cols, 2.0)
+    g = S.bf16_bits(S.bf16_to_f32(S.make_matrix((cols,), 5, 0.3)) + np.float32(1.0))
+    dy = S.make_matrix((rows, cols), 7, 1.0)
+    dres = S.make_matrix((rows, cols), 8, 0.5)
+    dx = empty_bf16(rows, cols)
+    V.vt_layernorm_backward(dev_bf16(x), dev_bf16(g), dev_bf16(dy), dev_bf16(dres), dx, rows, cols, 1e-6)
+    ref = S.bf16_to_f64(dres) + R.layer_norm_backward(S.bf16_to_f64(x), S.bf16_to_f64(g), 1e-6, S.bf16_to_f64(dy))
+    assert_close(host_f64(dx), ref, what=f"layernorm backward {rows}x{cols}")
+
+
+def _attn_bwd_case(B, H, N, D, seed, q_scale=1.0, atol=None):
+    q, k, v = S.make_qkv(B, H, N, D, seed)
+    if q_scale != 1.0:
+        q = S.bf16_bits(S.bf16_to_f32(q) * np.float32(q_scale))
+    dO = S.make_matrix((B * N, H * D), seed + 1)
+    dqkv = empty_bf16(B * N, 3 * H * D)
+    ws_bytes = V.vt_attention_backward_workspace_bytes(B, H, N, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    scale = D ** -0.5
+    V.vt_attention_backward(dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_bf16(dO), dqkv, B, H, N, D, scale, ws, ws_bytes)
+    V.vt_check()
+    got = host_f64(dqkv).reshape(B, N, 3, H, D)
+    qf, kf, vf = (S.bf16_to_f64(a) for a in (q, k, v))
+    dOf = S.bf16_to_f64(dO).reshape(B, N, H, D)
+    for b in range(B):
+        for h in range(H):
+            ref = R.attention_backward(qf[b, h], kf[b, h], vf[b, h], dOf[b, :, h], scale)
+            for j, name in enumerate(("dq", "dk", "dv")):
+                kw = {} if atol is None else dict(atol=atol)
+                assert_close(got[b, :, j, h], ref[j], what=f"attention backward {name} D={D} N={N} b={b} h={h}", **kw)
+
+
+@pytest.mark.parametrize("N", [1, 5, 64, 65, 127, 128, 129, 300, 1024])
+def test_attention_backward_d80_ragged(N):
+    _attn_bwd_case(2, 2, N, 80, 20 + N)
+
+
+@pytest.mark.parametrize("N", [64, 200])
+def test_attention_backward_d32(N):
+    _attn_bwd_case(2, 4, N, 32, 30 + N)
+
+
+def test_attention_backward_peaked_softmax():
+    # Large scores: probabilities close to one-hot, the log-sum-exp carries the row scale.
+    # There dS = P (dP - delta) with delta ~ dP of the dominant key: a cancellation that
+    # amplifies the bf16 rounding of P and dS, so single elements may miss the few-ulp
+    # element bound; the L2 gate stays 1e-2 and the element bound is widened to 2^-4 rms.
+    _attn_bwd_case(1, 2, 333, 80, 41, q_scale=5.0, atol=2.0 ** -4)
+
+
+def _tower_backward(cfg, hw, batch, affine, layers=None, seed=3):
+    c = dict(cfg, image=hw)
+    if layers is not None:
+        c["layers"] = layers
+    bits = S.make_weights(c, affine=affine, layers=layers)
+    tw = V.Tower(c, bits)
+    V.vt_enable_backward(tw.h)
+    gh, gw = hw[0] // 14, hw[1] // 14
+    grid = (1, gh, gw)
+    N = gh * gw
+    px = S.make_pixels(c, batch=batch, seed=seed)
+    d_tower = S.make_matrix((batch, N, c["hidden"]), seed + 5)
+    saved_bytes, ws_bytes = V.vt_backward_bytes(tw.h, batch, grid)
+    saved = torch.empty(saved_bytes, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    tower = empty_bf16(batch, N, c["hidden"])
+    V.vt_forward_saved(tw.h, dev_f32(px), grid, batch, tower, saved, saved_bytes, ws, ws_bytes)
+    dpx = torch.empty((batch, 3, hw[0], hw[1]), dtype=torch.float32, device="cuda")
+    V.vt_backward(tw.h, saved, grid, batch, dev_bf16(d_tower), dpx, ws, ws_bytes)
+    V.vt_check()
+    ref = R.tower_backward(px.astype(np.float64), S.weights_f64(bits), c, S.bf16_to_f64(d_tower))
+    assert_close(host_f64(tower), ref["tower"], rel=REL_L2_LAYER if c["layers"] <= 2 else REL_L2_FINAL,
+                 what="forward_saved tower")
+    assert_close(dpx.cpu().numpy().astype(np.float64), ref["d_pixels"], rel=REL_L2_FINAL,
+                 what=f"pixel gradient {hw} x{batch}, {c['layers']} layers of width {c['hidden']}")
+    tw.close()
+
+
+def test_tower_backward_tiny():
+    _tower_backward(S.get_config("tiny"), (56, 84), 2, affine=True)
+
+
+def test_tower_backward_full_width_one_layer_224():
+    _tower_backward(S.get_config("tower448"), (224, 224), 1, affine=True, layers=1)
+
+
+def test_tower_backward_full_width_two_layers_448():
+    # 1024 tokens: eight 128-row tiles per head in both backward kernels
+    _tower_backward(S.get_config("tower448"), (448, 448), 1, affine=False, layers=2, seed=4)
+
+
+def test_backward_needs_enable_and_still_images():
+    cfg = S.get_config("tiny")
+    tw = V.Tower(cfg, S.make_weights(cfg, affine=True))
+    with pytest.raises(V.VtError) as e:
+        V.vt_backward(tw.h, 16, (1, 4, 4), 1, 16, 16, 16, 1 << 30)
+    assert e.value.name == "VT_ERR_NOT_LOADED"
+    V.vt_enable_backward(tw.h)
+    with pytest.raises(V.VtError) as e:
+        V.vt_backward_bytes(tw.h, 1, (2, 4, 4))
+    assert e.value.name == "VT_ERR_SHAPE"
+    tw.close()

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libvt.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["gemm.cu", "attention.cu", "elementwise.cu", "tma.cpp", "vt_api.cpp", "attention_static.cu", "selftest.cu", "preprocess.cu"]
+SOURCES = ["gemm.cu", "attention.cu", "elementwise.cu", "tma.cpp", "vt_api.cpp", "attention_static.cu", "selftest.cu", "preprocess.cu", "attention_bwd.cu", "backward.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -347,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float o[D];
       load_cols<D>(tO, o);
       const int n = (qp * 2 + t) * S::BM + r;
+      if (p.lse && n < N) p.lse[static_cast<size_t>(bh) * p.ld_lse + n] = m_ref + __log2f(l);
       if (n < N) {
         const float inv = 1.0f / l;
 #pragma unroll

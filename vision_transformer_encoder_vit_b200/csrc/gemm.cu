@@ -130,15 +130,27 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
         const int cg = col + 8 * g;
         if (cg < p.N) {
           if (bias) add_bf16x8(v + 8 * g, bq[g]);
+          if (p.act >= ACT_DGELU_TANH) {
+            // backward of GELU: scale by gelu'(pre-activation), which `resid` carries
+            const uint32_t w[4] = {rq[g].x, rq[g].y, rq[g].z, rq[g].w};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float x = v[8 * g + i];
-            if (p.act == ACT_GELU_TANH) x = gelu_tanh(x);
-            else if (p.act == ACT_GELU_ERF) x = gelu_erf(x);
-            v[8 * g + i] = x;
+            for (int i = 0; i < 4; ++i) {
+              const float2 z = unpack_bf16x2(w[i]);
+              const bool th = p.act == ACT_DGELU_TANH;
+              v[8 * g + 2 * i] *= th ? gelu_tanh_grad(z.x) : gelu_erf_grad(z.x);
+              v[8 * g + 2 * i + 1] *= th ? gelu_tanh_grad(z.y) : gelu_erf_grad(z.y);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float x = v[8 * g + i];
+              if (p.act == ACT_GELU_TANH) x = gelu_tanh(x);
+              else if (p.act == ACT_GELU_ERF) x = gelu_erf(x);
+              v[8 * g + i] = x;
+            }
           }
           if (row < p.M) {
-            if (resid) add_bf16x8(v + 8 * g, rq[g]);
+            if (resid && p.act < ACT_DGELU_TANH) add_bf16x8(v + 8 * g, rq[g]);
             *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.ldo + cg) = pack_bf16x8(v + 8 * g);
           }
         }

@@ -62,7 +62,9 @@ __host__ __device__ inline int varlen_image(const VarlenTable& t, int row) {
 
 // ------------------------------------------------------------------ GEMM
 
-enum GemmAct : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2 };
+// ACT_DGELU_*: backward of GELU, out = (A W^T) * gelu'(aux) with aux passed as `resid`
+// (the pre-activation; not added).
+enum GemmAct : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2, ACT_DGELU_TANH = 3, ACT_DGELU_ERF = 4 };
 
 // out[M, N] = act(A[M, K] * W[N, K]^T + bias) (+ resid), bf16 in and out, fp32 accumulate.
 struct GemmParams {
@@ -115,9 +117,39 @@ struct AttnParams {
   // N is then the largest N_b (it sizes the grid).
   int varlen;
   VarlenTable vl;
+  // Optional: base-2 log-sum-exp of the scaled scores of every query row,
+  // lse[(b*H + h) * ld_lse + n] = log2(sum_j 2^(s_nj * scale * log2 e)), for the backward.
+  float* lse;
+  int ld_lse;
 };
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream);
 unsigned int attention_read_clear_error(cudaStream_t stream);
+
+// Attention backward for uniform batches (every image N tokens).  q, k, v, o-gradient
+// and the forward's lse in; dq, dk (rotated back by RoPE) and dv written into the
+// [B*N, ld_dqkv] qkv-gradient matrix at column blocks 0, H*D and 2*H*D.
+struct AttnBwdParams {
+  const void* q;      // [B, H, N, D] bf16, rotated
+  const void* k;      // [B, H, N, D] bf16, rotated
+  const void* v;      // [B, H, N, D] bf16
+  const void* qT;     // [B, H, D, ld] bf16 (q transposed)
+  const void* kT;     // [B, H, D, ld]
+  const void* dO;     // [B*N, H*D] bf16, gradient of the attention output
+  const void* dOT;    // [B, H, D, ld]
+  const float* lse;   // [B*H, ld_stats], from the forward
+  const float* delta; // [B*H, ld_stats], rowsum(dO * O) per query
+  int ld_stats;       // multiple of 64, >= N
+  void* dqkv;         // [B*N, ld_dqkv] bf16
+  int ld_dqkv;
+  int B, H, N, D, ld;  // ld: multiple of 8, >= N
+  float scale;
+  int rope;
+  int sections[3];
+  const float2* rope_tab;
+  int gh, gw, order;
+};
+cudaError_t launch_attention_backward(const AttnBwdParams& p, cudaStream_t stream);
+unsigned int attention_bwd_read_clear_error(cudaStream_t stream);
 
 // -------------------------------------------------------- memory-bound ops
 
@@ -160,6 +192,22 @@ cudaError_t launch_reorder_rows(const void* in, void* out, int B, int gt, int gh
 cudaError_t launch_attention_prep(const void* q, const void* k, const void* v, void* qr, void* kr, void* vt,
                                   int B, int H, int N, int D, int ld_vt, const int32_t* pos,
                                   const int sections[3], float theta, cudaStream_t stream);
+
+// ---------------------------------------------------------- backward, memory-bound
+
+// dx = dres + LayerNorm backward of x (gamma) applied to dy; dres may alias dx.
+cudaError_t launch_layernorm_backward(const void* x, const void* gamma, const void* dy, const void* dres, void* dx,
+                                      int rows, int cols, float eps, cudaStream_t stream);
+// delta[(b*H + h) * ld + n] = <dO, O> over head h of token b*N + n ([B*N, H*D] bf16 each).
+cudaError_t launch_attention_delta(const void* dO, const void* O, float* delta, int B, int N, int H, int D, int ld,
+                                   cudaStream_t stream);
+// For z = (b, h): out[c][r] = in[r][c], r < R, c < C; strides in bf16 elements.
+cudaError_t launch_transpose(const void* src, void* dst, int B, int H, int R, int C, long in_sb, long in_sh,
+                             long in_ld, long out_sb, long out_sh, long out_ld, cudaStream_t stream);
+// Patch-vector gradients [B*gh*gw, 3*tp*p*p] (tokens in `order`) -> pixel gradients
+// [B, 3, H, W] fp32 (sum over the repeated frames).
+cudaError_t launch_patch_fold(const void* du, float* dpixels, int B, int H, int W, int patch, int tp, int order,
+                              cudaStream_t stream);
 
 // -------------------------------------------------------------------- TMA
 

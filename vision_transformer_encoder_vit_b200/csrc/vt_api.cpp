@@ -42,7 +42,17 @@ inline int round8(int x) { return (x + 7) & ~7; }
 
 // ---------------------------------------------------------------- profiling
 
-enum { CLS_GEMM = 0, CLS_ATTN = 1, CLS_LN = 2, CLS_UNFOLD = 3, CLS_REORDER = 4, CLS_PREP = 5, CLS_COUNT = 6 };
+enum {
+  CLS_GEMM = 0,
+  CLS_ATTN = 1,
+  CLS_LN = 2,
+  CLS_UNFOLD = 3,
+  CLS_REORDER = 4,
+  CLS_PREP = 5,
+  CLS_ATTN_BWD = 6,
+  CLS_BWD_MISC = 7,
+  CLS_COUNT = 8
+};
 
 struct ProfRec {
   int cls;
@@ -169,6 +179,14 @@ struct vt_handle {
   const void *pa1_w, *pa1_b, *pa2_w, *pa2_b, *pb1_w, *pb1_b, *pb2_w, *pb2_b;
   void* qkv_pack = nullptr;  // owned: fused [3d, d] weights + [3d] biases per layer
   float2* rope_tab = nullptr;  // owned: [3][kRopeMaxPos][kRopePairs]
+  // Backward (vt_enable_backward): transposed weights, so every input-gradient product
+  // is a K-major GEMM.  qkv_t [d, 3d], o_t [d, d], fc1_t [d, m], fc2_t [m, d], pe_t [K0, d].
+  struct LayerT {
+    void *qkv_t, *o_t, *fc1_t, *fc2_t;
+  };
+  std::vector<LayerT> layers_t;
+  void* pe_t = nullptr;
+  void* bwd_pack = nullptr;  // owned: all of the above
 };
 
 namespace {
@@ -388,8 +406,9 @@ vt_status vt_create(const vt_config* cfg, vt_handle** out) {
 
 vt_status vt_destroy(vt_handle* h) {
   if (!h) return VT_OK;
-  if (h->qkv_pack || h->rope_tab) cudaDeviceSynchronize();
+  if (h->qkv_pack || h->rope_tab || h->bwd_pack) cudaDeviceSynchronize();
   if (h->qkv_pack) cudaFree(h->qkv_pack);
+  if (h->bwd_pack) cudaFree(h->bwd_pack);
   if (h->rope_tab) cudaFree(h->rope_tab);
   delete h;
   return VT_OK;
@@ -466,7 +485,15 @@ vt_status vt_load_weights(vt_handle* h, const vt_weight* w, int n) {
   for (auto& kv : byname)
     if (!used.count(kv.first)) return fail(VT_ERR_WEIGHT, "unknown weight %s", kv.first.c_str());
 
-  // Device-side state: fused qkv packs and RoPE tables.
+  // Device-side state: fused qkv packs and RoPE tables.  Transposed weights of an
+  // earlier vt_enable_backward no longer match: drop them.
+  if (h->bwd_pack) {
+    cudaDeviceSynchronize();
+    cudaFree(h->bwd_pack);
+    h->bwd_pack = nullptr;
+    h->layers_t.clear();
+    h->pe_t = nullptr;
+  }
   if (h->qkv_pack) {
     cudaFree(h->qkv_pack);
     h->qkv_pack = nullptr;
@@ -1039,9 +1066,12 @@ vt_status vt_check(void* stream) {
   const unsigned int ae = attention_read_clear_error(st);
   const unsigned int se = selftest_read_clear_error(st);
   const unsigned int pe = preprocess_read_clear_error(st);
-  if (ge || ae || se)
-    return fail(VT_ERR_TIMEOUT, "kernel wait limit reached (gemm flags %u, attention flags %u, self-test flags %u)",
-                ge, ae, se);
+  const unsigned int be = attention_bwd_read_clear_error(st);
+  if (ge || ae || se || be)
+    return fail(VT_ERR_TIMEOUT,
+                "kernel wait limit reached (gemm flags %u, attention flags %u, attention backward flags %u, "
+                "self-test flags %u)",
+                ge, ae, be, se);
   if (pe) return fail(VT_ERR_CUDA, "preprocess tap window above its bound (flags %u): results are wrong", pe);
   return VT_OK;
 }
@@ -1121,6 +1151,431 @@ vt_status vt_profile_launch(int64_t i, int* cls, double* ms, double* flops, doub
   if (flops) *flops = d.flops;
   if (bytes) *bytes = d.bytes;
   return VT_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ backward
+//
+// Gradient of a loss with respect to the pixels, given its gradient with respect to the
+// tower output: the reverse of every layer (recomputed from its saved input), then the
+// patch embedding and the fold onto the image.  The derivative follows the chain rule
+// through the forward of the "MiniMax-M3 Vision" model card (Architecture table); the
+// "v2_loaders" findings (summary, section 3) describe the loaders as differentiable,
+// their probe backpropagating the pooled tower feature to the image.
+
+namespace {
+
+struct BwdPlan {
+  int N, M, ld, lds;
+  size_t dx, xn, q, k, vt, a, x1, hmid, dO, qT, kT, dOT, v, dqkv, lse, delta, total;
+};
+
+BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
+  BwdPlan p;
+  p.N = N;
+  p.M = B * N;
+  p.ld = round8(N);
+  p.lds = (N + 63) / 64 * 64;
+  const size_t d = c.hidden, M = static_cast<size_t>(p.M);
+  const size_t K0 = 3ull * c.temporal_patch * c.patch * c.patch;
+  const size_t headT = static_cast<size_t>(B) * c.heads * c.head_dim * p.ld;  // [B, H, D, ld]
+  const size_t stats = static_cast<size_t>(B) * c.heads * p.lds;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  p.dx = take(M * d * 2);
+  p.xn = take(M * d * 2);
+  p.q = take(M * d * 2);
+  p.k = take(M * d * 2);
+  p.vt = take(headT * 2);
+  p.a = take(M * d * 2);
+  p.x1 = take(M * d * 2);
+  p.hmid = take(M * std::max<size_t>(c.mlp, K0) * 2);
+  p.dO = take(M * d * 2);
+  p.qT = take(headT * 2);
+  p.kT = take(headT * 2);
+  p.dOT = take(headT * 2);
+  p.v = take(M * d * 2);
+  p.dqkv = take(M * 3 * d * 2);
+  p.lse = take(stats * 4);
+  p.delta = take(stats * 4);
+  p.total = off;
+  return p;
+}
+
+vt_status run_layernorm_backward(const void* x, const void* g, const void* dy, const void* dres, void* dx, int rows,
+                                 int cols, float eps, cudaStream_t st) {
+  ProfScope ps(CLS_BWD_MISC, 0, 8.0 * rows * static_cast<double>(cols), st);
+  cudaError_t e = launch_layernorm_backward(x, g, dy, dres, dx, rows, cols, eps, st);
+  if (e != cudaSuccess) return cuda_fail(e, "layernorm backward launch");
+  return VT_OK;
+}
+
+// q, k [B, H, N, D] -> [B, H, D, ld]; dO [B*N, H*D] -> [B, H, D, ld]; vt [B, H, D, ld_v] -> v [B, H, N, D].
+vt_status run_bwd_transposes(const void* q, const void* k, const void* dO, const void* vt, int ld_v, void* qT,
+                             void* kT, void* dOT, void* v, int B, int H, int N, int D, int ld, cudaStream_t st) {
+  ProfScope ps(CLS_BWD_MISC, 0, 16.0 * B * H * static_cast<double>(N) * D, st);
+  const long hnd = static_cast<long>(H) * N * D, nd = static_cast<long>(N) * D;
+  const long hdl = static_cast<long>(H) * D * ld, dl = static_cast<long>(D) * ld;
+  cudaError_t e = launch_transpose(q, qT, B, H, N, D, hnd, nd, D, hdl, dl, ld, st);
+  if (e == cudaSuccess) e = launch_transpose(k, kT, B, H, N, D, hnd, nd, D, hdl, dl, ld, st);
+  if (e == cudaSuccess) e = launch_transpose(dO, dOT, B, H, N, D, hnd, D, static_cast<long>(H) * D, hdl, dl, ld, st);
+  if (e == cudaSuccess && vt) {
+    const long hdlv = static_cast<long>(H) * D * ld_v, dlv = static_cast<long>(D) * ld_v;
+    e = launch_transpose(vt, v, B, H, D, N, hdlv, dlv, ld_v, hnd, nd, D, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
+  return VT_OK;
+}
+
+vt_status run_attention_backward(const AttnBwdParams& p, cudaStream_t st) {
+  // 5 matrix products per head (S, dP, dV, dK, dQ): 10 N^2 D
+  ProfScope ps(CLS_ATTN_BWD, 10.0 * p.B * p.H * static_cast<double>(p.N) * p.N * p.D,
+               2.0 * p.B * p.H * static_cast<double>(p.N) * p.D * 8, st);
+  cudaError_t e = launch_attention_backward(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
+  return VT_OK;
+}
+
+// One layer backward on block-ordered tokens: dx (in: d loss / d layer output; out:
+// d loss / d layer input) given the layer's input x_in.
+vt_status run_layer_backward(vt_handle* h, int i, const void* x_in, int B, int gh, int gw, char* w, const BwdPlan& bp,
+                             cudaStream_t st) {
+  const vt_config& c = h->cfg;
+  const vt_handle::Layer& L = h->layers[i];
+  const vt_handle::LayerT& T = h->layers_t[i];
+  const int d = c.hidden, m = c.mlp, M = bp.M, N = bp.N, H = c.heads, D = c.head_dim;
+  void* dx = w + bp.dx;
+  void* xn = w + bp.xn;
+  void* x1 = w + bp.x1;
+  void* hmid = w + bp.hmid;
+  vt_status s;
+  // ---- recompute the forward of this layer
+  if ((s = run_layernorm(x_in, L.ln1_w, L.ln1_b, xn, M, d, c.ln_eps, st))) return s;
+  {
+    GemmParams p = gemm_params(xn, d, L.qkv_w, d, L.qkv_b, nullptr, 0, nullptr, 0, M, 3 * d, d, ACT_NONE);
+    p.q = w + bp.q;
+    p.k = w + bp.k;
+    p.vt = w + bp.vt;
+    p.heads = H;
+    p.head_dim = D;
+    p.ntok = N;
+    p.ld_vt = bp.ld;
+    p.gt = 1;
+    p.gh = gh;
+    p.gw = gw;
+    p.order = ORDER_BLOCK;
+    p.rope = c.use_rope;
+    for (int a = 0; a < 3; ++a) p.sections[a] = c.rope_sections[a];
+    p.rope_tab = h->rope_tab;
+    ProfScope ps(CLS_GEMM, 2.0 * M * 3.0 * d * d, 0, st);
+    cudaError_t e = launch_gemm(p, st, 1);
+    if (e != cudaSuccess) return cuda_fail(e, "qkv gemm launch");
+  }
+  const float scale = 1.0f / std::sqrt(static_cast<float>(D));
+  {
+    AttnParams a{};
+    a.q = w + bp.q;
+    a.k = w + bp.k;
+    a.vt = w + bp.vt;
+    a.o = w + bp.a;
+    a.B = B;
+    a.H = H;
+    a.N = N;
+    a.D = D;
+    a.ld_vt = bp.ld;
+    a.scale = scale;
+    a.lse = reinterpret_cast<float*>(w + bp.lse);
+    a.ld_lse = bp.lds;
+    if ((s = run_attention(a, st))) return s;
+  }
+  if ((s = run_gemm(gemm_params(w + bp.a, d, L.o_w, d, L.o_b, x_in, d, x1, d, M, d, d, ACT_NONE), st))) return s;
+  if ((s = run_layernorm(x1, L.ln2_w, L.ln2_b, xn, M, d, c.ln_eps, st))) return s;
+  if ((s = run_gemm(gemm_params(xn, d, L.fc1_w, d, L.fc1_b, nullptr, 0, hmid, m, M, m, d, ACT_NONE), st))) return s;
+  // ---- MLP branch: dz = (dx W2) * gelu'(z), dg = dz W1, dx += LN2^T(dg)
+  const int dact = c.gelu_tanh ? ACT_DGELU_TANH : ACT_DGELU_ERF;
+  if ((s = run_gemm(gemm_params(dx, d, T.fc2_t, d, nullptr, hmid, m, hmid, m, M, m, d, dact), st))) return s;
+  if ((s = run_gemm(gemm_params(hmid, m, T.fc1_t, m, nullptr, nullptr, 0, xn, d, M, d, m, ACT_NONE), st))) return s;
+  if ((s = run_layernorm_backward(x1, L.ln2_w, xn, dx, dx, M, d, c.ln_eps, st))) return s;
+  // ---- attention branch: dO = dx Wo, attention backward, dh = dqkv Wqkv, dx += LN1^T(dh)
+  if ((s = run_gemm(gemm_params(dx, d, T.o_t, d, nullptr, nullptr, 0, w + bp.dO, d, M, d, d, ACT_NONE), st))) return s;
+  {
+    ProfScope ps(CLS_BWD_MISC, 0, 4.0 * M * d + 4.0 * M * H, st);
+    cudaError_t e = launch_attention_delta(w + bp.dO, w + bp.a, reinterpret_cast<float*>(w + bp.delta), B, N, H, D,
+                                           bp.lds, st);
+    if (e != cudaSuccess) return cuda_fail(e, "delta launch");
+  }
+  if ((s = run_bwd_transposes(w + bp.q, w + bp.k, w + bp.dO, w + bp.vt, bp.ld, w + bp.qT, w + bp.kT, w + bp.dOT,
+                              w + bp.v, B, H, N, D, bp.ld, st)))
+    return s;
+  {
+    AttnBwdParams a{};
+    a.q = w + bp.q;
+    a.k = w + bp.k;
+    a.v = w + bp.v;
+    a.qT = w + bp.qT;
+    a.kT = w + bp.kT;
+    a.dO = w + bp.dO;
+    a.dOT = w + bp.dOT;
+    a.lse = reinterpret_cast<const float*>(w + bp.lse);
+    a.delta = reinterpret_cast<const float*>(w + bp.delta);
+    a.ld_stats = bp.lds;
+    a.dqkv = w + bp.dqkv;
+    a.ld_dqkv = 3 * d;
+    a.B = B;
+    a.H = H;
+    a.N = N;
+    a.D = D;
+    a.ld = bp.ld;
+    a.scale = scale;
+    a.rope = c.use_rope;
+    for (int j = 0; j < 3; ++j) a.sections[j] = c.rope_sections[j];
+    a.rope_tab = h->rope_tab;
+    a.gh = gh;
+    a.gw = gw;
+    a.order = ORDER_BLOCK;
+    if ((s = run_attention_backward(a, st))) return s;
+  }
+  if ((s = run_gemm(gemm_params(w + bp.dqkv, 3 * d, T.qkv_t, 3 * d, nullptr, nullptr, 0, xn, d, M, d, 3 * d,
+                                ACT_NONE),
+                    st)))
+    return s;
+  return run_layernorm_backward(x_in, L.ln1_w, xn, dx, dx, M, d, c.ln_eps, st);
+}
+
+vt_status check_backward_grid(const vt_handle* h, int B, const int32_t* grid_thw, int* gh, int* gw) {
+  int t;
+  vt_status s = check_grid(h, B, grid_thw, &t, gh, gw);
+  if (s) return s;
+  if ((s = check_still(t, "the backward"))) return s;
+  return VT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+vt_status vt_enable_backward(vt_handle* h) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  const vt_config& c = h->cfg;
+  if (!((c.head_dim == 80 && (!c.use_rope || (c.rope_sections[0] == 16 && c.rope_sections[1] == 32 &&
+                                               c.rope_sections[2] == 32))) ||
+        (c.head_dim == 32 && (!c.use_rope || (c.rope_sections[0] == 8 && c.rope_sections[1] == 12 &&
+                                               c.rope_sections[2] == 12)))))
+    return fail(VT_ERR_UNSUPPORTED, "the attention backward covers head_dim 80 (16/32/32) and 32 (8/12/12)");
+  if (h->bwd_pack) return VT_OK;
+  const size_t d = c.hidden, m = c.mlp, K0 = 3ull * c.temporal_patch * c.patch * c.patch;
+  const size_t per_layer = align256(3 * d * d * 2) + align256(d * d * 2) + 2 * align256(d * m * 2);
+  void* pack = nullptr;
+  cudaError_t e = cudaMalloc(&pack, per_layer * c.layers + align256(K0 * d * 2));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(transposed weights)");
+  std::vector<vt_handle::LayerT> lt(c.layers);
+  char* base = static_cast<char*>(pack);
+  for (int i = 0; i < c.layers && e == cudaSuccess; ++i) {
+    vt_handle::LayerT& T = lt[i];
+    const vt_handle::Layer& L = h->layers[i];
+    T.qkv_t = base;
+    T.o_t = base + align256(3 * d * d * 2);
+    T.fc1_t = static_cast<char*>(T.o_t) + align256(d * d * 2);
+    T.fc2_t = static_cast<char*>(T.fc1_t) + align256(d * m * 2);
+    base += per_layer;
+    // W [out, in] -> W^T [in, out]
+    e = launch_transpose(L.qkv_w, T.qkv_t, 1, 1, 3 * d, d, 0, 0, d, 0, 0, 3 * d, 0);
+    if (e == cudaSuccess) e = launch_transpose(L.o_w, T.o_t, 1, 1, d, d, 0, 0, d, 0, 0, d, 0);
+    if (e == cudaSuccess) e = launch_transpose(L.fc1_w, T.fc1_t, 1, 1, m, d, 0, 0, d, 0, 0, m, 0);
+    if (e == cudaSuccess) e = launch_transpose(L.fc2_w, T.fc2_t, 1, 1, d, m, 0, 0, m, 0, 0, d, 0);
+  }
+  void* pe_t = base;
+  if (e == cudaSuccess) e = launch_transpose(h->pe_w, pe_t, 1, 1, d, K0, 0, 0, K0, 0, 0, d, 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaFree(pack);
+    return cuda_fail(e, "transposing weights");
+  }
+  h->layers_t = std::move(lt);
+  h->pe_t = pe_t;
+  h->bwd_pack = pack;
+  return VT_OK;
+}
+
+vt_status vt_backward_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* saved_bytes,
+                            size_t* ws_bytes) {
+  if (!h || !saved_bytes || !ws_bytes) return fail(VT_ERR_INVALID_ARG, "handle and outputs must not be NULL");
+  int gh, gw;
+  vt_status s = check_backward_grid(h, B, grid_thw, &gh, &gw);
+  if (s) return s;
+  const vt_config& c = h->cfg;
+  const size_t M = static_cast<size_t>(B) * gh * gw;
+  *saved_bytes = static_cast<size_t>(c.layers) * align256(M * c.hidden * 2);
+  *ws_bytes = std::max(make_plan(c, B, 1, gh, gw).total, make_bwd_plan(c, B, gh * gw).total);
+  return VT_OK;
+}
+
+vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* tower_out,
+                           void* saved, size_t saved_bytes, void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!pixels || !tower_out || !saved || !ws) return fail(VT_ERR_INVALID_ARG, "pointers must not be NULL");
+  if (!aligned16(pixels) || !aligned16(tower_out) || !aligned16(saved) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int gh, gw;
+  if ((s = check_backward_grid(h, B, grid_thw, &gh, &gw))) return s;
+  size_t need_saved, need_ws;
+  vt_backward_bytes(h, B, grid_thw, &need_saved, &need_ws);
+  if (saved_bytes < need_saved || ws_bytes < need_ws)
+    return fail(VT_ERR_WORKSPACE, "saved (%zu < %zu) or workspace (%zu < %zu) too small", saved_bytes, need_saved,
+                ws_bytes, need_ws);
+  const vt_config& c = h->cfg;
+  const Plan pl = make_plan(c, B, 1, gh, gw);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const size_t layer_bytes = align256(static_cast<size_t>(pl.M) * c.hidden * 2);
+  auto layer_in = [&](int i) -> void* { return static_cast<char*>(saved) + i * layer_bytes; };
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  {
+    ProfScope ps(CLS_UNFOLD, 0, pl.M * (4.0 * 3 * c.patch * c.patch + 2.0 * K0), st);
+    cudaError_t e = launch_patch_unfold(pixels, w + pl.unfold, B, gh * c.patch, gw * c.patch, c.patch,
+                                        c.temporal_patch, ORDER_BLOCK, st);
+    if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
+  }
+  void* x0 = c.layers > 0 ? layer_in(0) : w + pl.x;
+  if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x0, c.hidden, pl.M, c.hidden,
+                                K0, ACT_NONE),
+                    st)))
+    return s;
+  for (int i = 0; i < c.layers; ++i) {
+    void* out = i + 1 < c.layers ? layer_in(i + 1) : w + pl.x;
+    if ((s = run_layer(h, i, layer_in(i), out, B, 1, gh, gw, ORDER_BLOCK, w, pl, st))) return s;
+  }
+  ProfScope ps(CLS_REORDER, 0, 4.0 * pl.M * c.hidden, st);
+  cudaError_t e = launch_reorder_rows(w + pl.x, tower_out, B, 1, gh, gw, c.hidden, 0, st);
+  if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+  return VT_OK;
+}
+
+vt_status vt_backward(vt_handle* h, const void* saved, const int32_t* grid_thw, int B, const void* d_tower,
+                      float* d_pixels, void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!h->bwd_pack) return fail(VT_ERR_NOT_LOADED, "call vt_enable_backward before vt_backward");
+  if (!saved || !d_tower || !d_pixels || !ws) return fail(VT_ERR_INVALID_ARG, "pointers must not be NULL");
+  if (!aligned16(saved) || !aligned16(d_tower) || !aligned16(d_pixels) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int gh, gw;
+  if ((s = check_backward_grid(h, B, grid_thw, &gh, &gw))) return s;
+  size_t need_saved, need_ws;
+  vt_backward_bytes(h, B, grid_thw, &need_saved, &need_ws);
+  if (ws_bytes < need_ws) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, need_ws);
+  const vt_config& c = h->cfg;
+  const int N = gh * gw, d = c.hidden;
+  const BwdPlan bp = make_bwd_plan(c, B, N);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const size_t layer_bytes = align256(static_cast<size_t>(bp.M) * d * 2);
+  {
+    ProfScope ps(CLS_REORDER, 0, 4.0 * bp.M * d, st);
+    cudaError_t e = launch_reorder_rows(d_tower, w + bp.dx, B, 1, gh, gw, d, 1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
+  }
+  for (int i = c.layers - 1; i >= 0; --i)
+    if ((s = run_layer_backward(h, i, static_cast<const char*>(saved) + i * layer_bytes, B, gh, gw, w, bp, st)))
+      return s;
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  if ((s = run_gemm(gemm_params(w + bp.dx, d, h->pe_t, d, nullptr, nullptr, 0, w + bp.hmid, K0, bp.M, K0, d,
+                                ACT_NONE),
+                    st)))
+    return s;
+  ProfScope ps(CLS_BWD_MISC, 0, 2.0 * bp.M * K0 + 4.0 * bp.M * 3 * c.patch * c.patch, st);
+  cudaError_t e = launch_patch_fold(w + bp.hmid, d_pixels, B, gh * c.patch, gw * c.patch, c.patch, c.temporal_patch,
+                                    ORDER_BLOCK, st);
+  if (e != cudaSuccess) return cuda_fail(e, "patch fold launch");
+  return VT_OK;
+}
+
+vt_status vt_attention_backward_workspace_bytes(int B, int H, int N, int D, size_t* out) {
+  if (!out || B <= 0 || H <= 0 || N <= 0 || D <= 0) return fail(VT_ERR_INVALID_ARG, "bad arguments");
+  const size_t ld = static_cast<size_t>(round8(N)), lds = (static_cast<size_t>(N) + 63) / 64 * 64;
+  const size_t headT = static_cast<size_t>(B) * H * D * ld;
+  const size_t tok = static_cast<size_t>(B) * N * H * D;
+  *out = 4 * align256(headT * 2) + align256(tok * 2) + 2 * align256(static_cast<size_t>(B) * H * lds * 4);
+  return VT_OK;
+}
+
+vt_status vt_attention_backward(const void* q, const void* k, const void* v, const void* dO, void* dqkv, int B, int H,
+                                int N, int D, float scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dqkv || !ws) return fail(VT_ERR_INVALID_ARG, "pointers must not be NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dqkv) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (B <= 0 || H <= 0 || N <= 0) return fail(VT_ERR_INVALID_ARG, "B, H, N must be positive");
+  if (!(scale > 0.f)) return fail(VT_ERR_INVALID_ARG, "scale must be positive");
+  if (D != 32 && D != 80) return fail(VT_ERR_UNSUPPORTED, "the attention backward covers head_dim 32 and 80");
+  if (static_cast<long long>(B) * H * N > (1ll << 31) - 256) return fail(VT_ERR_SHAPE, "too many rows");
+  size_t need;
+  vt_attention_backward_workspace_bytes(B, H, N, D, &need);
+  if (ws_bytes < need) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, need);
+  const int ld = round8(N), lds = (N + 63) / 64 * 64;
+  const size_t headT = static_cast<size_t>(B) * H * D * ld;
+  const size_t tok = static_cast<size_t>(B) * N * H * D;
+  char* w = static_cast<char*>(ws);
+  void* vt_ = w;
+  void* qT = w + align256(headT * 2);
+  void* kT = static_cast<char*>(qT) + align256(headT * 2);
+  void* dOT = static_cast<char*>(kT) + align256(headT * 2);
+  void* o = static_cast<char*>(dOT) + align256(headT * 2);
+  float* lse = reinterpret_cast<float*>(static_cast<char*>(o) + align256(tok * 2));
+  float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse) + align256(static_cast<size_t>(B) * H * lds * 4));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  vt_status s;
+  {
+    // v [B, H, N, D] -> v^T [B, H, D, ld] for the forward recomputation
+    const long hnd = static_cast<long>(H) * N * D, nd = static_cast<long>(N) * D;
+    const long hdl = static_cast<long>(H) * D * ld, dl = static_cast<long>(D) * ld;
+    cudaError_t e = launch_transpose(v, vt_, B, H, N, D, hnd, nd, D, hdl, dl, ld, st);
+    if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
+  }
+  AttnParams a{q, k, vt_, o, B, H, N, D, ld, scale};
+  a.lse = lse;
+  a.ld_lse = lds;
+  if ((s = run_attention(a, st))) return s;
+  {
+    cudaError_t e = launch_attention_delta(dO, o, delta, B, N, H, D, lds, st);
+    if (e != cudaSuccess) return cuda_fail(e, "delta launch");
+  }
+  if ((s = run_bwd_transposes(q, k, dO, nullptr, 0, qT, kT, dOT, nullptr, B, H, N, D, ld, st))) return s;
+  AttnBwdParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.qT = qT;
+  p.kT = kT;
+  p.dO = dO;
+  p.dOT = dOT;
+  p.lse = lse;
+  p.delta = delta;
+  p.ld_stats = lds;
+  p.dqkv = dqkv;
+  p.ld_dqkv = 3 * H * D;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.D = D;
+  p.ld = ld;
+  p.scale = scale;
+  return run_attention_backward(p, st);
+}
+
+vt_status vt_layernorm_backward(const void* x, const void* gamma, const void* dy, const void* dres, void* dx, int rows,
+                                int cols, float eps, void* stream) {
+  if (!x || !gamma || !dy || !dres || !dx) return fail(VT_ERR_INVALID_ARG, "pointers must not be NULL");
+  if (rows < 0 || cols <= 0 || cols % 8) return fail(VT_ERR_INVALID_ARG, "cols must be a positive multiple of 8");
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(dy) || !aligned16(dres) || !aligned16(dx))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return run_layernorm_backward(x, gamma, dy, dres, dx, rows, cols, eps, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -24,7 +24,8 @@ STATUS = {0: "VT_OK", 1: "VT_ERR_INVALID_ARG", 2: "VT_ERR_SHAPE", 3: "VT_ERR_NOT
           8: "VT_ERR_TIMEOUT"}
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
-PROFILE_CLASSES = ("gemm", "attention", "layernorm", "patch_unfold", "reorder", "attention_prep")
+PROFILE_CLASSES = ("gemm", "attention", "layernorm", "patch_unfold", "reorder", "attention_prep",
+                   "attention_backward", "backward_misc")
 
 
 class VtError(RuntimeError):
@@ -68,6 +69,13 @@ _SIGS = {
     "vt_forward_varlen": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_forward_video": ([_vp, _vp, _i, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_preprocess": ([_vp, _vp, _i32p, _i, _i32p, _fp, _fp, _vp, _vp]),
+    "vt_enable_backward": ([_vp]),
+    "vt_backward_bytes": ([_vp, _i, _i32p, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
+    "vt_forward_saved": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp, _sz, _vp]),
+    "vt_backward": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
+    "vt_attention_backward_workspace_bytes": ([_i, _i, _i, _i, ctypes.POINTER(_sz)]),
+    "vt_attention_backward": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "vt_layernorm_backward": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp]),
     "vt_forward_u8": ([_vp, _vp, _i32p, _i, _i32p, _fp, _fp, _vp, _vp, _vp, _sz, _vp]),
     "vt_tower_layer": ([_vp, _i, _vp, _vp, _i32p, _i, _vp, _sz, _vp]),
     "vt_patch_embed": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
@@ -216,6 +224,44 @@ def vt_forward_u8(h, images, src_hw, grid_thw, out, tower_out, ws, ws_bytes, mea
     _check(lib.vt_forward_u8(h, _ptr(images), _sizes(src_hw), len(src_hw), _grid(grid_thw), _stats(mean),
                              _stats(std), _ptr(out), _ptr(tower_out), _ptr(ws), ws_bytes, _stream(stream)),
            "vt_forward_u8")
+
+
+def vt_enable_backward(h) -> None:
+    _check(lib.vt_enable_backward(h), "vt_enable_backward")
+
+
+def vt_backward_bytes(h, B, grid_thw) -> tuple[int, int]:
+    """(saved-activation bytes, workspace bytes) of vt_forward_saved / vt_backward."""
+    a, b = _sz(), _sz()
+    _check(lib.vt_backward_bytes(h, B, _grid(grid_thw), ctypes.byref(a), ctypes.byref(b)), "vt_backward_bytes")
+    return a.value, b.value
+
+
+def vt_forward_saved(h, pixels, grid_thw, B, tower_out, saved, saved_bytes, ws, ws_bytes, stream=None) -> None:
+    _check(lib.vt_forward_saved(h, _ptr(pixels), _grid(grid_thw), B, _ptr(tower_out), _ptr(saved), saved_bytes,
+                                _ptr(ws), ws_bytes, _stream(stream)), "vt_forward_saved")
+
+
+def vt_backward(h, saved, grid_thw, B, d_tower, d_pixels, ws, ws_bytes, stream=None) -> None:
+    _check(lib.vt_backward(h, _ptr(saved), _grid(grid_thw), B, _ptr(d_tower), _ptr(d_pixels), _ptr(ws), ws_bytes,
+                           _stream(stream)), "vt_backward")
+
+
+def vt_attention_backward_workspace_bytes(B, H, N, D) -> int:
+    out = _sz()
+    _check(lib.vt_attention_backward_workspace_bytes(B, H, N, D, ctypes.byref(out)),
+           "vt_attention_backward_workspace_bytes")
+    return out.value
+
+
+def vt_attention_backward(q, k, v, dO, dqkv, B, H, N, D, scale, ws, ws_bytes, stream=None) -> None:
+    _check(lib.vt_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dqkv), B, H, N, D, scale, _ptr(ws),
+                                     ws_bytes, _stream(stream)), "vt_attention_backward")
+
+
+def vt_layernorm_backward(x, gamma, dy, dres, dx, rows, cols, eps, stream=None) -> None:
+    _check(lib.vt_layernorm_backward(_ptr(x), _ptr(gamma), _ptr(dy), _ptr(dres), _ptr(dx), rows, cols, eps,
+                                     _stream(stream)), "vt_layernorm_backward")
 
 
 def _grids(grids) -> ctypes.Array:
