@@ -82,6 +82,12 @@ def workload(name: str) -> dict:
                     tokens=sum(g[1] * g[2] for g in grids),
                     desc="full tower + 2x2 merge + projector on one packed batch of 8 images of mixed sizes "
                          + ", ".join(f"{h}x{w}" for h, w in images))
+    if name == "backward448":
+        cfg = S.get_config("tower448")
+        t, gh, gw = S.token_grid(cfg)
+        return dict(kind="backward", name=name, cfg=cfg, batch=cfg["batch"], grid=(t, gh, gw), tokens=t * gh * gw,
+                    desc=f"tower forward keeping every layer's input + backward to the pixels (32 layers), "
+                         f"{cfg['batch']} images of 448x448")
     if name == "u8_672":
         cfg = dict(S.get_config("tower448"), image=(672, 672))
         sizes = [(1080, 1920), (768, 1024), (480, 640), (3024, 4032), (1200, 1600), (720, 1280), (2000, 3000),
@@ -103,6 +109,18 @@ def workload(name: str) -> dict:
         return dict(kind="attn", name=name, batch=1, grid=(1, side, side), tokens=side * side, heads=16, D=80,
                     desc=f"attention only, 16 heads x 80, {side}x{side} tokens, 3D RoPE")
     raise SystemExit(f"unknown workload {name}")
+
+
+def backward_flops(cfg: dict, N: int) -> float:
+    """Algorithmic FLOPs of one image's tower forward plus its input-gradient backward:
+    every linear layer's dX product costs what its forward costs; the attention backward
+    is 5 products (S, dP, dV, dK, dQ) = 10 N^2 d.  The layer recomputation inside the
+    backward is not counted."""
+    d, m = cfg["hidden"], cfg["mlp"]
+    K0 = 3 * cfg["temporal_patch"] * cfg["patch"] ** 2
+    L = cfg["layers"]
+    gemm = 2 * N * K0 * d + L * 2 * N * d * (3 * d + d + 2 * m)
+    return 2 * gemm + L * (4 + 10) * N * N * d
 
 
 def tower_flops(cfg: dict, N: int) -> dict:
@@ -303,6 +321,26 @@ def run_gpu(args, wl):
         step_flops = sum(tower_flops(cfg, g[1] * g[2])["total"] for g in grids)
         units_per_step = B
         unit = "images/s"
+    elif wl["kind"] == "backward":
+        cfg = wl["cfg"]
+        tower = V.Tower(cfg, S.make_weights(cfg))
+        V.vt_enable_backward(tower.h)
+        px = torch.from_numpy(S.make_pixels(cfg, batch=B, seed=REP.replica_seed(cfg["seed"], rank))).to(dev)
+        d_tower = torch.from_numpy(S.make_matrix((B, N, cfg["hidden"]), 9).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        saved_bytes, ws_bytes = V.vt_backward_bytes(tower.h, B, grid)
+        saved = torch.empty(saved_bytes, dtype=torch.uint8, device=dev)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        tower_out = torch.empty((B, N, cfg["hidden"]), dtype=torch.bfloat16, device=dev)
+        d_px = torch.empty_like(px)
+
+        def launch(s_):
+            V.vt_forward_saved(tower.h, px, grid, B, tower_out, saved, saved_bytes, ws, ws_bytes, s_)
+            V.vt_backward(tower.h, saved, grid, B, d_tower, d_px, ws, ws_bytes, s_)
+
+        step_flops = B * backward_flops(cfg, N)
+        units_per_step = B
+        unit = "images/s"
     elif wl["kind"] == "u8":
         cfg = wl["cfg"]
         tower = V.Tower(cfg, S.make_weights(cfg))
@@ -440,6 +478,26 @@ def run_gpu(args, wl):
                    h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h.numel() * 2),
                    api="vt_forward_host")
         del ws_h
+    elif wl["kind"] == "backward":
+        cfg = wl["cfg"]
+        tower = V.Tower(cfg, S.make_weights(cfg))
+        V.vt_enable_backward(tower.h)
+        px = torch.from_numpy(S.make_pixels(cfg, batch=B, seed=REP.replica_seed(cfg["seed"], rank))).to(dev)
+        d_tower = torch.from_numpy(S.make_matrix((B, N, cfg["hidden"]), 9).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        saved_bytes, ws_bytes = V.vt_backward_bytes(tower.h, B, grid)
+        saved = torch.empty(saved_bytes, dtype=torch.uint8, device=dev)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        tower_out = torch.empty((B, N, cfg["hidden"]), dtype=torch.bfloat16, device=dev)
+        d_px = torch.empty_like(px)
+
+        def launch(s_):
+            V.vt_forward_saved(tower.h, px, grid, B, tower_out, saved, saved_bytes, ws, ws_bytes, s_)
+            V.vt_backward(tower.h, saved, grid, B, d_tower, d_px, ws, ws_bytes, s_)
+
+        step_flops = B * backward_flops(cfg, N)
+        units_per_step = B
+        unit = "images/s"
     elif wl["kind"] == "u8":
         # decoded images from pinned host memory -> device, forward, projected tokens back
         out_h = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory()
@@ -467,12 +525,13 @@ def run_gpu(args, wl):
 
     if rank == 0:
         # dominant kernel class by device time
-        dom = max(("gemm", "attention"), key=lambda c: prof[c]["ms"])
+        dom = max(("gemm", "attention", "attention_backward"), key=lambda c: prof[c]["ms"])
         p = prof[dom]
         achieved = p["flops"] / (p["ms"] / 1000.0) / 1e12 if p["ms"] > 0 else 0.0
         peak = peaks["bf16_tflops_sustained"]
-        roofline = dict(bound="tensor", kernel=("gemm_bf16_tcgen05 (all linear layers)" if dom == "gemm"
-                                                 else "attn_fwd_tcgen05"),
+        roofline = dict(bound="tensor", kernel={"gemm": "gemm_bf16_tcgen05 (all linear layers)",
+                                                "attention": "attn_fwd_tcgen05",
+                                                "attention_backward": "attn_bwd_dq + attn_bwd_dkdv"}[dom],
                         achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
                         peak_source=f"{peaks_kind} bf16 sustained",
                         traffic=recorded_traffic(dom, {"tower448": "tower448_b8"}.get(wl["name"], wl["name"])),

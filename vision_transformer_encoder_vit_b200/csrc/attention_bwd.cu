@@ -13,8 +13,10 @@
 // backpropagate through it to the image.
 //
 // Two kernels, every MMA operand K-major (transposed copies qT, kT, dOT are made
-// beforehand), one CTA = 6 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// the MMAs from one thread, warps 2..5 hold one row each per thread.
+// beforehand), one CTA = 10 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// the MMAs from one thread, warps 2..9 are two groups of four that each own one row per
+// thread and split every 64-column step between them (columns 0..31 and 32..63), so two
+// warps per SM sub-partition hide each other's latencies.
 //  * attn_bwd_dq: one CTA per 128 queries; 64-key steps stream K, V and K^T.
 //        S = Q K_j^T, dP = dO V_j^T  (TMEM, double-buffered)  -> dS (bf16, shared)
 //        dQ += dS K_j                (TMEM accumulator)
@@ -31,7 +33,8 @@ namespace {
 
 __device__ unsigned int g_attn_bwd_err;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kCompute = 256;  // threads of the two row groups
 
 __host__ __device__ constexpr uint32_t layout_code(int swizzle_bytes) {
   return swizzle_bytes == 128 ? 2u : swizzle_bytes == 64 ? 4u : 6u;
@@ -58,18 +61,22 @@ struct BwdShape {
   static constexpr int LIMIT = 232448;
   // attn_bwd_dq: fixed Q, dO; per stage K, V, K^T; dS double-buffered
   static constexpr int DQ_STAGE = 2 * SMALL + TR;
-  static constexpr int DQ_STAGES = 3;
+  static constexpr int DQ_AVAIL = LIMIT - 1024 - BAR_BYTES - 2 * BIG - 2 * PS;
+  static constexpr int DQ_STAGES = DQ_AVAIL / DQ_STAGE > 6 ? 6 : DQ_AVAIL / DQ_STAGE;
   static constexpr int DQ_SMEM = 1024 + 2 * BIG + DQ_STAGES * DQ_STAGE + 2 * PS + BAR_BYTES;
-  // attn_bwd_dkdv: fixed K, V; per stage Q, dO, Q^T, dO^T; P^T and dS^T double-buffered
-  static constexpr int KV_STAGE = 2 * SMALL + 2 * TR;
+  // attn_bwd_dkdv: fixed K, V; ring A holds Q, dO (read by the S^T, dP^T products and
+  // released right after them), ring B holds Q^T, dO^T (read by dV, dK); P^T and dS^T
+  // double-buffered
+  static constexpr int KV_STAGE_A = 2 * SMALL;
+  static constexpr int KV_STAGE_B = 2 * TR;
   static constexpr int KV_AVAIL = LIMIT - 1024 - BAR_BYTES - 2 * BIG - 4 * PS;
-  static constexpr int KV_STAGES = KV_AVAIL / KV_STAGE > 3 ? 3 : KV_AVAIL / KV_STAGE;
-  static constexpr int KV_SMEM = 1024 + 2 * BIG + KV_STAGES * KV_STAGE + 4 * PS + BAR_BYTES;
+  static constexpr int KV_STAGES = KV_AVAIL / (KV_STAGE_A + KV_STAGE_B) > 4 ? 4 : KV_AVAIL / (KV_STAGE_A + KV_STAGE_B);
+  static constexpr int KV_SMEM = 1024 + 2 * BIG + KV_STAGES * (KV_STAGE_A + KV_STAGE_B) + 4 * PS + BAR_BYTES;
   static constexpr int TMEM_COLS = 512;
   static_assert(C0 == 32 || C0 == 64, "chunk 0 width");
   static_assert(C1 == 0 || C1 == 16 || C1 == 32 || C1 == 64, "chunk 1 width");
   static_assert(D % 16 == 0 && D <= 128, "head_dim");
-  static_assert(KV_STAGES >= 2, "shared memory");
+  static_assert(KV_STAGES >= 2 && DQ_STAGES >= 3, "shared memory");
   static_assert(DQ_SMEM <= LIMIT && KV_SMEM <= LIMIT, "shared memory");
   static_assert(BIG % 1024 == 0 && SMALL % 1024 == 0 && TR % 1024 == 0 && (BR * C0 * 2) % 1024 == 0 &&
                     (BS * C0 * 2) % 1024 == 0,
@@ -172,8 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(&s_full[u], 1);
-      mbar_init(&s_free[u], 128);
-      mbar_init(&ds_full[u], 128);
+      mbar_init(&s_free[u], kCompute);
+      mbar_init(&ds_full[u], kCompute);
       mbar_init(&dq_done[u], 1);
     }
     mbar_init(drain, 1);
@@ -273,7 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (!skip) {
-    // ------------------------------------------------------- one query row per thread
+    // --------------------------- one query row per thread, half of each step's columns
+    const int grp = (warp - 2) >> 2;  // columns [32 grp, 32 grp + 32) of every step
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -295,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       uint8_t* ds_tile = sdS + u * S::PS;
-#pragma unroll
-      for (int c0 = 0; c0 < S::BS; c0 += 32) {
+      {
+        const int c0 = grp * 32;
         uint32_t sr[32], pr[32];
         tmem_ld32(tmem + lane_off + u * 128 + c0, sr);
         tmem_ld32(tmem + lane_off + u * 128 + 64 + c0, pr);
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&ds_full[u]);
     }
     if (ok) ok = mbar_wait(&dq_done[(nk - 1) & 1], ((nk - 1) >> 1) & 1, abort_flag, &g_attn_bwd_err);
-    if (ok) {
+    if (ok && grp == 0) {
       tc_fence_after();
       float v[D];
       load_cols<D>(tmem + lane_off + 256, v);
@@ -358,14 +366,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + S::BIG;
-  uint8_t* sStage = sV + S::BIG;  // per stage: Q [64 x D], dO [64 x D], Q^T [D x 64], dO^T [D x 64]
-  uint8_t* sP = sStage + ST * S::KV_STAGE;  // [2] P^T tiles, then [2] dS^T tiles
+  uint8_t* sA = sV + S::BIG;                // ring A, per stage: Q [64 x D], dO [64 x D]
+  uint8_t* sB = sA + ST * S::KV_STAGE_A;    // ring B, per stage: Q^T [D x 64], dO^T [D x 64]
+  uint8_t* sP = sB + ST * S::KV_STAGE_B;    // [2] P^T tiles, then [2] dS^T tiles
   uint8_t* sdS = sP + 2 * S::PS;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sdS + 2 * S::PS);
   uint64_t* fixed_full = bar;
-  uint64_t* st_full = bar + 1;
-  uint64_t* st_empty = st_full + ST;
-  uint64_t* s_full = st_empty + ST;  // [2]
+  uint64_t* a_full = bar + 1;
+  uint64_t* a_empty = a_full + ST;
+  uint64_t* b_full = a_empty + ST;
+  uint64_t* b_empty = b_full + ST;
+  uint64_t* s_full = b_empty + ST;  // [2]
   uint64_t* s_free = s_full + 2;
   uint64_t* pd_full = s_free + 2;
   uint64_t* pd_done = pd_full + 2;
@@ -382,14 +393,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(fixed_full, 1);
     for (int s = 0; s < ST; ++s) {
-      mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
+      mbar_init(&a_full[s], 1);
+      mbar_init(&a_empty[s], 1);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
       armed[s] = -1;
+      armed[ST + 1 + s] = -1;
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(&s_full[u], 1);
-      mbar_init(&s_free[u], 128);
-      mbar_init(&pd_full[u], 128);
+      mbar_init(&s_free[u], kCompute);
+      mbar_init(&pd_full[u], kCompute);
       mbar_init(&pd_done[u], 1);
     }
     mbar_init(drain, 1);
@@ -416,29 +430,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sV, &tmV0, fixed_full, 0, k_row);
       if (S::C1) tma_load_2d(sV + S::BR * S::C0 * 2, &tmV1, fixed_full, S::C0, k_row);
       armed[ST] = 0;
-      for (int i = 0; i < nq; ++i) {
-        const int s = i % ST;
-        const uint32_t ph = (i / ST) & 1;
-        if (!mbar_wait(&st_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) break;
-        uint8_t* sQ = sStage + s * S::KV_STAGE;
-        uint8_t* sdO = sQ + S::SMALL;
-        uint8_t* sQT = sdO + S::SMALL;
-        uint8_t* sOT = sQT + S::TR;
-        const int q_row = bh * N + i * S::BS;
-        const int o_row = b * N + i * S::BS;
-        mbar_arrive_expect_tx(&st_full[s], S::KV_STAGE);
-        tma_load_2d(sQ, &tmQ0, &st_full[s], 0, q_row);
-        if (S::C1) tma_load_2d(sQ + S::BS * S::C0 * 2, &tmQ1, &st_full[s], S::C0, q_row);
-        tma_load_2d(sdO, &tmO0, &st_full[s], h * D, o_row);
-        if (S::C1) tma_load_2d(sdO + S::BS * S::C0 * 2, &tmO1, &st_full[s], h * D + S::C0, o_row);
-        tma_load_2d(sQT, &tmQT, &st_full[s], i * S::BS, bh * D);
-        tma_load_2d(sOT, &tmOT, &st_full[s], i * S::BS, bh * D);
-        armed[s] = static_cast<int>(ph);
+      // Ring B trails ring A by one step: its tiles are read a step later.
+      bool go = true;
+      for (int i = 0; go && i <= nq; ++i) {
+        if (i < nq) {
+          const int s = i % ST;
+          const uint32_t ph = (i / ST) & 1;
+          if (!mbar_wait(&a_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) break;
+          uint8_t* sQ = sA + s * S::KV_STAGE_A;
+          uint8_t* sdO = sQ + S::SMALL;
+          const int q_row = bh * N + i * S::BS;
+          const int o_row = b * N + i * S::BS;
+          mbar_arrive_expect_tx(&a_full[s], S::KV_STAGE_A);
+          tma_load_2d(sQ, &tmQ0, &a_full[s], 0, q_row);
+          if (S::C1) tma_load_2d(sQ + S::BS * S::C0 * 2, &tmQ1, &a_full[s], S::C0, q_row);
+          tma_load_2d(sdO, &tmO0, &a_full[s], h * D, o_row);
+          if (S::C1) tma_load_2d(sdO + S::BS * S::C0 * 2, &tmO1, &a_full[s], h * D + S::C0, o_row);
+          armed[s] = static_cast<int>(ph);
+        }
+        if (i >= 1) {
+          const int ib = i - 1, s = ib % ST;
+          const uint32_t ph = (ib / ST) & 1;
+          if (!mbar_wait(&b_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) {
+            go = false;
+            break;
+          }
+          uint8_t* sQT = sB + s * S::KV_STAGE_B;
+          uint8_t* sOT = sQT + S::TR;
+          mbar_arrive_expect_tx(&b_full[s], S::KV_STAGE_B);
+          tma_load_2d(sQT, &tmQT, &b_full[s], ib * S::BS, bh * D);
+          tma_load_2d(sOT, &tmOT, &b_full[s], ib * S::BS, bh * D);
+          armed[ST + 1 + s] = static_cast<int>(ph);
+        }
       }
       if (*abort_flag) {
         if (armed[ST] >= 0) drain_wait(fixed_full, 0);
-        for (int s = 0; s < ST; ++s)
-          if (armed[s] >= 0) drain_wait(&st_full[s], static_cast<uint32_t>(armed[s]));
+        for (int s = 0; s < ST; ++s) {
+          if (armed[s] >= 0) drain_wait(&a_full[s], static_cast<uint32_t>(armed[s]));
+          if (armed[ST + 1 + s] >= 0) drain_wait(&b_full[s], static_cast<uint32_t>(armed[ST + 1 + s]));
+        }
       }
     }
   } else if (!skip && warp == 1) {
@@ -450,11 +480,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dV += P^T_i dO_i, dK += dS^T_i Q_i
       auto issue_kv = [&](int i) -> bool {
         const int u = i & 1;
+        if (!mbar_wait(&b_full[i % ST], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) return false;
         if (!mbar_wait(&pd_full[u], (i >> 1) & 1, abort_flag, &g_attn_bwd_err)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(sP + u * S::PS), da = smem_u32(sdS + u * S::PS);
-        const uint32_t st = smem_u32(sStage + (i % ST) * S::KV_STAGE);
-        const uint32_t qt_ = st + 2 * S::SMALL, ot = qt_ + S::TR;
+        const uint32_t qt_ = smem_u32(sB + (i % ST) * S::KV_STAGE_B), ot = qt_ + S::TR;
 #pragma unroll
         for (int ks = 0; ks < S::BS / 16; ++ks)
           umma_bf16(tmem + 256, wdesc(pa, ks), wdesc(ot, ks), idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
@@ -462,12 +492,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < S::BS / 16; ++ks)
           umma_bf16(tmem + 384, wdesc(da, ks), wdesc(qt_, ks), idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&pd_done[u]);
-        umma_commit(&st_empty[i % ST]);
+        umma_commit(&b_empty[i % ST]);
         return true;
       };
       for (int i = 0; ok && i < nq; ++i) {
         const int s = i % ST, u = i & 1;
-        if (!mbar_wait(&st_full[s], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) {
+        if (!mbar_wait(&a_full[s], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) {
           ok = false;
           break;
         }
@@ -477,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t kk = smem_u32(sK), kv = smem_u32(sV);
-        const uint32_t kq = smem_u32(sStage + s * S::KV_STAGE), ko = kq + S::SMALL;
+        const uint32_t kq = smem_u32(sA + s * S::KV_STAGE_A), ko = kq + S::SMALL;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           umma_bf16(tmem + u * 128, kdesc<D, 128>(kk, ks), kdesc<D, 64>(kq, ks), idesc_s, ks > 0 ? 1u : 0u);
@@ -486,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kv, ks), kdesc<D, 64>(ko, ks), idesc_s, ks > 0 ? 1u : 0u);
         issued = true;
         umma_commit(&s_full[u]);
+        umma_commit(&a_empty[s]);
         if (i >= 1) ok = issue_kv(i - 1);
       }
       if (ok) ok = issue_kv(nq - 1);
@@ -495,7 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (!skip) {
-    // --------------------------------------------------------- one key row per thread
+    // ----------------------------- one key row per thread, half of each step's columns
+    const int grp = (warp - 2) >> 2;  // columns [32 grp, 32 grp + 32) of every step
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -518,8 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint8_t* p_tile = sP + u * S::PS;
       uint8_t* d_tile = sdS + u * S::PS;
-#pragma unroll
-      for (int c0 = 0; c0 < S::BS; c0 += 32) {
+      {
+        const int c0 = grp * 32;
         uint32_t sr[32], pr[32];
         tmem_ld32(tmem + lane_off + u * 128 + c0, sr);
         tmem_ld32(tmem + lane_off + u * 128 + 64 + c0, pr);
@@ -557,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int width = p.H * D;
       bf16* row = static_cast<bf16*>(p.dqkv) + (static_cast<size_t>(b) * N + n) * p.ld_dqkv;
-      {
+      if (grp == 0) {  // dK
         float v[D];
         load_cols<D>(tmem + lane_off + 384, v);
         if (row_ok) {
@@ -569,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(v + 8 * g);
         }
       }
-      {
+      if (grp == 1) {  // dV
         float v[D];
         load_cols<D>(tmem + lane_off + 256, v);
         if (row_ok) {
