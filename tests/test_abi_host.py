@@ -204,8 +204,10 @@ def test_preprocess_argument_checks_need_no_device():
 
 
 def test_backward_argument_checks_need_no_device():
+    # v^T [B, H, D, ceil8(N)], the recomputed output [B*N, H*D], log-sum-exp and delta
+    # [B*H, ceil64(N)] fp32: linear in N, no N^2 term
     assert V.vt_attention_backward_workspace_bytes(2, 16, 100, 80) == \
-        4 * ((2 * 16 * 80 * 104 * 2 + 255) // 256 * 256) + (2 * 100 * 16 * 80 * 2 + 255) // 256 * 256 + \
+        (2 * 16 * 80 * 104 * 2 + 255) // 256 * 256 + (2 * 100 * 16 * 80 * 2 + 255) // 256 * 256 + \
         2 * ((2 * 16 * 128 * 4 + 255) // 256 * 256)
     for D, code in ((64, "VT_ERR_UNSUPPORTED"), (80, "VT_ERR_WORKSPACE")):
         with pytest.raises(V.VtError) as e:

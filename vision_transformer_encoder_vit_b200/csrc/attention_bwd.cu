@@ -12,17 +12,21 @@
 // "v2_loaders - Differentiable Vision Tower Loaders (spark2)" (summary, section 3)
 // backpropagate through it to the image.
 //
-// Two kernels, every MMA operand K-major (transposed copies qT, kT, dOT are made
-// beforehand), one CTA = 10 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// Two kernels, one CTA = 10 warps: warp 0 issues TMA loads, warp 1 owns TMEM and issues
 // the MMAs from one thread, warps 2..9 are two groups of four that each own one row per
 // thread and split every 64-column step between them (columns 0..31 and 32..63), so two
 // warps per SM sub-partition hide each other's latencies.
-//  * attn_bwd_dq: one CTA per 128 queries; 64-key steps stream K, V and K^T.
+//  * attn_bwd_dq: one CTA per 128 queries; 64-key steps stream K and V^T.
 //        S = Q K_j^T, dP = dO V_j^T  (TMEM, double-buffered)  -> dS (bf16, shared)
 //        dQ += dS K_j                (TMEM accumulator)
-//  * attn_bwd_dkdv: one CTA per 128 keys; 64-query steps stream Q, dO, Q^T, dO^T.
+//  * attn_bwd_dkdv: one CTA per 128 keys; 64-query steps stream Q and dO.
 //        S^T = K Q_i^T, dP^T = V dO_i^T                      -> P^T, dS^T (bf16, shared)
 //        dV += P^T dO_i, dK += dS^T Q_i
+// A tile staged once serves both products that read it: the row-major [64 x D] tiles of
+// K, Q and dO are the K-major B operand of the score products and, read MN-major (the
+// MMA's B-transpose bit), the B operand of dQ, dK and dV; the [D x 64] tile of v^T is the
+// MN-major B operand of dP.  So no transposed copy is made and every operand byte
+// crosses from L2 once per step.
 #include <math.h>
 
 #include "internal.h"
@@ -53,25 +57,23 @@ struct BwdShape {
   static constexpr int SBO0 = 8 * SW0, SBO1 = 8 * SW1;
   static constexpr int BR = 128;            // rows a CTA owns (queries or keys)
   static constexpr int BS = 64;             // rows streamed per step
-  static constexpr int BIG = BR * D * 2;    // [128 x D] K-major tile
-  static constexpr int SMALL = BS * D * 2;  // [64 x D] K-major tile
-  static constexpr int TR = D * BS * 2;     // [D x 64] tile of a transposed operand
+  static constexpr int BIG = BR * D * 2;    // [128 x D] row-major tile
+  static constexpr int SMALL = BS * D * 2;  // [64 x D] row-major tile
+  static constexpr int TR = D * BS * 2;     // [D x 64] tile of v^T
   static constexpr int PS = BR * BS * 2;    // [128 x 64] bf16 tile written by the threads
   static constexpr int BAR_BYTES = 256;
   static constexpr int LIMIT = 232448;
-  // attn_bwd_dq: fixed Q, dO; per stage K, V, K^T; dS double-buffered
-  static constexpr int DQ_STAGE = 2 * SMALL + TR;
+  static constexpr int MAX_STAGES = 6;
+  // attn_bwd_dq: fixed Q, dO; per stage K, V^T; dS double-buffered
+  static constexpr int DQ_STAGE = SMALL + TR;
   static constexpr int DQ_AVAIL = LIMIT - 1024 - BAR_BYTES - 2 * BIG - 2 * PS;
-  static constexpr int DQ_STAGES = DQ_AVAIL / DQ_STAGE > 6 ? 6 : DQ_AVAIL / DQ_STAGE;
+  static constexpr int DQ_STAGES = DQ_AVAIL / DQ_STAGE > MAX_STAGES ? MAX_STAGES : DQ_AVAIL / DQ_STAGE;
   static constexpr int DQ_SMEM = 1024 + 2 * BIG + DQ_STAGES * DQ_STAGE + 2 * PS + BAR_BYTES;
-  // attn_bwd_dkdv: fixed K, V; ring A holds Q, dO (read by the S^T, dP^T products and
-  // released right after them), ring B holds Q^T, dO^T (read by dV, dK); P^T and dS^T
-  // double-buffered
-  static constexpr int KV_STAGE_A = 2 * SMALL;
-  static constexpr int KV_STAGE_B = 2 * TR;
+  // attn_bwd_dkdv: fixed K, V; per stage Q, dO; P^T and dS^T double-buffered
+  static constexpr int KV_STAGE = 2 * SMALL;
   static constexpr int KV_AVAIL = LIMIT - 1024 - BAR_BYTES - 2 * BIG - 4 * PS;
-  static constexpr int KV_STAGES = KV_AVAIL / (KV_STAGE_A + KV_STAGE_B) > 4 ? 4 : KV_AVAIL / (KV_STAGE_A + KV_STAGE_B);
-  static constexpr int KV_SMEM = 1024 + 2 * BIG + KV_STAGES * (KV_STAGE_A + KV_STAGE_B) + 4 * PS + BAR_BYTES;
+  static constexpr int KV_STAGES = KV_AVAIL / KV_STAGE > MAX_STAGES ? MAX_STAGES : KV_AVAIL / KV_STAGE;
+  static constexpr int KV_SMEM = 1024 + 2 * BIG + KV_STAGES * KV_STAGE + 4 * PS + BAR_BYTES;
   static constexpr int TMEM_COLS = 512;
   static_assert(C0 == 32 || C0 == 64, "chunk 0 width");
   static_assert(C1 == 0 || C1 == 16 || C1 == 32 || C1 == 64, "chunk 1 width");
@@ -95,6 +97,23 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t tile, int ks) {
 
 // Descriptor of K-step ks (16 columns) of a [rows x 64] tile with 128-byte rows.
 __device__ __forceinline__ uint64_t wdesc(uint32_t tile, int ks) { return smem_desc(tile + ks * 32, 1024, 2); }
+
+// The same row-major [64 x D] tile read MN-major: K runs down the 64 rows, N along the
+// channels.  Chunk c (0: channels [0, C0), 1: [C0, D)) is one swizzle atom wide in N, so
+// only the start address (16 rows per K-step) and the 8-row stride SBO matter.
+template <int D, int chunk>
+__device__ __forceinline__ uint64_t mndesc(uint32_t tile, int ks) {
+  using S = BwdShape<D>;
+  if (chunk == 0) return smem_desc(tile + ks * 16 * S::SW0, S::SBO0, S::LAY0);
+  return smem_desc(tile + S::BS * S::C0 * 2 + ks * 16 * S::SW1, S::SBO1, S::LAY1);
+}
+
+// A [D x 64] tile of v^T with 128-byte rows, read as an MN-major operand (N = 64 keys
+// along a row, K = channels down the rows): 16 rows per K-step.
+__device__ __forceinline__ uint64_t vtdesc(uint32_t tile, int ks) { return smem_desc(tile + ks * 2048, 1024, 2); }
+
+// Instruction descriptor with the B operand MN-major (bit 16).
+__host__ __device__ constexpr uint32_t idesc_bmn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 16); }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
@@ -141,8 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
                 const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                 const __grid_constant__ CUtensorMap tmK0, const __grid_constant__ CUtensorMap tmK1,
-                const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmV1,
-                const __grid_constant__ CUtensorMap tmKT, const AttnBwdParams p) {
+                const __grid_constant__ CUtensorMap tmVT, const AttnBwdParams p) {
   constexpr int D = HL::D;
   using S = BwdShape<D>;
   constexpr int ST = S::DQ_STAGES;
@@ -150,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sdO = sQ + S::BIG;
-  uint8_t* sStage = sdO + S::BIG;  // per stage: K [64 x D], V [64 x D], K^T [D x 64]
+  uint8_t* sStage = sdO + S::BIG;  // per stage: K [64 x D], V^T [D x 64]
   uint8_t* sdS = sStage + ST * S::DQ_STAGE;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sdS + 2 * S::PS);
   uint64_t* fixed_full = bar;
@@ -213,15 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (j / ST) & 1;
         if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) break;
         uint8_t* sK = sStage + s * S::DQ_STAGE;
-        uint8_t* sV = sK + S::SMALL;
-        uint8_t* sKT = sV + S::SMALL;
+        uint8_t* sVT = sK + S::SMALL;
         const int k_row = bh * N + j * S::BS;
         mbar_arrive_expect_tx(&kv_full[s], S::DQ_STAGE);
         tma_load_2d(sK, &tmK0, &kv_full[s], 0, k_row);
         if (S::C1) tma_load_2d(sK + S::BS * S::C0 * 2, &tmK1, &kv_full[s], S::C0, k_row);
-        tma_load_2d(sV, &tmV0, &kv_full[s], 0, k_row);
-        if (S::C1) tma_load_2d(sV + S::BS * S::C0 * 2, &tmV1, &kv_full[s], S::C0, k_row);
-        tma_load_2d(sKT, &tmKT, &kv_full[s], j * S::BS, bh * D);
+        tma_load_2d(sVT, &tmVT, &kv_full[s], j * S::BS, bh * D);
         armed[s] = static_cast<int>(ph);
       }
       if (*abort_flag) {
@@ -233,19 +248,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (!skip && warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BS);
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D);
+      constexpr uint32_t idesc_p = idesc_bmn(128, S::BS);
+      constexpr uint32_t idesc_q0 = idesc_bmn(128, S::C0);
+      constexpr uint32_t idesc_q1 = idesc_bmn(128, S::C1 ? S::C1 : 16);
       bool issued = false;
       bool ok = mbar_wait(fixed_full, 0, abort_flag, &g_attn_bwd_err);
-      // dQ += dS_i K_i
+      // dQ += dS_i K_i, K_i read MN-major from its row-major tile (channel chunks)
       auto issue_dq = [&](int i) -> bool {
         const int u = i & 1;
         if (!mbar_wait(&ds_full[u], (i >> 1) & 1, abort_flag, &g_attn_bwd_err)) return false;
         tc_fence_after();
         const uint32_t a = smem_u32(sdS + u * S::PS);
-        const uint32_t bt = smem_u32(sStage + (i % ST) * S::DQ_STAGE + 2 * S::SMALL);
+        const uint32_t kk = smem_u32(sStage + (i % ST) * S::DQ_STAGE);
 #pragma unroll
-        for (int ks = 0; ks < S::BS / 16; ++ks)
-          umma_bf16(tmem + 256, wdesc(a, ks), wdesc(bt, ks), idesc_q, (i > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < S::BS / 16; ++ks) {
+          const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
+          umma_bf16(tmem + 256, wdesc(a, ks), mndesc<D, 0>(kk, ks), idesc_q0, acc);
+          if (S::C1) umma_bf16(tmem + 256 + S::C0, wdesc(a, ks), mndesc<D, 1>(kk, ks), idesc_q1, acc);
+        }
         umma_commit(&dq_done[u]);
         umma_commit(&kv_empty[i % ST]);
         return true;
@@ -262,13 +282,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t kq = smem_u32(sQ), kd = smem_u32(sdO);
-        const uint32_t kk = smem_u32(sStage + s * S::DQ_STAGE), kv = kk + S::SMALL;
+        const uint32_t kk = smem_u32(sStage + s * S::DQ_STAGE), kvt = kk + S::SMALL;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           umma_bf16(tmem + u * 128, kdesc<D, 128>(kq, ks), kdesc<D, 64>(kk, ks), idesc_s, ks > 0 ? 1u : 0u);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kd, ks), kdesc<D, 64>(kv, ks), idesc_s, ks > 0 ? 1u : 0u);
+          umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kd, ks), vtdesc(kvt, ks), idesc_p, ks > 0 ? 1u : 0u);
         issued = true;
         umma_commit(&s_full[u]);
         if (j >= 1) ok = issue_dq(j - 1);
@@ -357,7 +377,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmV1,
                   const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
                   const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
-                  const __grid_constant__ CUtensorMap tmQT, const __grid_constant__ CUtensorMap tmOT,
                   const AttnBwdParams p) {
   constexpr int D = HL::D;
   using S = BwdShape<D>;
@@ -366,17 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + S::BIG;
-  uint8_t* sA = sV + S::BIG;                // ring A, per stage: Q [64 x D], dO [64 x D]
-  uint8_t* sB = sA + ST * S::KV_STAGE_A;    // ring B, per stage: Q^T [D x 64], dO^T [D x 64]
-  uint8_t* sP = sB + ST * S::KV_STAGE_B;    // [2] P^T tiles, then [2] dS^T tiles
+  uint8_t* sStage = sV + S::BIG;           // per stage: Q [64 x D], dO [64 x D]
+  uint8_t* sP = sStage + ST * S::KV_STAGE;  // [2] P^T tiles, then [2] dS^T tiles
   uint8_t* sdS = sP + 2 * S::PS;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sdS + 2 * S::PS);
   uint64_t* fixed_full = bar;
-  uint64_t* a_full = bar + 1;
-  uint64_t* a_empty = a_full + ST;
-  uint64_t* b_full = a_empty + ST;
-  uint64_t* b_empty = b_full + ST;
-  uint64_t* s_full = b_empty + ST;  // [2]
+  uint64_t* st_full = bar + 1;
+  uint64_t* st_empty = st_full + ST;
+  uint64_t* s_full = st_empty + ST;  // [2]
   uint64_t* s_free = s_full + 2;
   uint64_t* pd_full = s_free + 2;
   uint64_t* pd_done = pd_full + 2;
@@ -393,12 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(fixed_full, 1);
     for (int s = 0; s < ST; ++s) {
-      mbar_init(&a_full[s], 1);
-      mbar_init(&a_empty[s], 1);
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
       armed[s] = -1;
-      armed[ST + 1 + s] = -1;
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(&s_full[u], 1);
@@ -430,74 +443,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sV, &tmV0, fixed_full, 0, k_row);
       if (S::C1) tma_load_2d(sV + S::BR * S::C0 * 2, &tmV1, fixed_full, S::C0, k_row);
       armed[ST] = 0;
-      // Ring B trails ring A by one step: its tiles are read a step later.
-      bool go = true;
-      for (int i = 0; go && i <= nq; ++i) {
-        if (i < nq) {
-          const int s = i % ST;
-          const uint32_t ph = (i / ST) & 1;
-          if (!mbar_wait(&a_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) break;
-          uint8_t* sQ = sA + s * S::KV_STAGE_A;
-          uint8_t* sdO = sQ + S::SMALL;
-          const int q_row = bh * N + i * S::BS;
-          const int o_row = b * N + i * S::BS;
-          mbar_arrive_expect_tx(&a_full[s], S::KV_STAGE_A);
-          tma_load_2d(sQ, &tmQ0, &a_full[s], 0, q_row);
-          if (S::C1) tma_load_2d(sQ + S::BS * S::C0 * 2, &tmQ1, &a_full[s], S::C0, q_row);
-          tma_load_2d(sdO, &tmO0, &a_full[s], h * D, o_row);
-          if (S::C1) tma_load_2d(sdO + S::BS * S::C0 * 2, &tmO1, &a_full[s], h * D + S::C0, o_row);
-          armed[s] = static_cast<int>(ph);
-        }
-        if (i >= 1) {
-          const int ib = i - 1, s = ib % ST;
-          const uint32_t ph = (ib / ST) & 1;
-          if (!mbar_wait(&b_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) {
-            go = false;
-            break;
-          }
-          uint8_t* sQT = sB + s * S::KV_STAGE_B;
-          uint8_t* sOT = sQT + S::TR;
-          mbar_arrive_expect_tx(&b_full[s], S::KV_STAGE_B);
-          tma_load_2d(sQT, &tmQT, &b_full[s], ib * S::BS, bh * D);
-          tma_load_2d(sOT, &tmOT, &b_full[s], ib * S::BS, bh * D);
-          armed[ST + 1 + s] = static_cast<int>(ph);
-        }
+      for (int i = 0; i < nq; ++i) {
+        const int s = i % ST;
+        const uint32_t ph = (i / ST) & 1;
+        if (!mbar_wait(&st_empty[s], ph ^ 1u, abort_flag, &g_attn_bwd_err)) break;
+        uint8_t* sQ = sStage + s * S::KV_STAGE;
+        uint8_t* sdO = sQ + S::SMALL;
+        const int q_row = bh * N + i * S::BS;
+        const int o_row = b * N + i * S::BS;
+        mbar_arrive_expect_tx(&st_full[s], S::KV_STAGE);
+        tma_load_2d(sQ, &tmQ0, &st_full[s], 0, q_row);
+        if (S::C1) tma_load_2d(sQ + S::BS * S::C0 * 2, &tmQ1, &st_full[s], S::C0, q_row);
+        tma_load_2d(sdO, &tmO0, &st_full[s], h * D, o_row);
+        if (S::C1) tma_load_2d(sdO + S::BS * S::C0 * 2, &tmO1, &st_full[s], h * D + S::C0, o_row);
+        armed[s] = static_cast<int>(ph);
       }
       if (*abort_flag) {
         if (armed[ST] >= 0) drain_wait(fixed_full, 0);
-        for (int s = 0; s < ST; ++s) {
-          if (armed[s] >= 0) drain_wait(&a_full[s], static_cast<uint32_t>(armed[s]));
-          if (armed[ST + 1 + s] >= 0) drain_wait(&b_full[s], static_cast<uint32_t>(armed[ST + 1 + s]));
-        }
+        for (int s = 0; s < ST; ++s)
+          if (armed[s] >= 0) drain_wait(&st_full[s], static_cast<uint32_t>(armed[s]));
       }
     }
   } else if (!skip && warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BS);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D);
+      constexpr uint32_t idesc_o0 = idesc_bmn(128, S::C0);
+      constexpr uint32_t idesc_o1 = idesc_bmn(128, S::C1 ? S::C1 : 16);
       bool issued = false;
       bool ok = mbar_wait(fixed_full, 0, abort_flag, &g_attn_bwd_err);
-      // dV += P^T_i dO_i, dK += dS^T_i Q_i
+      // dV += P^T_i dO_i, dK += dS^T_i Q_i; dO_i and Q_i read MN-major (channel chunks)
       auto issue_kv = [&](int i) -> bool {
         const int u = i & 1;
-        if (!mbar_wait(&b_full[i % ST], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) return false;
         if (!mbar_wait(&pd_full[u], (i >> 1) & 1, abort_flag, &g_attn_bwd_err)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(sP + u * S::PS), da = smem_u32(sdS + u * S::PS);
-        const uint32_t qt_ = smem_u32(sB + (i % ST) * S::KV_STAGE_B), ot = qt_ + S::TR;
+        const uint32_t kq = smem_u32(sStage + (i % ST) * S::KV_STAGE), ko = kq + S::SMALL;
 #pragma unroll
-        for (int ks = 0; ks < S::BS / 16; ++ks)
-          umma_bf16(tmem + 256, wdesc(pa, ks), wdesc(ot, ks), idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
-#pragma unroll
-        for (int ks = 0; ks < S::BS / 16; ++ks)
-          umma_bf16(tmem + 384, wdesc(da, ks), wdesc(qt_, ks), idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < S::BS / 16; ++ks) {
+          const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
+          umma_bf16(tmem + 256, wdesc(pa, ks), mndesc<D, 0>(ko, ks), idesc_o0, acc);
+          if (S::C1) umma_bf16(tmem + 256 + S::C0, wdesc(pa, ks), mndesc<D, 1>(ko, ks), idesc_o1, acc);
+          umma_bf16(tmem + 384, wdesc(da, ks), mndesc<D, 0>(kq, ks), idesc_o0, acc);
+          if (S::C1) umma_bf16(tmem + 384 + S::C0, wdesc(da, ks), mndesc<D, 1>(kq, ks), idesc_o1, acc);
+        }
         umma_commit(&pd_done[u]);
-        umma_commit(&b_empty[i % ST]);
+        umma_commit(&st_empty[i % ST]);
         return true;
       };
       for (int i = 0; ok && i < nq; ++i) {
         const int s = i % ST, u = i & 1;
-        if (!mbar_wait(&a_full[s], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) {
+        if (!mbar_wait(&st_full[s], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) {
           ok = false;
           break;
         }
@@ -507,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t kk = smem_u32(sK), kv = smem_u32(sV);
-        const uint32_t kq = smem_u32(sA + s * S::KV_STAGE_A), ko = kq + S::SMALL;
+        const uint32_t kq = smem_u32(sStage + s * S::KV_STAGE), ko = kq + S::SMALL;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           umma_bf16(tmem + u * 128, kdesc<D, 128>(kk, ks), kdesc<D, 64>(kq, ks), idesc_s, ks > 0 ? 1u : 0u);
@@ -516,7 +511,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kv, ks), kdesc<D, 64>(ko, ks), idesc_s, ks > 0 ? 1u : 0u);
         issued = true;
         umma_commit(&s_full[u]);
-        umma_commit(&a_empty[s]);
         if (i >= 1) ok = issue_kv(i - 1);
       }
       if (ok) ok = issue_kv(nq - 1);
@@ -636,9 +630,9 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   }
   const uint64_t rows = static_cast<uint64_t>(p.B) * p.H * p.N;  // rows of q, k, v [B, H, N, D]
   const uint64_t tok = static_cast<uint64_t>(p.B) * p.N;          // rows of dO [B * N, H * D]
-  const uint64_t trows = static_cast<uint64_t>(p.B) * p.H * D;    // rows of qT, kT, dOT [B, H, D, ld]
+  const uint64_t trows = static_cast<uint64_t>(p.B) * p.H * D;    // rows of v^T [B, H, D, ld]
   CUtensorMap q0_128, q1_128, o0_128, o1_128, q0_64, q1_64, o0_64, o1_64;
-  CUtensorMap k0_64, k1_64, v0_64, v1_64, k0_128, k1_128, v0_128, v1_128, kT, qT, oT;
+  CUtensorMap k0_64, k1_64, k0_128, k1_128, v0_128, v1_128, vT;
   auto mk = [&](CUtensorMap* m, const void* base, uint64_t r, uint64_t ld, int box_rows, int col0_width, int sw) {
     return make_tmap_2d(m, base, r, ld, ld, box_rows, col0_width, sw);
   };
@@ -646,7 +640,7 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   const int C0 = S::C0, C1 = S::C1;
   ok = ok && mk(&q0_128, p.q, rows, D, 128, C0, S::SW0) && mk(&q0_64, p.q, rows, D, 64, C0, S::SW0);
   ok = ok && mk(&k0_128, p.k, rows, D, 128, C0, S::SW0) && mk(&k0_64, p.k, rows, D, 64, C0, S::SW0);
-  ok = ok && mk(&v0_128, p.v, rows, D, 128, C0, S::SW0) && mk(&v0_64, p.v, rows, D, 64, C0, S::SW0);
+  ok = ok && mk(&v0_128, p.v, rows, D, 128, C0, S::SW0);
   ok = ok && make_tmap_2d(&o0_128, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 128,
                           C0, S::SW0);
   ok = ok && make_tmap_2d(&o0_64, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 64, C0,
@@ -654,28 +648,25 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   if (C1) {
     ok = ok && mk(&q1_128, p.q, rows, D, 128, C1, S::SW1) && mk(&q1_64, p.q, rows, D, 64, C1, S::SW1);
     ok = ok && mk(&k1_128, p.k, rows, D, 128, C1, S::SW1) && mk(&k1_64, p.k, rows, D, 64, C1, S::SW1);
-    ok = ok && mk(&v1_128, p.v, rows, D, 128, C1, S::SW1) && mk(&v1_64, p.v, rows, D, 64, C1, S::SW1);
+    ok = ok && mk(&v1_128, p.v, rows, D, 128, C1, S::SW1);
     ok = ok && make_tmap_2d(&o1_128, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 128,
                             C1, S::SW1);
     ok = ok && make_tmap_2d(&o1_64, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 64,
                             C1, S::SW1);
   } else {
-    q1_128 = q0_128, q1_64 = q0_64, k1_128 = k0_128, k1_64 = k0_64, v1_128 = v0_128, v1_64 = v0_64;
+    q1_128 = q0_128, q1_64 = q0_64, k1_128 = k0_128, k1_64 = k0_64, v1_128 = v0_128;
     o1_128 = o0_128, o1_64 = o0_64;
   }
-  // Transposed operands: [B*H*D rows, N columns] with row stride ld; columns past N read
-  // as zero, so padding never enters an MMA.
-  ok = ok && make_tmap_2d(&kT, p.kT, trows, p.N, p.ld, D, 64, 128);
-  ok = ok && make_tmap_2d(&qT, p.qT, trows, p.N, p.ld, D, 64, 128);
-  ok = ok && make_tmap_2d(&oT, p.dOT, trows, p.N, p.ld, D, 64, 128);
+  // v^T: [B*H*D rows, N columns] with row stride ld; columns past N read as zero, so
+  // padding never enters an MMA.
+  ok = ok && make_tmap_2d(&vT, p.vt, trows, p.N, p.ld, D, 64, 128);
   if (!ok) return cudaErrorInvalidValue;
   dim3 grid((p.N + S::BR - 1) / S::BR, p.H, p.B);
-  attn_bwd_dq<HL><<<grid, kThreads, S::DQ_SMEM, stream>>>(q0_128, q1_128, o0_128, o1_128, k0_64, k1_64, v0_64,
-                                                          v1_64, kT, p);
+  attn_bwd_dq<HL><<<grid, kThreads, S::DQ_SMEM, stream>>>(q0_128, q1_128, o0_128, o1_128, k0_64, k1_64, vT, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dkdv<HL><<<grid, kThreads, S::KV_SMEM, stream>>>(k0_128, k1_128, v0_128, v1_128, q0_64, q1_64, o0_64,
-                                                            o1_64, qT, oT, p);
+                                                            o1_64, p);
   return cudaGetLastError();
 }
 

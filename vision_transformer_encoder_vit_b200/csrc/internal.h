@@ -132,10 +132,8 @@ struct AttnBwdParams {
   const void* q;      // [B, H, N, D] bf16, rotated
   const void* k;      // [B, H, N, D] bf16, rotated
   const void* v;      // [B, H, N, D] bf16
-  const void* qT;     // [B, H, D, ld] bf16 (q transposed)
-  const void* kT;     // [B, H, D, ld]
+  const void* vt;     // [B, H, D, ld] bf16 (v transposed, as the forward uses it)
   const void* dO;     // [B*N, H*D] bf16, gradient of the attention output
-  const void* dOT;    // [B, H, D, ld]
   const float* lse;   // [B*H, ld_stats], from the forward
   const float* delta; // [B*H, ld_stats], rowsum(dO * O) per query
   int ld_stats;       // multiple of 64, >= N

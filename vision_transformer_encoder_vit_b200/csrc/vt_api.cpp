@@ -1168,7 +1168,7 @@ namespace {
 
 struct BwdPlan {
   int N, M, ld, lds;
-  size_t dx, xn, q, k, vt, a, x1, hmid, dO, qT, kT, dOT, v, dqkv, lse, delta, total;
+  size_t dx, xn, q, k, vt, a, x1, hmid, dO, v, dqkv, lse, delta, total;
 };
 
 BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
@@ -1196,9 +1196,6 @@ BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
   p.x1 = take(M * d * 2);
   p.hmid = take(M * std::max<size_t>(c.mlp, K0) * 2);
   p.dO = take(M * d * 2);
-  p.qT = take(headT * 2);
-  p.kT = take(headT * 2);
-  p.dOT = take(headT * 2);
   p.v = take(M * d * 2);
   p.dqkv = take(M * 3 * d * 2);
   p.lse = take(stats * 4);
@@ -1215,19 +1212,13 @@ vt_status run_layernorm_backward(const void* x, const void* g, const void* dy, c
   return VT_OK;
 }
 
-// q, k [B, H, N, D] -> [B, H, D, ld]; dO [B*N, H*D] -> [B, H, D, ld]; vt [B, H, D, ld_v] -> v [B, H, N, D].
-vt_status run_bwd_transposes(const void* q, const void* k, const void* dO, const void* vt, int ld_v, void* qT,
-                             void* kT, void* dOT, void* v, int B, int H, int N, int D, int ld, cudaStream_t st) {
-  ProfScope ps(CLS_BWD_MISC, 0, 16.0 * B * H * static_cast<double>(N) * D, st);
+// vt [B, H, D, ld] -> v [B, H, N, D]: the row-major v the dk/dv kernel reads as an
+// A operand.
+vt_status run_v_rows(const void* vt, int ld, void* v, int B, int H, int N, int D, cudaStream_t st) {
+  ProfScope ps(CLS_BWD_MISC, 0, 4.0 * B * H * static_cast<double>(N) * D, st);
   const long hnd = static_cast<long>(H) * N * D, nd = static_cast<long>(N) * D;
   const long hdl = static_cast<long>(H) * D * ld, dl = static_cast<long>(D) * ld;
-  cudaError_t e = launch_transpose(q, qT, B, H, N, D, hnd, nd, D, hdl, dl, ld, st);
-  if (e == cudaSuccess) e = launch_transpose(k, kT, B, H, N, D, hnd, nd, D, hdl, dl, ld, st);
-  if (e == cudaSuccess) e = launch_transpose(dO, dOT, B, H, N, D, hnd, D, static_cast<long>(H) * D, hdl, dl, ld, st);
-  if (e == cudaSuccess && vt) {
-    const long hdlv = static_cast<long>(H) * D * ld_v, dlv = static_cast<long>(D) * ld_v;
-    e = launch_transpose(vt, v, B, H, D, N, hdlv, dlv, ld_v, hnd, nd, D, st);
-  }
+  cudaError_t e = launch_transpose(vt, v, B, H, D, N, hdl, dl, ld, hnd, nd, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
   return VT_OK;
 }
@@ -1309,18 +1300,14 @@ vt_status run_layer_backward(vt_handle* h, int i, const void* x_in, int B, int g
                                            bp.lds, st);
     if (e != cudaSuccess) return cuda_fail(e, "delta launch");
   }
-  if ((s = run_bwd_transposes(w + bp.q, w + bp.k, w + bp.dO, w + bp.vt, bp.ld, w + bp.qT, w + bp.kT, w + bp.dOT,
-                              w + bp.v, B, H, N, D, bp.ld, st)))
-    return s;
+  if ((s = run_v_rows(w + bp.vt, bp.ld, w + bp.v, B, H, N, D, st))) return s;
   {
     AttnBwdParams a{};
     a.q = w + bp.q;
     a.k = w + bp.k;
     a.v = w + bp.v;
-    a.qT = w + bp.qT;
-    a.kT = w + bp.kT;
+    a.vt = w + bp.vt;
     a.dO = w + bp.dO;
-    a.dOT = w + bp.dOT;
     a.lse = reinterpret_cast<const float*>(w + bp.lse);
     a.delta = reinterpret_cast<const float*>(w + bp.delta);
     a.ld_stats = bp.lds;
@@ -1502,7 +1489,7 @@ vt_status vt_attention_backward_workspace_bytes(int B, int H, int N, int D, size
   const size_t ld = static_cast<size_t>(round8(N)), lds = (static_cast<size_t>(N) + 63) / 64 * 64;
   const size_t headT = static_cast<size_t>(B) * H * D * ld;
   const size_t tok = static_cast<size_t>(B) * N * H * D;
-  *out = 4 * align256(headT * 2) + align256(tok * 2) + 2 * align256(static_cast<size_t>(B) * H * lds * 4);
+  *out = align256(headT * 2) + align256(tok * 2) + 2 * align256(static_cast<size_t>(B) * H * lds * 4);
   return VT_OK;
 }
 
@@ -1523,10 +1510,7 @@ vt_status vt_attention_backward(const void* q, const void* k, const void* v, con
   const size_t tok = static_cast<size_t>(B) * N * H * D;
   char* w = static_cast<char*>(ws);
   void* vt_ = w;
-  void* qT = w + align256(headT * 2);
-  void* kT = static_cast<char*>(qT) + align256(headT * 2);
-  void* dOT = static_cast<char*>(kT) + align256(headT * 2);
-  void* o = static_cast<char*>(dOT) + align256(headT * 2);
+  void* o = w + align256(headT * 2);
   float* lse = reinterpret_cast<float*>(static_cast<char*>(o) + align256(tok * 2));
   float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse) + align256(static_cast<size_t>(B) * H * lds * 4));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1546,15 +1530,12 @@ vt_status vt_attention_backward(const void* q, const void* k, const void* v, con
     cudaError_t e = launch_attention_delta(dO, o, delta, B, N, H, D, lds, st);
     if (e != cudaSuccess) return cuda_fail(e, "delta launch");
   }
-  if ((s = run_bwd_transposes(q, k, dO, nullptr, 0, qT, kT, dOT, nullptr, B, H, N, D, ld, st))) return s;
   AttnBwdParams p{};
   p.q = q;
   p.k = k;
   p.v = v;
-  p.qT = qT;
-  p.kT = kT;
+  p.vt = vt_;
   p.dO = dO;
-  p.dOT = dOT;
   p.lse = lse;
   p.delta = delta;
   p.ld_stats = lds;
