@@ -44,7 +44,7 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-KERNEL_SOURCES = {"gemm": "gemm.cu", "attention": "attention.cu"}
+KERNEL_SOURCES = {"gemm": "gemm.cu", "attention": "attention.cu", "attention_backward": "attention_bwd.cu"}
 
 
 def recorded_traffic(cls: str, workload_name: str):
