@@ -69,8 +69,10 @@ struct BwdShape {
   static constexpr int DQ_AVAIL = LIMIT - 1024 - BAR_BYTES - 2 * BIG - 2 * PS;
   static constexpr int DQ_STAGES = DQ_AVAIL / DQ_STAGE > MAX_STAGES ? MAX_STAGES : DQ_AVAIL / DQ_STAGE;
   static constexpr int DQ_SMEM = 1024 + 2 * BIG + DQ_STAGES * DQ_STAGE + 2 * PS + BAR_BYTES;
-  // attn_bwd_dkdv: fixed K, V; per stage Q, dO; P^T and dS^T double-buffered
-  static constexpr int KV_STAGE = 2 * SMALL;
+  // attn_bwd_dkdv: fixed K, V; per stage Q, dO and the 64 queries' log-sum-exp and delta
+  // (fp32, in the stage's last 1024-byte block); P^T and dS^T double-buffered
+  static constexpr int KV_STATS = 2 * SMALL;  // offset of the statistics in a stage
+  static constexpr int KV_STAGE = 2 * SMALL + 1024;
   static constexpr int KV_AVAIL = LIMIT - 1024 - BAR_BYTES - 2 * BIG - 4 * PS;
   static constexpr int KV_STAGES = KV_AVAIL / KV_STAGE > MAX_STAGES ? MAX_STAGES : KV_AVAIL / KV_STAGE;
   static constexpr int KV_SMEM = 1024 + 2 * BIG + KV_STAGES * KV_STAGE + 4 * PS + BAR_BYTES;
@@ -98,14 +100,17 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t tile, int ks) {
 // Descriptor of K-step ks (16 columns) of a [rows x 64] tile with 128-byte rows.
 __device__ __forceinline__ uint64_t wdesc(uint32_t tile, int ks) { return smem_desc(tile + ks * 32, 1024, 2); }
 
-// The same row-major [64 x D] tile read MN-major: K runs down the 64 rows, N along the
-// channels.  Chunk c (0: channels [0, C0), 1: [C0, D)) is one swizzle atom wide in N, so
-// only the start address (16 rows per K-step) and the 8-row stride SBO matter.
-template <int D, int chunk>
-__device__ __forceinline__ uint64_t mndesc(uint32_t tile, int ks) {
-  using S = BwdShape<D>;
-  if (chunk == 0) return smem_desc(tile + ks * 16 * S::SW0, S::SBO0, S::LAY0);
-  return smem_desc(tile + S::BS * S::C0 * 2 + ks * 16 * S::SW1, S::SBO1, S::LAY1);
+// Streamed [64 x D] row-major tiles (K in dq; Q and dO in dk/dv) are staged as D/16
+// chunks of [64 rows x 16 channels], 32-byte swizzled, 2048 bytes each.  Read K-major
+// (score products, K = channels), K-step ks is chunk ks with 8-row stride 256.  Read
+// MN-major (gradient products, K = the 64 rows, N = the D channels), K-step ks starts 16
+// rows down (512 bytes) and one descriptor spans all D channels: N advances chunk by
+// chunk (leading byte offset 2048), so each K-step is a single N = D product.
+constexpr int kChunk = 64 * 32;
+__device__ __forceinline__ uint64_t kdesc32(uint32_t tile, int ks) { return smem_desc(tile + ks * kChunk, 256, 6); }
+__device__ __forceinline__ uint64_t mndesc32(uint32_t tile, int ks) {
+  const uint64_t d = smem_desc(tile + ks * 16 * 32, 256, 6);
+  return (d & ~(static_cast<uint64_t>(0x3FFF) << 16)) | (static_cast<uint64_t>(kChunk >> 4) << 16);
 }
 
 // A [D x 64] tile of v^T with 128-byte rows, read as an MN-major operand (N = 64 keys
@@ -148,6 +153,14 @@ __device__ __forceinline__ void unrope(float* v, const AttnBwdParams& p, int n) 
   unrope_block<HL::S0 + HL::S1, HL::S2>(v, tab + static_cast<size_t>(2 * kRopeMaxPos + wp) * kRopePairs);
 }
 
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned), completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // Writes 8 bf16 values to 16-byte chunk `cc` of row r of a 128-byte-swizzled tile.
 __device__ __forceinline__ void store_sw128(uint8_t* tile, int r, int cc, const float* v8) {
   *reinterpret_cast<uint4*>(tile + r * 128 + ((cc ^ (r & 7)) << 4)) = pack_bf16x8(v8);
@@ -159,8 +172,8 @@ template <class HL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
                 const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
-                const __grid_constant__ CUtensorMap tmK0, const __grid_constant__ CUtensorMap tmK1,
-                const __grid_constant__ CUtensorMap tmVT, const AttnBwdParams p) {
+                const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmVT,
+                const AttnBwdParams p) {
   constexpr int D = HL::D;
   using S = BwdShape<D>;
   constexpr int ST = S::DQ_STAGES;
@@ -234,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sVT = sK + S::SMALL;
         const int k_row = bh * N + j * S::BS;
         mbar_arrive_expect_tx(&kv_full[s], S::DQ_STAGE);
-        tma_load_2d(sK, &tmK0, &kv_full[s], 0, k_row);
-        if (S::C1) tma_load_2d(sK + S::BS * S::C0 * 2, &tmK1, &kv_full[s], S::C0, k_row);
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) tma_load_2d(sK + c * kChunk, &tmK16, &kv_full[s], c * 16, k_row);
         tma_load_2d(sVT, &tmVT, &kv_full[s], j * S::BS, bh * D);
         armed[s] = static_cast<int>(ph);
       }
@@ -249,8 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BS);
       constexpr uint32_t idesc_p = idesc_bmn(128, S::BS);
-      constexpr uint32_t idesc_q0 = idesc_bmn(128, S::C0);
-      constexpr uint32_t idesc_q1 = idesc_bmn(128, S::C1 ? S::C1 : 16);
+      constexpr uint32_t idesc_q = idesc_bmn(128, D);
       bool issued = false;
       bool ok = mbar_wait(fixed_full, 0, abort_flag, &g_attn_bwd_err);
       // dQ += dS_i K_i, K_i read MN-major from its row-major tile (channel chunks)
@@ -263,8 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < S::BS / 16; ++ks) {
           const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
-          umma_bf16(tmem + 256, wdesc(a, ks), mndesc<D, 0>(kk, ks), idesc_q0, acc);
-          if (S::C1) umma_bf16(tmem + 256 + S::C0, wdesc(a, ks), mndesc<D, 1>(kk, ks), idesc_q1, acc);
+          umma_bf16(tmem + 256, wdesc(a, ks), mndesc32(kk, ks), idesc_q, acc);
         }
         umma_commit(&dq_done[u]);
         umma_commit(&kv_empty[i % ST]);
@@ -283,12 +294,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t kq = smem_u32(sQ), kd = smem_u32(sdO);
         const uint32_t kk = smem_u32(sStage + s * S::DQ_STAGE), kvt = kk + S::SMALL;
+        // the two products accumulate into different TMEM columns: interleave their K-steps
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(tmem + u * 128, kdesc<D, 128>(kq, ks), kdesc<D, 64>(kk, ks), idesc_s, ks > 0 ? 1u : 0u);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
+        for (int ks = 0; ks < D / 16; ++ks) {
+          umma_bf16(tmem + u * 128, kdesc<D, 128>(kq, ks), kdesc32(kk, ks), idesc_s, ks > 0 ? 1u : 0u);
           umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kd, ks), vtdesc(kvt, ks), idesc_p, ks > 0 ? 1u : 0u);
+        }
         issued = true;
         umma_commit(&s_full[u]);
         if (j >= 1) ok = issue_dq(j - 1);
@@ -375,8 +386,7 @@ template <class HL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmK0, const __grid_constant__ CUtensorMap tmK1,
                   const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmV1,
-                  const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1,
-                  const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
+                  const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmO16,
                   const AttnBwdParams p) {
   constexpr int D = HL::D;
   using S = BwdShape<D>;
@@ -451,11 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sdO = sQ + S::SMALL;
         const int q_row = bh * N + i * S::BS;
         const int o_row = b * N + i * S::BS;
-        mbar_arrive_expect_tx(&st_full[s], S::KV_STAGE);
-        tma_load_2d(sQ, &tmQ0, &st_full[s], 0, q_row);
-        if (S::C1) tma_load_2d(sQ + S::BS * S::C0 * 2, &tmQ1, &st_full[s], S::C0, q_row);
-        tma_load_2d(sdO, &tmO0, &st_full[s], h * D, o_row);
-        if (S::C1) tma_load_2d(sdO + S::BS * S::C0 * 2, &tmO1, &st_full[s], h * D + S::C0, o_row);
+        const size_t st0 = static_cast<size_t>(bh) * p.ld_stats + i * S::BS;
+        mbar_arrive_expect_tx(&st_full[s], 2 * S::SMALL + 2 * S::BS * 4);
+        bulk_load(sQ + S::KV_STATS, p.lse + st0, S::BS * 4, &st_full[s]);
+        bulk_load(sQ + S::KV_STATS + S::BS * 4, p.delta + st0, S::BS * 4, &st_full[s]);
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          tma_load_2d(sQ + c * kChunk, &tmQ16, &st_full[s], c * 16, q_row);
+          tma_load_2d(sdO + c * kChunk, &tmO16, &st_full[s], h * D + c * 16, o_row);
+        }
         armed[s] = static_cast<int>(ph);
       }
       if (*abort_flag) {
@@ -467,8 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (!skip && warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BS);
-      constexpr uint32_t idesc_o0 = idesc_bmn(128, S::C0);
-      constexpr uint32_t idesc_o1 = idesc_bmn(128, S::C1 ? S::C1 : 16);
+      constexpr uint32_t idesc_o = idesc_bmn(128, D);
       bool issued = false;
       bool ok = mbar_wait(fixed_full, 0, abort_flag, &g_attn_bwd_err);
       // dV += P^T_i dO_i, dK += dS^T_i Q_i; dO_i and Q_i read MN-major (channel chunks)
@@ -481,10 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < S::BS / 16; ++ks) {
           const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
-          umma_bf16(tmem + 256, wdesc(pa, ks), mndesc<D, 0>(ko, ks), idesc_o0, acc);
-          if (S::C1) umma_bf16(tmem + 256 + S::C0, wdesc(pa, ks), mndesc<D, 1>(ko, ks), idesc_o1, acc);
-          umma_bf16(tmem + 384, wdesc(da, ks), mndesc<D, 0>(kq, ks), idesc_o0, acc);
-          if (S::C1) umma_bf16(tmem + 384 + S::C0, wdesc(da, ks), mndesc<D, 1>(kq, ks), idesc_o1, acc);
+          umma_bf16(tmem + 256, wdesc(pa, ks), mndesc32(ko, ks), idesc_o, acc);
+          umma_bf16(tmem + 384, wdesc(da, ks), mndesc32(kq, ks), idesc_o, acc);
         }
         umma_commit(&pd_done[u]);
         umma_commit(&st_empty[i % ST]);
@@ -503,12 +514,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t kk = smem_u32(sK), kv = smem_u32(sV);
         const uint32_t kq = smem_u32(sStage + s * S::KV_STAGE), ko = kq + S::SMALL;
+        // the two products accumulate into different TMEM columns: interleave their K-steps
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(tmem + u * 128, kdesc<D, 128>(kk, ks), kdesc<D, 64>(kq, ks), idesc_s, ks > 0 ? 1u : 0u);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kv, ks), kdesc<D, 64>(ko, ks), idesc_s, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          umma_bf16(tmem + u * 128, kdesc<D, 128>(kk, ks), kdesc32(kq, ks), idesc_s, ks > 0 ? 1u : 0u);
+          umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kv, ks), kdesc32(ko, ks), idesc_s, ks > 0 ? 1u : 0u);
+        }
         issued = true;
         umma_commit(&s_full[u]);
         if (i >= 1) ok = issue_kv(i - 1);
@@ -528,8 +539,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n = kt * S::BR + r;
     const bool row_ok = n < N;
     const float sl2 = p.scale * 1.4426950408889634f;
-    const float* lse_bh = p.lse + static_cast<size_t>(bh) * p.ld_stats;
-    const float* dlt_bh = p.delta + static_cast<size_t>(bh) * p.ld_stats;
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
       const int u = i & 1;
@@ -541,7 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
+      // the step's statistics arrived with its stage (that phase cannot advance before
+      // this step's gradient products, which wait for these threads)
+      if (!mbar_wait(&st_full[i % ST], (i / ST) & 1, abort_flag, &g_attn_bwd_err)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
+      const float* stats = reinterpret_cast<const float*>(sStage + (i % ST) * S::KV_STAGE + S::KV_STATS);
       uint8_t* p_tile = sP + u * S::PS;
       uint8_t* d_tile = sdS + u * S::PS;
       {
@@ -549,12 +565,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sr[32], pr[32];
         tmem_ld32(tmem + lane_off + u * 128 + c0, sr);
         tmem_ld32(tmem + lane_off + u * 128 + 64 + c0, pr);
-        const int q0 = i * S::BS + c0;  // first query of this chunk (< ld_stats - 31)
+        const int q0 = i * S::BS + c0;  // first query of this chunk
         float lq[32], dq[32];
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
-          const float4 a = __ldg(reinterpret_cast<const float4*>(lse_bh + q0) + g);
-          const float4 c = __ldg(reinterpret_cast<const float4*>(dlt_bh + q0) + g);
+          const float4 a = reinterpret_cast<const float4*>(stats + c0)[g];
+          const float4 c = reinterpret_cast<const float4*>(stats + S::BS + c0)[g];
           lq[4 * g] = a.x, lq[4 * g + 1] = a.y, lq[4 * g + 2] = a.z, lq[4 * g + 3] = a.w;
           dq[4 * g] = c.x, dq[4 * g + 1] = c.y, dq[4 * g + 2] = c.z, dq[4 * g + 3] = c.w;
         }
@@ -631,42 +647,38 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   const uint64_t rows = static_cast<uint64_t>(p.B) * p.H * p.N;  // rows of q, k, v [B, H, N, D]
   const uint64_t tok = static_cast<uint64_t>(p.B) * p.N;          // rows of dO [B * N, H * D]
   const uint64_t trows = static_cast<uint64_t>(p.B) * p.H * D;    // rows of v^T [B, H, D, ld]
-  CUtensorMap q0_128, q1_128, o0_128, o1_128, q0_64, q1_64, o0_64, o1_64;
-  CUtensorMap k0_64, k1_64, k0_128, k1_128, v0_128, v1_128, vT;
+  CUtensorMap q0_128, q1_128, o0_128, o1_128, q16, o16, k16, k0_128, k1_128, v0_128, v1_128, vT;
   auto mk = [&](CUtensorMap* m, const void* base, uint64_t r, uint64_t ld, int box_rows, int col0_width, int sw) {
     return make_tmap_2d(m, base, r, ld, ld, box_rows, col0_width, sw);
   };
   bool ok = true;
   const int C0 = S::C0, C1 = S::C1;
-  ok = ok && mk(&q0_128, p.q, rows, D, 128, C0, S::SW0) && mk(&q0_64, p.q, rows, D, 64, C0, S::SW0);
-  ok = ok && mk(&k0_128, p.k, rows, D, 128, C0, S::SW0) && mk(&k0_64, p.k, rows, D, 64, C0, S::SW0);
+  ok = ok && mk(&q0_128, p.q, rows, D, 128, C0, S::SW0) && mk(&q16, p.q, rows, D, 64, 16, 32);
+  ok = ok && mk(&k0_128, p.k, rows, D, 128, C0, S::SW0) && mk(&k16, p.k, rows, D, 64, 16, 32);
   ok = ok && mk(&v0_128, p.v, rows, D, 128, C0, S::SW0);
   ok = ok && make_tmap_2d(&o0_128, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 128,
                           C0, S::SW0);
-  ok = ok && make_tmap_2d(&o0_64, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 64, C0,
-                          S::SW0);
+  ok = ok && make_tmap_2d(&o16, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 64, 16,
+                          32);
   if (C1) {
-    ok = ok && mk(&q1_128, p.q, rows, D, 128, C1, S::SW1) && mk(&q1_64, p.q, rows, D, 64, C1, S::SW1);
-    ok = ok && mk(&k1_128, p.k, rows, D, 128, C1, S::SW1) && mk(&k1_64, p.k, rows, D, 64, C1, S::SW1);
+    ok = ok && mk(&q1_128, p.q, rows, D, 128, C1, S::SW1);
+    ok = ok && mk(&k1_128, p.k, rows, D, 128, C1, S::SW1);
     ok = ok && mk(&v1_128, p.v, rows, D, 128, C1, S::SW1);
     ok = ok && make_tmap_2d(&o1_128, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 128,
                             C1, S::SW1);
-    ok = ok && make_tmap_2d(&o1_64, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 64,
-                            C1, S::SW1);
+
   } else {
-    q1_128 = q0_128, q1_64 = q0_64, k1_128 = k0_128, k1_64 = k0_64, v1_128 = v0_128;
-    o1_128 = o0_128, o1_64 = o0_64;
+    q1_128 = q0_128, k1_128 = k0_128, v1_128 = v0_128, o1_128 = o0_128;
   }
   // v^T: [B*H*D rows, N columns] with row stride ld; columns past N read as zero, so
   // padding never enters an MMA.
   ok = ok && make_tmap_2d(&vT, p.vt, trows, p.N, p.ld, D, 64, 128);
   if (!ok) return cudaErrorInvalidValue;
   dim3 grid((p.N + S::BR - 1) / S::BR, p.H, p.B);
-  attn_bwd_dq<HL><<<grid, kThreads, S::DQ_SMEM, stream>>>(q0_128, q1_128, o0_128, o1_128, k0_64, k1_64, vT, p);
+  attn_bwd_dq<HL><<<grid, kThreads, S::DQ_SMEM, stream>>>(q0_128, q1_128, o0_128, o1_128, k16, vT, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv<HL><<<grid, kThreads, S::KV_SMEM, stream>>>(k0_128, k1_128, v0_128, v1_128, q0_64, q1_64, o0_64,
-                                                            o1_64, p);
+  attn_bwd_dkdv<HL><<<grid, kThreads, S::KV_SMEM, stream>>>(k0_128, k1_128, v0_128, v1_128, q16, o16, p);
   return cudaGetLastError();
 }
 
