@@ -103,6 +103,11 @@ def workload(name: str) -> dict:
         return dict(kind="video", name=name, cfg=cfg, batch=2, frames=frames, grid=(t, gh, gw), tokens=t * gh * gw,
                     desc=f"full tower + 2x2 merge + projector, 2 clips of {frames} frames of {side}x{side} "
                          f"({t} temporal patches, {t * gh * gw} tokens per clip)")
+    if name.startswith("attnbwd"):  # attnbwd<N>: the backward alone, 8 images of N tokens
+        n = int(name[7:])
+        return dict(kind="attn_bwd", name=name, batch=8, grid=None, tokens=n, heads=16, D=80,
+                    desc=f"attention backward only (dq, dk, dv from q, k, v, dO; recomputed forward), "
+                         f"8 images x 16 heads x 80, {n} tokens, no rotary embedding")
     if name.startswith("attn"):
         n = int(name[4:])
         side = int(round(n ** 0.5))
@@ -371,6 +376,21 @@ def run_gpu(args, wl):
         step_flops = B * tower_flops(cfg, N)["total"]
         units_per_step = B
         unit = "clips/s"
+    elif wl["kind"] == "attn_bwd":
+        H, D = wl["heads"], wl["D"]
+        q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+                   for a in S.make_qkv(B, H, N, D, 3))
+        dO = torch.from_numpy(S.make_matrix((B * N, H * D), 4).view(np.int16)).view(torch.bfloat16).to(dev)
+        dqkv = torch.empty((B * N, 3 * H * D), dtype=torch.bfloat16, device=dev)
+        ws_bytes = V.vt_attention_backward_workspace_bytes(B, H, N, D)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def launch(s_):
+            V.vt_attention_backward(q, k, v, dO, dqkv, B, H, N, D, D ** -0.5, ws, ws_bytes, s_)
+
+        step_flops = 10.0 * B * H * N * N * D
+        units_per_step = 1
+        unit = "calls/s"
     else:
         H, D = wl["heads"], wl["D"]
         q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -559,8 +579,8 @@ def run_gpu(args, wl):
                         tokens_per_image=per_unit, merged_tokens_per_image=per_unit / 4,
                         l2="flushed (512 MB write) between timed steps", launch="cuda graph" if graph else "eager",
                         parallelism=f"replicas x{world}"),
-            tokens_per_s=value * per_unit if wl["kind"] != "attn" else None,
-            output_tokens_per_s=value * per_unit / 4 if wl["kind"] != "attn" else None,
+            tokens_per_s=value * per_unit if wl["kind"] not in ("attn", "attn_bwd") else None,
+            output_tokens_per_s=value * per_unit / 4 if wl["kind"] not in ("attn", "attn_bwd") else None,
             tflops=world * step_flops * args.steps / (ms / 1000.0) / 1e12,
             roofline=roofline, kernel_classes=classes,
             cpu_baseline=cpu, e2e=e2e,
