@@ -211,7 +211,7 @@ VT_API vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int3
 
 /* ---------------------------------------------------------------- backward
  * Gradient of a scalar loss with respect to the pixels, given its gradient with
- * respect to the tower output: every layer backwards (recomputed from its saved input),
+ * respect to the tower output: every layer backwards from the activations its forward saved,
  * then the patch embedding and the fold onto the image.  Weights are constants (no
  * weight gradients).  Source: "v2_loaders - Differentiable Vision Tower Loaders
  * (spark2)", summary and section 3 (the loaders are differentiable; the probe
@@ -224,14 +224,18 @@ VT_API vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int3
  * Synchronises the device.  VT_ERR_UNSUPPORTED for other head layouts. */
 VT_API vt_status vt_enable_backward(vt_handle* h);
 
-/* Bytes of the saved-activation buffer (every layer's input, L * B*N*hidden bf16) and of
- * the workspace (covers both vt_forward_saved and vt_backward).  Host only. */
+/* Bytes of the saved-activation buffer and of the workspace (which covers both
+ * vt_forward_saved and vt_backward).  The saved buffer keeps, for every layer, what its
+ * backward needs so that nothing is recomputed: the layer input, the rotated q and k,
+ * v^T, the attention output and its per-query log-sum-exp, the residual stream after
+ * attention and the MLP pre-activation (about (12*hidden + 2*mlp) bytes per token and
+ * layer, 25.7 KB at the 1280/5120 tower).  Host only. */
 VT_API vt_status vt_backward_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* saved_bytes,
                                    size_t* ws_bytes);
 
-/* Forward of the tower that keeps every layer's input in `saved` (device, opaque layout)
- * and writes the tower output tower_out (device bf16 [B, N, hidden], raster order).
- * pixels as vt_forward. */
+/* Forward of the tower that fills `saved` (device, opaque layout, vt_backward_bytes) and
+ * writes the tower output tower_out (device bf16 [B, N, hidden], raster order).  pixels
+ * as vt_forward; the arithmetic is vt_forward's. */
 VT_API vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* grid_thw, int B, void* tower_out,
                                   void* saved, size_t saved_bytes, void* ws, size_t ws_bytes, void* stream);
 

@@ -218,7 +218,9 @@ def test_backward_argument_checks_need_no_device():
     assert _status(e) == "VT_ERR_INVALID_ARG"
     h = V.vt_create(S.get_config("tower448"))
     saved, ws = V.vt_backward_bytes(h, 2, (1, 32, 32))
-    assert saved == 32 * 2 * 1024 * 1280 * 2  # every layer's input
+    # per layer: input, q, k, v^T, attention output, mid residual (6 x [M, 1280] bf16),
+    # MLP pre-activation [M, 5120] bf16, log-sum-exp [B*H, 1024] fp32; M = 2048 tokens
+    assert saved == 32 * (6 * 2048 * 1280 * 2 + 2048 * 5120 * 2 + 2 * 16 * 1024 * 4)
     assert ws >= V.vt_workspace_bytes(h, 2, (1, 32, 32))
     with pytest.raises(V.VtError) as e:
         V.vt_backward_bytes(h, 1, (2, 8, 8))

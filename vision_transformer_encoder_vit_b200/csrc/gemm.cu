@@ -15,8 +15,12 @@
 //    and BN/2 rows of B, so an SM streams 32 KB of operands per 64-deep K step instead
 //    of 48 KB, and six stages fit in shared memory.  The even CTA issues the MMAs and
 //    both CTAs drain their own 128 accumulator rows.  No load uses multicast.
-// CTA = 6 warps: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the MMAs
-// (one thread), warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// CTA = 6 or 10 warps: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the MMAs
+// (one thread), the rest run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).  The
+// plain epilogue (bias / GELU / residual) has two groups of four warps that take the
+// 32-column chunks of a tile alternately, so two warps per SM sub-partition hide each
+// other's load and store latency (short-K GEMMs are otherwise bound by their epilogue);
+// the QKV epilogue, which keeps a whole head per thread, has one group.
 // K steps are 64 deep (one 128-byte swizzle atom); two TMEM accumulators let the
 // epilogue of one tile overlap the main loop of the next.  Tiles are walked m-fastest
 // by a persistent grid, so concurrently running CTAs share each weight tile via L2.
@@ -30,7 +34,12 @@ __device__ unsigned int g_gemm_err;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 192;
+// Epilogue warp groups and threads per CTA for an epilogue kind.
+template <class RL>
+struct Epi {
+  static constexpr int GROUPS = RL::D == 0 ? 2 : 1;
+  static constexpr int THREADS = 64 + 128 * GROUPS;
+};
 
 template <int BN, bool PAIR>
 struct GemmShape {
@@ -87,9 +96,11 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 // Drains one accumulator: this thread's row `row`, columns [col0, col0 + BN), the
 // warp's TMEM lane quadrant at t_row.  Waits for the accumulator (tfull, phase
 // `parity`) itself, after issuing the loads it can issue early.  Returns false on abort.
+// Group `grp` of Epi<RL>::GROUPS drains 32-column chunks grp, grp + GROUPS, ... (plain
+// epilogue); the QKV epilogue has one group.
 template <int BN, class RL, bool PAIR>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int col0, uint32_t t_row, uint64_t* tfull,
-                                              uint32_t parity, volatile int* abort_flag) {
+                                              uint32_t parity, volatile int* abort_flag, int grp) {
   auto wait_acc = [&]() -> bool {
     const bool ok = PAIR ? mbar_wait_cluster(tfull, parity, abort_flag, &g_gemm_err)
                          : mbar_wait(tfull, parity, abort_flag, &g_gemm_err);
@@ -114,15 +125,16 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
                     : zero;
       }
     };
+    constexpr int STEP = 32 * Epi<RL>::GROUPS;
     uint4 bq[4], rq[4];
-    prefetch(col0, bq, rq);
+    prefetch(col0 + 32 * grp, bq, rq);
     if (!wait_acc()) return false;
 #pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 32) {
+    for (int c0 = 32 * grp; c0 < BN; c0 += STEP) {
       const int col = col0 + c0;
       if (col >= p.N) break;
       uint4 bn_[4] = {zero, zero, zero, zero}, rn_[4] = {zero, zero, zero, zero};
-      if (c0 + 32 < BN) prefetch(col + 32, bn_, rn_);
+      if (c0 + STEP < BN) prefetch(col + STEP, bn_, rn_);
       float v[32];
       load_cols<32>(t_row + c0, v);
 #pragma unroll
@@ -130,6 +142,9 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
         const int cg = col + 8 * g;
         if (cg < p.N) {
           if (bias) add_bf16x8(v + 8 * g, bq[g]);
+          if (p.pre_out && row < p.M)  // pre-activation kept for a later backward
+            *reinterpret_cast<uint4*>(static_cast<bf16*>(p.pre_out) + static_cast<size_t>(row) * p.ldo + cg) =
+                pack_bf16x8(v + 8 * g);
           if (p.act >= ACT_DGELU_TANH) {
             // backward of GELU: scale by gelu'(pre-activation), which `resid` carries
             const uint32_t w[4] = {rq[g].x, rq[g].y, rq[g].z, rq[g].w};
@@ -227,7 +242,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
 // ------------------------------------------------------------ one CTA per tile
 
 template <int BN, class RL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmParams p) {
   using S = GemmShape<BN, false>;
@@ -259,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 128 * Epi<RL>::GROUPS);
     }
     mbar_init(drain, 1);
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_gemm_err) != 0) ? 1 : 0;
@@ -362,13 +377,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (!skip) {
     // ------------------------------------------------------------- epilogue
     const int quad = warp & 3;
+    const int grp = (warp - 2) >> 2;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-      if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag)) break;
+      if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp)) break;
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -386,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------- two CTAs per 256-row tile
 
 template <int BN, class RL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const GemmParams p) {
   using S = GemmShape<BN, true>;
@@ -421,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&tempty[a], 8 * Epi<RL>::GROUPS);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_gemm_err) != 0) ? 1 : 0;
@@ -535,6 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (!skip) {
     // ------------------------------------------------------------- epilogue
     const int quad = warp & 3;
+    const int grp = (warp - 2) >> 2;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
@@ -542,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-      if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag)) break;
+      if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp)) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -579,7 +596,7 @@ cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
   if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN, kBK, 128)) return cudaErrorInvalidValue;
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  gemm_bf16_tcgen05<BN, RL><<<grid, kThreads, S::SMEM_BYTES, stream>>>(ta, tb, p);
+  gemm_bf16_tcgen05<BN, RL><<<grid, Epi<RL>::THREADS, S::SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
@@ -601,7 +618,7 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(Epi<RL>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = S::SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -79,6 +79,7 @@ struct GemmParams {
   void* out;          // [M, ldo] bf16
   int ldo;
   int act;
+  void* pre_out;  // optional [M, ldo] bf16: the values before the activation (bias added)
   // QKV mode: output columns are [q | k | v], each heads*head_dim wide.  q and k are
   // rotated (3D RoPE) and written [B, heads, ntok, head_dim]; v is written transposed
   // [B, heads, head_dim, ld_vt].

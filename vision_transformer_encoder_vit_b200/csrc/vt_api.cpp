@@ -1166,9 +1166,47 @@ vt_status vt_profile_launch(int64_t i, int* cls, double* ms, double* flops, doub
 
 namespace {
 
+// What the forward keeps of every layer for the backward (so that the backward runs no
+// forward GEMM or attention again): the layer input, the rotated q and k, v^T, the
+// attention output and its per-query log-sum-exp, the residual stream after attention,
+// and the MLP pre-activation.  Offsets within one layer's block.
+struct SavedLayout {
+  int N, M, ld, lds;
+  size_t x, q, k, vt, a, x1, z, lse, per_layer;
+};
+
+SavedLayout saved_layout(const vt_config& c, int B, int N) {
+  SavedLayout L;
+  L.N = N;
+  L.M = B * N;
+  L.ld = round8(N);
+  L.lds = (N + 63) / 64 * 64;
+  const size_t d = c.hidden, M = static_cast<size_t>(L.M);
+  const size_t headT = static_cast<size_t>(B) * c.heads * c.head_dim * L.ld;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.x = take(M * d * 2);
+  L.q = take(M * d * 2);
+  L.k = take(M * d * 2);
+  L.vt = take(headT * 2);
+  L.a = take(M * d * 2);
+  L.x1 = take(M * d * 2);
+  L.z = take(M * static_cast<size_t>(c.mlp) * 2);
+  L.lse = take(static_cast<size_t>(B) * c.heads * L.lds * 4);
+  L.per_layer = off;
+  return L;
+}
+
+// Backward workspace: the running gradient dx, scratch for the gradients of the LayerNorm
+// outputs (dg, dh), the MLP gradient (also the patch-vector gradient at the end), dO, v
+// in rows, the [M, 3d] qkv gradient and the per-query delta.
 struct BwdPlan {
   int N, M, ld, lds;
-  size_t dx, xn, q, k, vt, a, x1, hmid, dO, v, dqkv, lse, delta, total;
+  size_t dx, xn, hmid, dO, v, dqkv, delta, total;
 };
 
 BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
@@ -1179,7 +1217,6 @@ BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
   p.lds = (N + 63) / 64 * 64;
   const size_t d = c.hidden, M = static_cast<size_t>(p.M);
   const size_t K0 = 3ull * c.temporal_patch * c.patch * c.patch;
-  const size_t headT = static_cast<size_t>(B) * c.heads * c.head_dim * p.ld;  // [B, H, D, ld]
   const size_t stats = static_cast<size_t>(B) * c.heads * p.lds;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -1189,16 +1226,10 @@ BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
   };
   p.dx = take(M * d * 2);
   p.xn = take(M * d * 2);
-  p.q = take(M * d * 2);
-  p.k = take(M * d * 2);
-  p.vt = take(headT * 2);
-  p.a = take(M * d * 2);
-  p.x1 = take(M * d * 2);
   p.hmid = take(M * std::max<size_t>(c.mlp, K0) * 2);
   p.dO = take(M * d * 2);
   p.v = take(M * d * 2);
   p.dqkv = take(M * 3 * d * 2);
-  p.lse = take(stats * 4);
   p.delta = take(stats * 4);
   p.total = off;
   return p;
@@ -1232,83 +1263,100 @@ vt_status run_attention_backward(const AttnBwdParams& p, cudaStream_t st) {
   return VT_OK;
 }
 
+// One layer forward on block-ordered tokens that keeps what the backward needs in the
+// layer's saved block `sv` (its input x is already there); writes the layer output to
+// x_out.  Same kernels and arithmetic as run_layer.
+vt_status run_layer_saving(vt_handle* h, int i, char* sv, const SavedLayout& sl, void* x_out, int B, int gh, int gw,
+                           char* w, const Plan& pl, cudaStream_t st) {
+  const vt_config& c = h->cfg;
+  const vt_handle::Layer& L = h->layers[i];
+  const int d = c.hidden, m = c.mlp, M = sl.M;
+  void* xn = w + pl.xn;
+  void* hmid = w + pl.hmid;
+  vt_status s;
+  if ((s = run_layernorm(sv + sl.x, L.ln1_w, L.ln1_b, xn, M, d, c.ln_eps, st))) return s;
+  {
+    GemmParams p = gemm_params(xn, d, L.qkv_w, d, L.qkv_b, nullptr, 0, nullptr, 0, M, 3 * d, d, ACT_NONE);
+    p.q = sv + sl.q;
+    p.k = sv + sl.k;
+    p.vt = sv + sl.vt;
+    p.heads = c.heads;
+    p.head_dim = c.head_dim;
+    p.ntok = sl.N;
+    p.ld_vt = sl.ld;
+    p.gt = 1;
+    p.gh = gh;
+    p.gw = gw;
+    p.order = ORDER_BLOCK;
+    p.rope = c.use_rope;
+    for (int j = 0; j < 3; ++j) p.sections[j] = c.rope_sections[j];
+    p.rope_tab = h->rope_tab;
+    ProfScope ps(CLS_GEMM, 2.0 * M * 3.0 * d * d, 0, st);
+    cudaError_t e = launch_gemm(p, st, 1);
+    if (e != cudaSuccess) return cuda_fail(e, "qkv gemm launch");
+  }
+  {
+    AttnParams a{};
+    a.q = sv + sl.q;
+    a.k = sv + sl.k;
+    a.vt = sv + sl.vt;
+    a.o = sv + sl.a;
+    a.B = B;
+    a.H = c.heads;
+    a.N = sl.N;
+    a.D = c.head_dim;
+    a.ld_vt = sl.ld;
+    a.scale = 1.0f / std::sqrt(static_cast<float>(c.head_dim));
+    a.lse = reinterpret_cast<float*>(sv + sl.lse);
+    a.ld_lse = sl.lds;
+    if ((s = run_attention(a, st))) return s;
+  }
+  if ((s = run_gemm(gemm_params(sv + sl.a, d, L.o_w, d, L.o_b, sv + sl.x, d, sv + sl.x1, d, M, d, d, ACT_NONE), st)))
+    return s;
+  if ((s = run_layernorm(sv + sl.x1, L.ln2_w, L.ln2_b, xn, M, d, c.ln_eps, st))) return s;
+  {
+    GemmParams p = gemm_params(xn, d, L.fc1_w, d, L.fc1_b, nullptr, 0, hmid, m, M, m, d,
+                               c.gelu_tanh ? ACT_GELU_TANH : ACT_GELU_ERF);
+    p.pre_out = sv + sl.z;  // the pre-activation, for the GELU derivative
+    if ((s = run_gemm(p, st))) return s;
+  }
+  return run_gemm(gemm_params(hmid, m, L.fc2_w, m, L.fc2_b, sv + sl.x1, d, x_out, d, M, d, m, ACT_NONE), st);
+}
+
 // One layer backward on block-ordered tokens: dx (in: d loss / d layer output; out:
-// d loss / d layer input) given the layer's input x_in.
-vt_status run_layer_backward(vt_handle* h, int i, const void* x_in, int B, int gh, int gw, char* w, const BwdPlan& bp,
-                             cudaStream_t st) {
+// d loss / d layer input), from the layer's saved block.
+vt_status run_layer_backward(vt_handle* h, int i, const char* sv, const SavedLayout& sl, int B, int gh, int gw,
+                             char* w, const BwdPlan& bp, cudaStream_t st) {
   const vt_config& c = h->cfg;
   const vt_handle::Layer& L = h->layers[i];
   const vt_handle::LayerT& T = h->layers_t[i];
   const int d = c.hidden, m = c.mlp, M = bp.M, N = bp.N, H = c.heads, D = c.head_dim;
   void* dx = w + bp.dx;
   void* xn = w + bp.xn;
-  void* x1 = w + bp.x1;
   void* hmid = w + bp.hmid;
   vt_status s;
-  // ---- recompute the forward of this layer
-  if ((s = run_layernorm(x_in, L.ln1_w, L.ln1_b, xn, M, d, c.ln_eps, st))) return s;
-  {
-    GemmParams p = gemm_params(xn, d, L.qkv_w, d, L.qkv_b, nullptr, 0, nullptr, 0, M, 3 * d, d, ACT_NONE);
-    p.q = w + bp.q;
-    p.k = w + bp.k;
-    p.vt = w + bp.vt;
-    p.heads = H;
-    p.head_dim = D;
-    p.ntok = N;
-    p.ld_vt = bp.ld;
-    p.gt = 1;
-    p.gh = gh;
-    p.gw = gw;
-    p.order = ORDER_BLOCK;
-    p.rope = c.use_rope;
-    for (int a = 0; a < 3; ++a) p.sections[a] = c.rope_sections[a];
-    p.rope_tab = h->rope_tab;
-    ProfScope ps(CLS_GEMM, 2.0 * M * 3.0 * d * d, 0, st);
-    cudaError_t e = launch_gemm(p, st, 1);
-    if (e != cudaSuccess) return cuda_fail(e, "qkv gemm launch");
-  }
-  const float scale = 1.0f / std::sqrt(static_cast<float>(D));
-  {
-    AttnParams a{};
-    a.q = w + bp.q;
-    a.k = w + bp.k;
-    a.vt = w + bp.vt;
-    a.o = w + bp.a;
-    a.B = B;
-    a.H = H;
-    a.N = N;
-    a.D = D;
-    a.ld_vt = bp.ld;
-    a.scale = scale;
-    a.lse = reinterpret_cast<float*>(w + bp.lse);
-    a.ld_lse = bp.lds;
-    if ((s = run_attention(a, st))) return s;
-  }
-  if ((s = run_gemm(gemm_params(w + bp.a, d, L.o_w, d, L.o_b, x_in, d, x1, d, M, d, d, ACT_NONE), st))) return s;
-  if ((s = run_layernorm(x1, L.ln2_w, L.ln2_b, xn, M, d, c.ln_eps, st))) return s;
-  if ((s = run_gemm(gemm_params(xn, d, L.fc1_w, d, L.fc1_b, nullptr, 0, hmid, m, M, m, d, ACT_NONE), st))) return s;
   // ---- MLP branch: dz = (dx W2) * gelu'(z), dg = dz W1, dx += LN2^T(dg)
   const int dact = c.gelu_tanh ? ACT_DGELU_TANH : ACT_DGELU_ERF;
-  if ((s = run_gemm(gemm_params(dx, d, T.fc2_t, d, nullptr, hmid, m, hmid, m, M, m, d, dact), st))) return s;
+  if ((s = run_gemm(gemm_params(dx, d, T.fc2_t, d, nullptr, sv + sl.z, m, hmid, m, M, m, d, dact), st))) return s;
   if ((s = run_gemm(gemm_params(hmid, m, T.fc1_t, m, nullptr, nullptr, 0, xn, d, M, d, m, ACT_NONE), st))) return s;
-  if ((s = run_layernorm_backward(x1, L.ln2_w, xn, dx, dx, M, d, c.ln_eps, st))) return s;
+  if ((s = run_layernorm_backward(sv + sl.x1, L.ln2_w, xn, dx, dx, M, d, c.ln_eps, st))) return s;
   // ---- attention branch: dO = dx Wo, attention backward, dh = dqkv Wqkv, dx += LN1^T(dh)
   if ((s = run_gemm(gemm_params(dx, d, T.o_t, d, nullptr, nullptr, 0, w + bp.dO, d, M, d, d, ACT_NONE), st))) return s;
   {
     ProfScope ps(CLS_BWD_MISC, 0, 4.0 * M * d + 4.0 * M * H, st);
-    cudaError_t e = launch_attention_delta(w + bp.dO, w + bp.a, reinterpret_cast<float*>(w + bp.delta), B, N, H, D,
+    cudaError_t e = launch_attention_delta(w + bp.dO, sv + sl.a, reinterpret_cast<float*>(w + bp.delta), B, N, H, D,
                                            bp.lds, st);
     if (e != cudaSuccess) return cuda_fail(e, "delta launch");
   }
-  if ((s = run_v_rows(w + bp.vt, bp.ld, w + bp.v, B, H, N, D, st))) return s;
+  if ((s = run_v_rows(sv + sl.vt, sl.ld, w + bp.v, B, H, N, D, st))) return s;
   {
     AttnBwdParams a{};
-    a.q = w + bp.q;
-    a.k = w + bp.k;
+    a.q = sv + sl.q;
+    a.k = sv + sl.k;
     a.v = w + bp.v;
-    a.vt = w + bp.vt;
+    a.vt = sv + sl.vt;
     a.dO = w + bp.dO;
-    a.lse = reinterpret_cast<const float*>(w + bp.lse);
+    a.lse = reinterpret_cast<const float*>(sv + sl.lse);
     a.delta = reinterpret_cast<const float*>(w + bp.delta);
     a.ld_stats = bp.lds;
     a.dqkv = w + bp.dqkv;
@@ -1317,8 +1365,8 @@ vt_status run_layer_backward(vt_handle* h, int i, const void* x_in, int B, int g
     a.H = H;
     a.N = N;
     a.D = D;
-    a.ld = bp.ld;
-    a.scale = scale;
+    a.ld = sl.ld;
+    a.scale = 1.0f / std::sqrt(static_cast<float>(D));
     a.rope = c.use_rope;
     for (int j = 0; j < 3; ++j) a.sections[j] = c.rope_sections[j];
     a.rope_tab = h->rope_tab;
@@ -1331,7 +1379,7 @@ vt_status run_layer_backward(vt_handle* h, int i, const void* x_in, int B, int g
                                 ACT_NONE),
                     st)))
     return s;
-  return run_layernorm_backward(x_in, L.ln1_w, xn, dx, dx, M, d, c.ln_eps, st);
+  return run_layernorm_backward(sv + sl.x, L.ln1_w, xn, dx, dx, M, d, c.ln_eps, st);
 }
 
 vt_status check_backward_grid(const vt_handle* h, int B, const int32_t* grid_thw, int* gh, int* gw) {
@@ -1397,8 +1445,7 @@ vt_status vt_backward_bytes(const vt_handle* h, int B, const int32_t* grid_thw, 
   vt_status s = check_backward_grid(h, B, grid_thw, &gh, &gw);
   if (s) return s;
   const vt_config& c = h->cfg;
-  const size_t M = static_cast<size_t>(B) * gh * gw;
-  *saved_bytes = static_cast<size_t>(c.layers) * align256(M * c.hidden * 2);
+  *saved_bytes = static_cast<size_t>(c.layers) * saved_layout(c, B, gh * gw).per_layer;
   *ws_bytes = std::max(make_plan(c, B, 1, gh, gw).total, make_bwd_plan(c, B, gh * gw).total);
   return VT_OK;
 }
@@ -1419,10 +1466,10 @@ vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* gri
                 ws_bytes, need_ws);
   const vt_config& c = h->cfg;
   const Plan pl = make_plan(c, B, 1, gh, gw);
+  const SavedLayout sl = saved_layout(c, B, gh * gw);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  const size_t layer_bytes = align256(static_cast<size_t>(pl.M) * c.hidden * 2);
-  auto layer_in = [&](int i) -> void* { return static_cast<char*>(saved) + i * layer_bytes; };
+  auto block = [&](int i) -> char* { return static_cast<char*>(saved) + i * sl.per_layer; };
   const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
   {
     ProfScope ps(CLS_UNFOLD, 0, pl.M * (4.0 * 3 * c.patch * c.patch + 2.0 * K0), st);
@@ -1430,14 +1477,14 @@ vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* gri
                                         c.temporal_patch, ORDER_BLOCK, st);
     if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
   }
-  void* x0 = c.layers > 0 ? layer_in(0) : w + pl.x;
+  void* x0 = c.layers > 0 ? static_cast<void*>(block(0) + sl.x) : static_cast<void*>(w + pl.x);
   if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x0, c.hidden, pl.M, c.hidden,
                                 K0, ACT_NONE),
                     st)))
     return s;
   for (int i = 0; i < c.layers; ++i) {
-    void* out = i + 1 < c.layers ? layer_in(i + 1) : w + pl.x;
-    if ((s = run_layer(h, i, layer_in(i), out, B, 1, gh, gw, ORDER_BLOCK, w, pl, st))) return s;
+    void* out = i + 1 < c.layers ? static_cast<void*>(block(i + 1) + sl.x) : static_cast<void*>(w + pl.x);
+    if ((s = run_layer_saving(h, i, block(i), sl, out, B, gh, gw, w, pl, st))) return s;
   }
   ProfScope ps(CLS_REORDER, 0, 4.0 * pl.M * c.hidden, st);
   cudaError_t e = launch_reorder_rows(w + pl.x, tower_out, B, 1, gh, gw, c.hidden, 0, st);
@@ -1461,16 +1508,16 @@ vt_status vt_backward(vt_handle* h, const void* saved, const int32_t* grid_thw, 
   const vt_config& c = h->cfg;
   const int N = gh * gw, d = c.hidden;
   const BwdPlan bp = make_bwd_plan(c, B, N);
+  const SavedLayout sl = saved_layout(c, B, N);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  const size_t layer_bytes = align256(static_cast<size_t>(bp.M) * d * 2);
   {
     ProfScope ps(CLS_REORDER, 0, 4.0 * bp.M * d, st);
     cudaError_t e = launch_reorder_rows(d_tower, w + bp.dx, B, 1, gh, gw, d, 1, st);
     if (e != cudaSuccess) return cuda_fail(e, "reorder launch");
   }
   for (int i = c.layers - 1; i >= 0; --i)
-    if ((s = run_layer_backward(h, i, static_cast<const char*>(saved) + i * layer_bytes, B, gh, gw, w, bp, st)))
+    if ((s = run_layer_backward(h, i, static_cast<const char*>(saved) + i * sl.per_layer, sl, B, gh, gw, w, bp, st)))
       return s;
   const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
   if ((s = run_gemm(gemm_params(w + bp.dx, d, h->pe_t, d, nullptr, nullptr, 0, w + bp.hmid, K0, bp.M, K0, d,
