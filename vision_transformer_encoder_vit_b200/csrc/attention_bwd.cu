@@ -19,14 +19,15 @@
 //  * attn_bwd_dq: one CTA per 128 queries; 64-key steps stream K and V^T.
 //        S = Q K_j^T, dP = dO V_j^T  (TMEM, double-buffered)  -> dS (bf16, shared)
 //        dQ += dS K_j                (TMEM accumulator)
-//  * attn_bwd_dkdv: one CTA per 128 keys; 64-query steps stream Q and dO.
+//  * attn_bwd_dkdv: one CTA per 128 keys (K and v^T staged once); 64-query steps stream
+//    Q and dO.
 //        S^T = K Q_i^T, dP^T = V dO_i^T                      -> P^T, dS^T (bf16, shared)
 //        dV += P^T dO_i, dK += dS^T Q_i
 // A tile staged once serves both products that read it: the row-major [64 x D] tiles of
 // K, Q and dO are the K-major B operand of the score products and, read MN-major (the
-// MMA's B-transpose bit), the B operand of dQ, dK and dV; the [D x 64] tile of v^T is the
-// MN-major B operand of dP.  So no transposed copy is made and every operand byte
-// crosses from L2 once per step.
+// MMA's B-transpose bit), the B operand of dQ, dK and dV; the [D x 64] tiles of v^T are
+// the MN-major B operand of dP and the MN-major A operand of dP^T.  So no transposed copy
+// is made and every operand byte crosses from L2 once per step.
 #include <math.h>
 
 #include "internal.h"
@@ -116,6 +117,19 @@ __device__ __forceinline__ uint64_t mndesc32(uint32_t tile, int ks) {
 // A [D x 64] tile of v^T with 128-byte rows, read as an MN-major operand (N = 64 keys
 // along a row, K = channels down the rows): 16 rows per K-step.
 __device__ __forceinline__ uint64_t vtdesc(uint32_t tile, int ks) { return smem_desc(tile + ks * 2048, 1024, 2); }
+
+// v^T of a CTA's 128 keys staged as two [D x 64] boxes (128-byte rows: 64 keys of one
+// channel), read as the MN-major A operand V (M = the 128 keys along the rows, K = the
+// channels down the rows): 16 rows per K-step, the second 64 keys one box further
+// (leading byte offset = one box).
+template <int D>
+__device__ __forceinline__ uint64_t vadesc(uint32_t tile, int ks) {
+  const uint64_t d = smem_desc(tile + ks * 2048, 1024, 2);
+  return (d & ~(static_cast<uint64_t>(0x3FFF) << 16)) | (static_cast<uint64_t>((D * 128) >> 4) << 16);
+}
+
+// Instruction descriptor with the A operand MN-major (bit 15).
+__host__ __device__ constexpr uint32_t idesc_amn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 15); }
 
 // Instruction descriptor with the B operand MN-major (bit 16).
 __host__ __device__ constexpr uint32_t idesc_bmn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 16); }
@@ -385,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <class HL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmK0, const __grid_constant__ CUtensorMap tmK1,
-                  const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmV1,
-                  const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmO16,
+                  const __grid_constant__ CUtensorMap tmVT, const __grid_constant__ CUtensorMap tmQ16,
+                  const __grid_constant__ CUtensorMap tmO16,
                   const AttnBwdParams p) {
   constexpr int D = HL::D;
   using S = BwdShape<D>;
@@ -394,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
-  uint8_t* sV = sK + S::BIG;
-  uint8_t* sStage = sV + S::BIG;           // per stage: Q [64 x D], dO [64 x D]
+  uint8_t* sVT = sK + S::BIG;              // v^T of this CTA's keys: two [D x 64] boxes
+  uint8_t* sStage = sVT + S::BIG;          // per stage: Q [64 x D], dO [64 x D]
   uint8_t* sP = sStage + ST * S::KV_STAGE;  // [2] P^T tiles, then [2] dS^T tiles
   uint8_t* sdS = sP + 2 * S::PS;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sdS + 2 * S::PS);
@@ -450,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(fixed_full, 2 * S::BIG);
       tma_load_2d(sK, &tmK0, fixed_full, 0, k_row);
       if (S::C1) tma_load_2d(sK + S::BR * S::C0 * 2, &tmK1, fixed_full, S::C0, k_row);
-      tma_load_2d(sV, &tmV0, fixed_full, 0, k_row);
-      if (S::C1) tma_load_2d(sV + S::BR * S::C0 * 2, &tmV1, fixed_full, S::C0, k_row);
+      tma_load_2d(sVT, &tmVT, fixed_full, kt * S::BR, bh * D);
+      tma_load_2d(sVT + D * 128, &tmVT, fixed_full, kt * S::BR + 64, bh * D);
       armed[ST] = 0;
       for (int i = 0; i < nq; ++i) {
         const int s = i % ST;
@@ -482,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BS);
       constexpr uint32_t idesc_o = idesc_bmn(128, D);
+      constexpr uint32_t idesc_vs = idesc_amn(128, S::BS);  // dP^T = V dO^T with V read MN-major
       bool issued = false;
       bool ok = mbar_wait(fixed_full, 0, abort_flag, &g_attn_bwd_err);
       // dV += P^T_i dO_i, dK += dS^T_i Q_i; dO_i and Q_i read MN-major (channel chunks)
@@ -512,13 +527,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t kk = smem_u32(sK), kv = smem_u32(sV);
+        const uint32_t kk = smem_u32(sK), kv = smem_u32(sVT);
         const uint32_t kq = smem_u32(sStage + s * S::KV_STAGE), ko = kq + S::SMALL;
         // the two products accumulate into different TMEM columns: interleave their K-steps
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           umma_bf16(tmem + u * 128, kdesc<D, 128>(kk, ks), kdesc32(kq, ks), idesc_s, ks > 0 ? 1u : 0u);
-          umma_bf16(tmem + u * 128 + 64, kdesc<D, 128>(kv, ks), kdesc32(ko, ks), idesc_s, ks > 0 ? 1u : 0u);
+          umma_bf16(tmem + u * 128 + 64, vadesc<D>(kv, ks), kdesc32(ko, ks), idesc_vs, ks > 0 ? 1u : 0u);
         }
         issued = true;
         umma_commit(&s_full[u]);
@@ -647,7 +662,7 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   const uint64_t rows = static_cast<uint64_t>(p.B) * p.H * p.N;  // rows of q, k, v [B, H, N, D]
   const uint64_t tok = static_cast<uint64_t>(p.B) * p.N;          // rows of dO [B * N, H * D]
   const uint64_t trows = static_cast<uint64_t>(p.B) * p.H * D;    // rows of v^T [B, H, D, ld]
-  CUtensorMap q0_128, q1_128, o0_128, o1_128, q16, o16, k16, k0_128, k1_128, v0_128, v1_128, vT;
+  CUtensorMap q0_128, q1_128, o0_128, o1_128, q16, o16, k16, k0_128, k1_128, vT;
   auto mk = [&](CUtensorMap* m, const void* base, uint64_t r, uint64_t ld, int box_rows, int col0_width, int sw) {
     return make_tmap_2d(m, base, r, ld, ld, box_rows, col0_width, sw);
   };
@@ -655,7 +670,6 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   const int C0 = S::C0, C1 = S::C1;
   ok = ok && mk(&q0_128, p.q, rows, D, 128, C0, S::SW0) && mk(&q16, p.q, rows, D, 64, 16, 32);
   ok = ok && mk(&k0_128, p.k, rows, D, 128, C0, S::SW0) && mk(&k16, p.k, rows, D, 64, 16, 32);
-  ok = ok && mk(&v0_128, p.v, rows, D, 128, C0, S::SW0);
   ok = ok && make_tmap_2d(&o0_128, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 128,
                           C0, S::SW0);
   ok = ok && make_tmap_2d(&o16, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 64, 16,
@@ -663,12 +677,11 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   if (C1) {
     ok = ok && mk(&q1_128, p.q, rows, D, 128, C1, S::SW1);
     ok = ok && mk(&k1_128, p.k, rows, D, 128, C1, S::SW1);
-    ok = ok && mk(&v1_128, p.v, rows, D, 128, C1, S::SW1);
     ok = ok && make_tmap_2d(&o1_128, p.dO, tok, static_cast<uint64_t>(p.H) * D, static_cast<uint64_t>(p.H) * D, 128,
                             C1, S::SW1);
 
   } else {
-    q1_128 = q0_128, k1_128 = k0_128, v1_128 = v0_128, o1_128 = o0_128;
+    q1_128 = q0_128, k1_128 = k0_128, o1_128 = o0_128;
   }
   // v^T: [B*H*D rows, N columns] with row stride ld; columns past N read as zero, so
   // padding never enters an MMA.
@@ -678,7 +691,7 @@ cudaError_t launch_bwd(const AttnBwdParams& p, cudaStream_t stream) {
   attn_bwd_dq<HL><<<grid, kThreads, S::DQ_SMEM, stream>>>(q0_128, q1_128, o0_128, o1_128, k16, vT, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv<HL><<<grid, kThreads, S::KV_SMEM, stream>>>(k0_128, k1_128, v0_128, v1_128, q16, o16, p);
+  attn_bwd_dkdv<HL><<<grid, kThreads, S::KV_SMEM, stream>>>(k0_128, k1_128, vT, q16, o16, p);
   return cudaGetLastError();
 }
 

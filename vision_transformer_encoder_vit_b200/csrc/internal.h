@@ -132,7 +132,6 @@ unsigned int attention_read_clear_error(cudaStream_t stream);
 struct AttnBwdParams {
   const void* q;      // [B, H, N, D] bf16, rotated
   const void* k;      // [B, H, N, D] bf16, rotated
-  const void* v;      // [B, H, N, D] bf16
   const void* vt;     // [B, H, D, ld] bf16 (v transposed, as the forward uses it)
   const void* dO;     // [B*N, H*D] bf16, gradient of the attention output
   const float* lse;   // [B*H, ld_stats], from the forward

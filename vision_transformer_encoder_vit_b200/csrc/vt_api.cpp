@@ -1202,11 +1202,11 @@ SavedLayout saved_layout(const vt_config& c, int B, int N) {
 }
 
 // Backward workspace: the running gradient dx, scratch for the gradients of the LayerNorm
-// outputs (dg, dh), the MLP gradient (also the patch-vector gradient at the end), dO, v
-// in rows, the [M, 3d] qkv gradient and the per-query delta.
+// outputs (dg, dh), the MLP gradient (also the patch-vector gradient at the end), dO,
+// the [M, 3d] qkv gradient and the per-query delta.
 struct BwdPlan {
   int N, M, ld, lds;
-  size_t dx, xn, hmid, dO, v, dqkv, delta, total;
+  size_t dx, xn, hmid, dO, dqkv, delta, total;
 };
 
 BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
@@ -1228,7 +1228,6 @@ BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
   p.xn = take(M * d * 2);
   p.hmid = take(M * std::max<size_t>(c.mlp, K0) * 2);
   p.dO = take(M * d * 2);
-  p.v = take(M * d * 2);
   p.dqkv = take(M * 3 * d * 2);
   p.delta = take(stats * 4);
   p.total = off;
@@ -1240,17 +1239,6 @@ vt_status run_layernorm_backward(const void* x, const void* g, const void* dy, c
   ProfScope ps(CLS_BWD_MISC, 0, 8.0 * rows * static_cast<double>(cols), st);
   cudaError_t e = launch_layernorm_backward(x, g, dy, dres, dx, rows, cols, eps, st);
   if (e != cudaSuccess) return cuda_fail(e, "layernorm backward launch");
-  return VT_OK;
-}
-
-// vt [B, H, D, ld] -> v [B, H, N, D]: the row-major v the dk/dv kernel reads as an
-// A operand.
-vt_status run_v_rows(const void* vt, int ld, void* v, int B, int H, int N, int D, cudaStream_t st) {
-  ProfScope ps(CLS_BWD_MISC, 0, 4.0 * B * H * static_cast<double>(N) * D, st);
-  const long hnd = static_cast<long>(H) * N * D, nd = static_cast<long>(N) * D;
-  const long hdl = static_cast<long>(H) * D * ld, dl = static_cast<long>(D) * ld;
-  cudaError_t e = launch_transpose(vt, v, B, H, D, N, hdl, dl, ld, hnd, nd, D, st);
-  if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
   return VT_OK;
 }
 
@@ -1348,12 +1336,10 @@ vt_status run_layer_backward(vt_handle* h, int i, const char* sv, const SavedLay
                                            bp.lds, st);
     if (e != cudaSuccess) return cuda_fail(e, "delta launch");
   }
-  if ((s = run_v_rows(sv + sl.vt, sl.ld, w + bp.v, B, H, N, D, st))) return s;
   {
     AttnBwdParams a{};
     a.q = sv + sl.q;
     a.k = sv + sl.k;
-    a.v = w + bp.v;
     a.vt = sv + sl.vt;
     a.dO = w + bp.dO;
     a.lse = reinterpret_cast<const float*>(sv + sl.lse);
@@ -1580,7 +1566,6 @@ vt_status vt_attention_backward(const void* q, const void* k, const void* v, con
   AttnBwdParams p{};
   p.q = q;
   p.k = k;
-  p.v = v;
   p.vt = vt_;
   p.dO = dO;
   p.lse = lse;
