@@ -479,69 +479,65 @@ def run_gpu(args, wl):
     # ---------------- end to end through the C ABI with host buffers
     e2e = None
     if wl["kind"] == "tower":
-        ws_h = torch.empty(V.vt_forward_host_workspace_bytes(tower.h, B, grid), dtype=torch.uint8, device=dev)
-        out_h = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory()
-        V.vt_forward_host(tower.h, px_host, grid, B, out_h, ws_h, ws_h.numel(), stream)
+        # A serving pipeline: batches alternate between two streams, each with its own
+        # workspace and pinned output, so one batch's copies overlap the other's forward.
+        # Every step still copies its pixels in and its projected tokens out.
+        wsb_h = V.vt_forward_host_workspace_bytes(tower.h, B, grid)
+        ws_h = [torch.empty(wsb_h, dtype=torch.uint8, device=dev) for _ in range(2)]
+        out_h = [torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        streams = [stream, torch.cuda.Stream(device=dev)]
+        for i in range(2):
+            V.vt_forward_host(tower.h, px_host, grid, B, out_h[i], ws_h[i], wsb_h, streams[i])
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e_s = torch.cuda.Event(enable_timing=True)
         e_e = torch.cuda.Event(enable_timing=True)
         e_s.record(stream)
-        for _ in range(args.steps):
-            V.vt_forward_host(tower.h, px_host, grid, B, out_h, ws_h, ws_h.numel(), stream)
+        streams[1].wait_event(e_s)
+        for i in range(args.steps):
+            V.vt_forward_host_async(tower.h, px_host, grid, B, out_h[i % 2], ws_h[i % 2], wsb_h, streams[i % 2])
+        stream.wait_stream(streams[1])
         e_e.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_s.elapsed_time(e_e)
         e2e_ms = REP.max_over_ranks(e2e_ms, dev)
         e2e = dict(value=REP.job_throughput(B, args.steps, e2e_ms, world), unit=unit,
-                   h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h.numel() * 2),
-                   api="vt_forward_host")
+                   h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h[0].numel() * 2),
+                   api="vt_forward_host_async, two streams")
         del ws_h
-    elif wl["kind"] == "backward":
-        cfg = wl["cfg"]
-        tower = V.Tower(cfg, S.make_weights(cfg))
-        V.vt_enable_backward(tower.h)
-        px = torch.from_numpy(S.make_pixels(cfg, batch=B, seed=REP.replica_seed(cfg["seed"], rank))).to(dev)
-        d_tower = torch.from_numpy(S.make_matrix((B, N, cfg["hidden"]), 9).view(np.int16)).view(
-            torch.bfloat16).to(dev)
-        saved_bytes, ws_bytes = V.vt_backward_bytes(tower.h, B, grid)
-        saved = torch.empty(saved_bytes, dtype=torch.uint8, device=dev)
-        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-        tower_out = torch.empty((B, N, cfg["hidden"]), dtype=torch.bfloat16, device=dev)
-        d_px = torch.empty_like(px)
-
-        def launch(s_):
-            V.vt_forward_saved(tower.h, px, grid, B, tower_out, saved, saved_bytes, ws, ws_bytes, s_)
-            V.vt_backward(tower.h, saved, grid, B, d_tower, d_px, ws, ws_bytes, s_)
-
-        step_flops = B * backward_flops(cfg, N)
-        units_per_step = B
-        unit = "images/s"
     elif wl["kind"] == "u8":
-        # decoded images from pinned host memory -> device, forward, projected tokens back
-        out_h = torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory()
+        # decoded images from pinned host memory -> device, forward, projected tokens back;
+        # batches alternate between two streams with their own buffers (serving pipeline)
+        streams = [stream, torch.cuda.Stream(device=dev)]
+        bufs = [(img, ws, out), (torch.empty_like(img), torch.empty_like(ws), torch.empty_like(out))]
+        out_h = [torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
 
-        def e2e_step():
-            img.copy_(img_host, non_blocking=True)
-            launch(stream)
-            out_h.copy_(out, non_blocking=True)
+        def e2e_step(i):
+            im, w_, o_ = bufs[i % 2]
+            with torch.cuda.stream(streams[i % 2]):
+                im.copy_(img_host, non_blocking=True)
+                V.vt_forward_u8(tower.h, im, sizes, grid, o_, None, w_, w_.numel(), stream=streams[i % 2])
+                out_h[i % 2].copy_(o_, non_blocking=True)
 
-        e2e_step()
+        e2e_step(0)
+        e2e_step(1)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e_s = torch.cuda.Event(enable_timing=True)
         e_e = torch.cuda.Event(enable_timing=True)
         e_s.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        streams[1].wait_event(e_s)
+        for i in range(args.steps):
+            e2e_step(i)
+        stream.wait_stream(streams[1])
         e_e.record(stream)
         torch.cuda.synchronize()
         e2e_ms = REP.max_over_ranks(e_s.elapsed_time(e_e), dev)
         e2e = dict(value=REP.job_throughput(B, args.steps, e2e_ms, world), unit=unit,
-                   h2d_bytes_per_step=int(img_host.numel()), d2h_bytes_per_step=int(out_h.numel() * 2),
-                   api="vt_forward_u8 (+ host copies)")
+                   h2d_bytes_per_step=int(img_host.numel()), d2h_bytes_per_step=int(out_h[0].numel() * 2),
+                   api="vt_forward_u8 (+ host copies), two streams")
 
     if rank == 0:
         # dominant kernel class by device time

@@ -147,6 +147,15 @@ VT_API vt_status vt_forward_host(vt_handle* h, const float* pixels_host, const i
                           void* out_host, void* ws, size_t ws_bytes, void* stream);
 VT_API vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out);
 
+/* vt_forward_host without the final synchronisation: the copies and the forward are
+ * enqueued on `stream` and the call returns.  out_host holds the result, and ws, the
+ * pixels and out_host may be reused, only after the caller has synchronised the stream.
+ * Calls on two streams with separate workspaces and output buffers overlap one batch's
+ * copies with another batch's forward (a serving pipeline).  pixels_host and out_host
+ * must be pinned for the copies to be asynchronous. */
+VT_API vt_status vt_forward_host_async(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B,
+                                       void* out_host, void* ws, size_t ws_bytes, void* stream);
+
 /* Video: B clips of `frames` frames each, all frames of one size.
  *   clips     device fp32 [B, frames, 3, H, W], already normalised
  *   frames    >= 1; temporal patch t takes frames t*tp .. t*tp+tp-1 (tp = the config's

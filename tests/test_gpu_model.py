@@ -237,3 +237,25 @@ def test_forward_rejects_small_workspace_and_bad_grid():
     assert e.value.name == "VT_ERR_SHAPE"
     V.vt_check()
     tw.close()
+
+
+def test_host_forward_async_on_two_streams_matches_sync():
+    cfg = S.get_config("tiny")
+    bits = S.make_weights(cfg, affine=True)
+    tw = V.Tower(cfg, bits)
+    grid = (1, 8, 8)
+    px = [torch.from_numpy(S.make_pixels(cfg, batch=2, seed=s)).pin_memory() for s in (1, 2)]
+    wsb = V.vt_forward_host_workspace_bytes(tw.h, 2, grid)
+    ws = [torch.empty(wsb, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    ref = [torch.empty((2, 16, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    got = [torch.empty_like(r).pin_memory() for r in ref]
+    for i in range(2):
+        V.vt_forward_host(tw.h, px[i], grid, 2, ref[i], ws[i], wsb)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for i in range(2):
+        V.vt_forward_host_async(tw.h, px[i], grid, 2, got[i], ws[i], wsb, streams[i])
+    torch.cuda.synchronize()
+    V.vt_check()
+    for i in range(2):
+        assert torch.equal(got[i].view(torch.int16), ref[i].view(torch.int16))
+    tw.close()

@@ -847,8 +847,22 @@ vt_status vt_forward_host_workspace_bytes(const vt_handle* h, int B, const int32
   return VT_OK;
 }
 
+// vt_forward_host without the final synchronisation (see include/vt.h).
+static vt_status forward_host(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B, void* out_host,
+                              void* ws, size_t ws_bytes, void* stream, bool sync);
+
 vt_status vt_forward_host(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B, void* out_host,
                           void* ws, size_t ws_bytes, void* stream) {
+  return forward_host(h, pixels_host, grid_thw, B, out_host, ws, ws_bytes, stream, true);
+}
+
+vt_status vt_forward_host_async(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B,
+                                void* out_host, void* ws, size_t ws_bytes, void* stream) {
+  return forward_host(h, pixels_host, grid_thw, B, out_host, ws, ws_bytes, stream, false);
+}
+
+static vt_status forward_host(vt_handle* h, const float* pixels_host, const int32_t* grid_thw, int B, void* out_host,
+                              void* ws, size_t ws_bytes, void* stream, bool sync) {
   vt_status s = check_loaded(h);
   if (s) return s;
   if (!pixels_host || !out_host || !ws) return fail(VT_ERR_INVALID_ARG, "pixels, out and ws must not be NULL");
@@ -869,7 +883,7 @@ vt_status vt_forward_host(vt_handle* h, const float* pixels_host, const int32_t*
   if ((s = vt_forward(h, dpx, grid_thw, B, dout, nullptr, ws, base, stream))) return s;
   if ((e = cudaMemcpyAsync(out_host, dout, o, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
     return cuda_fail(e, "copying the output to the host");
-  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream synchronisation");
+  if (sync && (e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream synchronisation");
   return VT_OK;
 }
 

@@ -65,6 +65,7 @@ _SIGS = {
     "vt_forward": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_forward_host": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_forward_host_workspace_bytes": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
+    "vt_forward_host_async": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_workspace_bytes_varlen": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
     "vt_forward_varlen": ([_vp, _vp, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
     "vt_forward_video": ([_vp, _vp, _i, _i32p, _i, _vp, _vp, _vp, _sz, _vp]),
@@ -293,6 +294,12 @@ def vt_forward_host_workspace_bytes(h: int, B: int, grid_thw) -> int:
 def vt_forward_host(h, pixels_host, grid_thw, B, out_host, ws, ws_bytes, stream=None) -> None:
     _check(lib.vt_forward_host(h, _ptr(pixels_host), _grid(grid_thw), B, _ptr(out_host), _ptr(ws), ws_bytes,
                                _stream(stream)), "vt_forward_host")
+
+
+def vt_forward_host_async(h, pixels_host, grid_thw, B, out_host, ws, ws_bytes, stream=None) -> None:
+    """Enqueues vt_forward_host on `stream` without synchronising it."""
+    _check(lib.vt_forward_host_async(h, _ptr(pixels_host), _grid(grid_thw), B, _ptr(out_host), _ptr(ws), ws_bytes,
+                                     _stream(stream)), "vt_forward_host_async")
 
 
 def vt_tower_layer(h, layer, x_in, x_out, grid_thw, B, ws, ws_bytes, stream=None) -> None:
