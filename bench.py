@@ -119,8 +119,8 @@ def workload(name: str) -> dict:
 def backward_flops(cfg: dict, N: int) -> float:
     """Algorithmic FLOPs of one image's tower forward plus its input-gradient backward:
     every linear layer's dX product costs what its forward costs; the attention backward
-    is 5 products (S, dP, dV, dK, dQ) = 10 N^2 d.  The layer recomputation inside the
-    backward is not counted."""
+    is 5 products (S, dP, dV, dK, dQ) = 10 N^2 d; the score products it recomputes are
+    not counted."""
     d, m = cfg["hidden"], cfg["mlp"]
     K0 = 3 * cfg["temporal_patch"] * cfg["patch"] ** 2
     L = cfg["layers"]

@@ -1172,7 +1172,7 @@ vt_status vt_profile_launch(int64_t i, int* cls, double* ms, double* flops, doub
 // ------------------------------------------------------------------ backward
 //
 // Gradient of a loss with respect to the pixels, given its gradient with respect to the
-// tower output: the reverse of every layer (recomputed from its saved input), then the
+// tower output: the reverse of every layer (from the activations its forward saved), then the
 // patch embedding and the fold onto the image.  The derivative follows the chain rule
 // through the forward of the "MiniMax-M3 Vision" model card (Architecture table); the
 // "v2_loaders" findings (summary, section 3) describe the loaders as differentiable,
