@@ -52,7 +52,10 @@ struct GemmShape {
   static constexpr int ACC_COLS = BN <= 128 ? 128 : 256;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  // Output staging of the plain epilogue: per epilogue warp two [32 x 32] bf16 boxes.
+  static constexpr int EPI_BOX = 32 * 32 * 2;
+  static constexpr int EPI_BYTES = 8 * 2 * EPI_BOX;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tiles must keep 1024-byte alignment");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
   static_assert(!PAIR || (BN / 2) % 8 == 0, "half of B must be whole 8-row groups");
@@ -93,14 +96,32 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
   }
 }
 
+// Bulk tensor store of a [32 x 32] box from this CTA's shared memory (the caller's
+// async-proxy fence precedes it), tracked by the issuing thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_2d(const void* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most one committed group still reads its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Drains one accumulator: this thread's row `row`, columns [col0, col0 + BN), the
 // warp's TMEM lane quadrant at t_row.  Waits for the accumulator (tfull, phase
 // `parity`) itself, after issuing the loads it can issue early.  Returns false on abort.
 // Group `grp` of Epi<RL>::GROUPS drains 32-column chunks grp, grp + GROUPS, ... (plain
 // epilogue); the QKV epilogue has one group.
+//
+// The plain epilogue writes `out` through shared memory: each warp packs its 32 rows x 32
+// columns into one of its two 64-byte-swizzled staging boxes (`stage`, alternating with
+// `sbuf`) and one lane stores the box with a bulk tensor store (tmC: [M, N] with row
+// stride ldo, box 32 x 32), which clips rows and columns past the matrix.
 template <int BN, class RL, bool PAIR>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int col0, uint32_t t_row, uint64_t* tfull,
-                                              uint32_t parity, volatile int* abort_flag, int grp) {
+                                              uint32_t parity, volatile int* abort_flag, int grp,
+                                              const CUtensorMap* tmC, uint8_t* stage, int& sbuf) {
   auto wait_acc = [&]() -> bool {
     const bool ok = PAIR ? mbar_wait_cluster(tfull, parity, abort_flag, &g_gemm_err)
                          : mbar_wait(tfull, parity, abort_flag, &g_gemm_err);
@@ -110,7 +131,6 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
   if constexpr (RL::D == 0) {
     const bf16* bias = static_cast<const bf16*>(p.bias);
     const bf16* resid = static_cast<const bf16*>(p.resid);
-    bf16* out = static_cast<bf16*>(p.out);
     // Bias and residual of a 32-column chunk are loaded one chunk ahead (the first
     // chunk before waiting for the accumulator) so that no global-load latency sits
     // between the TMEM read and the store.
@@ -164,12 +184,25 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
               v[8 * g + i] = x;
             }
           }
-          if (row < p.M) {
-            if (resid && p.act < ACT_DGELU_TANH) add_bf16x8(v + 8 * g, rq[g]);
-            *reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * p.ldo + cg) = pack_bf16x8(v + 8 * g);
-          }
+          if (resid && p.act < ACT_DGELU_TANH) add_bf16x8(v + 8 * g, rq[g]);
         }
       }
+      // Stage the warp's 32 x 32 box (row = lane; 16-byte chunk g of a 64-byte row at
+      // g ^ ((lane >> 1) & 3), the 64-byte swizzle) and store it with one bulk copy.
+      const int lane = threadIdx.x & 31;
+      uint8_t* box = stage + sbuf * (32 * 32 * 2);
+      if (lane == 0) bulk_wait_read1();  // the store that last read this box is done
+      __syncwarp();
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        *reinterpret_cast<uint4*>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = pack_bf16x8(v + 8 * g);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmC, box, col, row - lane);
+        bulk_commit();
+      }
+      sbuf ^= 1;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         bq[g] = bn_[g];
@@ -244,13 +277,14 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
 template <int BN, class RL>
 __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using S = GemmShape<BN, false>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S::STAGES * S::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);
+  uint8_t* sEpi = sB + S::STAGES * S::B_BYTES;  // output staging, two boxes per epilogue warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BYTES);
   uint64_t* empty = full + S::STAGES;
   uint64_t* tfull = empty + S::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -378,16 +412,21 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     // ------------------------------------------------------------- epilogue
     const int quad = warp & 3;
     const int grp = (warp - 2) >> 2;
+    uint8_t* stage = sEpi + (warp - 2) * 2 * S::EPI_BOX;
+    int sbuf = 0;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-      if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp)) break;
+      if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp, &tmC,
+                                        stage, sbuf))
+        break;
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
+    if ((threadIdx.x & 31) == 0) bulk_wait_all();  // every staged box has reached memory
   }
 
   tc_fence_before();
@@ -404,13 +443,14 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
 template <int BN, class RL>
 __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const GemmParams p) {
+                           const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
   using S = GemmShape<BN, true>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S::STAGES * S::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);  // used in the even CTA
+  uint8_t* sEpi = sB + S::STAGES * S::B_BYTES;  // output staging, two boxes per epilogue warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BYTES);  // used in the even CTA
   uint64_t* empty = full + S::STAGES;                                          // both CTAs
   uint64_t* tfull = empty + S::STAGES;                                         // both CTAs
   uint64_t* tempty = tfull + 2;                                                // even CTA
@@ -553,17 +593,22 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     const int quad = warp & 3;
     const int grp = (warp - 2) >> 2;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
+    uint8_t* stage = sEpi + (warp - 2) * 2 * S::EPI_BOX;
+    int sbuf = 0;
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
       const int acc = it & 1;
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-      if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp)) break;
+      if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp, &tmC,
+                                       stage, sbuf))
+        break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
     }
+    if (lane == 0) bulk_wait_all();  // every staged box has reached memory
   }
 
   // Neither CTA may leave while the pair's MMAs, loads or arrivals can still touch it.
@@ -594,9 +639,11 @@ cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, p.A, p.M, p.K, p.lda, kBM, kBK, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN, kBK, 128)) return cudaErrorInvalidValue;
+  CUtensorMap tc = tb;  // the QKV epilogue writes its own layouts
+  if (RL::D == 0 && !make_tmap_2d(&tc, p.out, p.M, p.N, p.ldo, 32, 32, 64)) return cudaErrorInvalidValue;
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  gemm_bf16_tcgen05<BN, RL><<<grid, Epi<RL>::THREADS, S::SMEM_BYTES, stream>>>(ta, tb, p);
+  gemm_bf16_tcgen05<BN, RL><<<grid, Epi<RL>::THREADS, S::SMEM_BYTES, stream>>>(ta, tb, tc, p);
   return cudaGetLastError();
 }
 
@@ -613,6 +660,8 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, p.A, p.M, p.K, p.lda, kBM, kBK, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN / 2, kBK, 128)) return cudaErrorInvalidValue;
+  CUtensorMap tc = tb;  // the QKV epilogue writes its own layouts
+  if (RL::D == 0 && !make_tmap_2d(&tc, p.out, p.M, p.N, p.ldo, 32, 32, 64)) return cudaErrorInvalidValue;
   const int tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
   const int max_pairs = device_sm_count() / 2;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -628,7 +677,7 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, tc, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
