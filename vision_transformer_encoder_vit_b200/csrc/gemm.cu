@@ -121,7 +121,8 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 template <int BN, class RL, bool PAIR>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int col0, uint32_t t_row, uint64_t* tfull,
                                               uint32_t parity, volatile int* abort_flag, int grp,
-                                              const CUtensorMap* tmC, uint8_t* stage, int& sbuf) {
+                                              const CUtensorMap* tmC, const CUtensorMap* tmZ, uint8_t* stage,
+                                              int& sbuf) {
   auto wait_acc = [&]() -> bool {
     const bool ok = PAIR ? mbar_wait_cluster(tfull, parity, abort_flag, &g_gemm_err)
                          : mbar_wait(tfull, parity, abort_flag, &g_gemm_err);
@@ -157,14 +158,34 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
       if (c0 + STEP < BN) prefetch(col + STEP, bn_, rn_);
       float v[32];
       load_cols<32>(t_row + c0, v);
+      const int lane = threadIdx.x & 31;
+      // Stages the warp's 32 x 32 box of `vals` (row = lane; 16-byte chunk g of a 64-byte
+      // row at g ^ ((lane >> 1) & 3), the 64-byte swizzle) and stores it with one bulk copy.
+      auto store_box = [&](const CUtensorMap* map, const float* vals) {
+        uint8_t* box = stage + sbuf * (32 * 32 * 2);
+        if (lane == 0) bulk_wait_read1();  // the store that last read this box is done
+        __syncwarp();
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          *reinterpret_cast<uint4*>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = pack_bf16x8(vals + 8 * g);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(map, box, col, row - lane);
+          bulk_commit();
+        }
+        sbuf ^= 1;
+      };
+      if (bias) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          if (col + 8 * g < p.N) add_bf16x8(v + 8 * g, bq[g]);
+      }
+      if (p.pre_out) store_box(tmZ, v);  // pre-activation kept for a later backward
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int cg = col + 8 * g;
         if (cg < p.N) {
-          if (bias) add_bf16x8(v + 8 * g, bq[g]);
-          if (p.pre_out && row < p.M)  // pre-activation kept for a later backward
-            *reinterpret_cast<uint4*>(static_cast<bf16*>(p.pre_out) + static_cast<size_t>(row) * p.ldo + cg) =
-                pack_bf16x8(v + 8 * g);
           if (p.act >= ACT_DGELU_TANH) {
             // backward of GELU: scale by gelu'(pre-activation), which `resid` carries
             const uint32_t w[4] = {rq[g].x, rq[g].y, rq[g].z, rq[g].w};
@@ -187,22 +208,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
           if (resid && p.act < ACT_DGELU_TANH) add_bf16x8(v + 8 * g, rq[g]);
         }
       }
-      // Stage the warp's 32 x 32 box (row = lane; 16-byte chunk g of a 64-byte row at
-      // g ^ ((lane >> 1) & 3), the 64-byte swizzle) and store it with one bulk copy.
-      const int lane = threadIdx.x & 31;
-      uint8_t* box = stage + sbuf * (32 * 32 * 2);
-      if (lane == 0) bulk_wait_read1();  // the store that last read this box is done
-      __syncwarp();
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-        *reinterpret_cast<uint4*>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = pack_bf16x8(v + 8 * g);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(tmC, box, col, row - lane);
-        bulk_commit();
-      }
-      sbuf ^= 1;
+      store_box(tmC, v);
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         bq[g] = bn_[g];
@@ -277,7 +283,8 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
 template <int BN, class RL>
 __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmZ,
+                      const GemmParams p) {
   using S = GemmShape<BN, false>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       const int row = mb * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
       if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp, &tmC,
-                                        stage, sbuf))
+                                        &tmZ, stage, sbuf))
         break;
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -443,7 +450,8 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
 template <int BN, class RL>
 __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+                           const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmZ,
+                           const GemmParams p) {
   using S = GemmShape<BN, true>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -602,7 +610,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
       if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp, &tmC,
-                                       stage, sbuf))
+                                       &tmZ, stage, sbuf))
         break;
       tc_fence_before();
       __syncwarp();
@@ -639,11 +647,13 @@ cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, p.A, p.M, p.K, p.lda, kBM, kBK, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN, kBK, 128)) return cudaErrorInvalidValue;
-  CUtensorMap tc = tb;  // the QKV epilogue writes its own layouts
+  CUtensorMap tc = tb, tz = tb;  // the QKV epilogue writes its own layouts
   if (RL::D == 0 && !make_tmap_2d(&tc, p.out, p.M, p.N, p.ldo, 32, 32, 64)) return cudaErrorInvalidValue;
+  if (RL::D == 0 && p.pre_out && !make_tmap_2d(&tz, p.pre_out, p.M, p.N, p.ldo, 32, 32, 64))
+    return cudaErrorInvalidValue;
   const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + BN - 1) / BN);
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  gemm_bf16_tcgen05<BN, RL><<<grid, Epi<RL>::THREADS, S::SMEM_BYTES, stream>>>(ta, tb, tc, p);
+  gemm_bf16_tcgen05<BN, RL><<<grid, Epi<RL>::THREADS, S::SMEM_BYTES, stream>>>(ta, tb, tc, tz, p);
   return cudaGetLastError();
 }
 
@@ -660,8 +670,10 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, p.A, p.M, p.K, p.lda, kBM, kBK, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, p.W, p.N, p.K, p.ldw, BN / 2, kBK, 128)) return cudaErrorInvalidValue;
-  CUtensorMap tc = tb;  // the QKV epilogue writes its own layouts
+  CUtensorMap tc = tb, tz = tb;  // the QKV epilogue writes its own layouts
   if (RL::D == 0 && !make_tmap_2d(&tc, p.out, p.M, p.N, p.ldo, 32, 32, 64)) return cudaErrorInvalidValue;
+  if (RL::D == 0 && p.pre_out && !make_tmap_2d(&tz, p.pre_out, p.M, p.N, p.ldo, 32, 32, 64))
+    return cudaErrorInvalidValue;
   const int tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
   const int max_pairs = device_sm_count() / 2;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -677,7 +689,7 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, tc, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, tc, tz, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
