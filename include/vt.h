@@ -1,6 +1,8 @@
 /*
  * vt.h — C ABI of libvt, a B200 (sm_100a) implementation of the forward pass of a
- * CLIP-style ViT vision tower with a 2x2-merge projector.
+ * CLIP-style ViT vision tower with a 2x2-merge projector, with variable-resolution
+ * batches, video clips, GPU preprocessing of decoded images and the backward pass to the
+ * pixels.
  *
  * The model is the one described by the "MiniMax-M3 Vision" model card (Architecture
  * table): patch 14, Conv3d patch embedding with temporal patch 2, 32 pre-LN layers of
@@ -16,10 +18,12 @@
  *  - Ownership: the library never frees caller memory.  Weights passed to
  *    vt_load_weights are borrowed and must outlive the handle.  Workspaces are owned by
  *    the caller.  The library's only device memory is the handle's fused QKV weight
- *    pack (when q, k, v are loaded separately) and its RoPE cos/sin tables.
+ *    pack (when q, k, v are loaded separately), its RoPE cos/sin tables, the transposed
+ *    weights of vt_enable_backward, and the fixed scratch of vt_attention_static.
  *  - Every compute call is asynchronous on the given stream (a cudaStream_t passed as
  *    void*, NULL = legacy default stream), allocates nothing and does not synchronise,
- *    except vt_load_weights, vt_destroy, vt_check and vt_forward_host as documented.
+ *    except vt_load_weights, vt_enable_backward, vt_destroy, vt_check and
+ *    vt_forward_host as documented.
  *  - Errors: every call returns a vt_status.  Argument errors are detected on the host
  *    before anything is launched.  vt_last_error() returns a message for the last
  *    failure of the calling thread.  No C++ exception crosses this interface.
