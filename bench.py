@@ -275,6 +275,92 @@ def run_reference(args, wl):
 
 # ------------------------------------------------------------------ GPU arm
 
+def _best_ms(torch, fn, stream, reps: int = 20, trials: int = 3) -> float:
+    """Best of `trials` event-timed batches of `reps` back-to-back calls (warm L2), ms per call."""
+    for _ in range(3):
+        fn()
+    best = float("inf")
+    for _ in range(trials):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b) / reps)
+    return best
+
+
+def comparators(V, wl, dev, stream) -> dict:
+    """Context only, never on the product path: the library's own kernels (vt_linear,
+    vt_attention) against torch's on the same shapes, timed the same way (warm L2,
+    back-to-back calls, best of three batches) after the benchmark's timed region.
+    torch's linear is cuBLAS(Lt) with its bias epilogue; its attention is
+    scaled_dot_product_attention on the flash and cuDNN backends, each where torch
+    offers it for these shapes."""
+    import torch
+    import torch.nn.functional as F
+    g = torch.Generator(device=dev).manual_seed(11)
+    rows = []
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+    def row(name, flops, ours, theirs: dict):
+        t_o = _best_ms(torch, ours, stream)
+        r = dict(op=name, ours_tflops=flops / t_o / 1e9, ours_us=1000 * t_o)
+        for k, fn in theirs.items():
+            try:
+                t = _best_ms(torch, fn, stream)
+                r[f"{k}_tflops"], r[f"{k}_us"] = flops / t / 1e9, 1000 * t
+            except Exception as e:  # a backend torch does not offer for this shape
+                r[f"{k}_tflops"], r[f"{k}_error"] = None, str(e).splitlines()[0][:120]
+        rows.append(r)
+
+    if wl["kind"] in ("tower", "varlen", "u8", "video", "backward"):
+        cfg = wl["cfg"]
+        d, m, P = cfg["hidden"], cfg["mlp"], cfg["proj_hidden"]
+        M = wl["batch"] * wl["tokens"] if wl["kind"] != "varlen" else wl["tokens"]
+        shapes = [("qkv", M, 3 * d, d, 0), ("o_proj", M, d, d, 0), ("fc1", M, m, d, 0), ("fc2", M, d, m, 0),
+                  ("fc1+gelu_tanh", M, m, d, 1), ("proj_patch_fc2", M, P, P, 0),
+                  ("proj_merge_fc1", M // 4, P, 4 * P, 0)]
+        for name, Mr, Nr, Kr, act in shapes:
+            A, W, bias = rnd(Mr, Kr), rnd(Nr, Kr, scale=0.02), rnd(Nr, scale=0.02)
+            out = torch.empty((Mr, Nr), dtype=torch.bfloat16, device=dev)
+            ours = (lambda A=A, W=W, bias=bias, out=out, Mr=Mr, Nr=Nr, Kr=Kr, act=act:
+                    V.vt_linear(A, W, bias, None, out, Mr, Nr, Kr, act, stream))
+            lib = ((lambda A=A, W=W, bias=bias: F.gelu(F.linear(A, W, bias), approximate="tanh")) if act else
+                   (lambda A=A, W=W, bias=bias: F.linear(A, W, bias)))
+            row(f"{name} [{Mr}x{Kr}]x[{Kr}x{Nr}]", 2.0 * Mr * Nr * Kr, ours,
+                {"torch_cublas" + ("_plus_gelu_kernel" if act else ""): lib})
+            del A, W, bias, out
+    B = wl["batch"] if wl["kind"] not in ("attn", "varlen") else 1
+    N = wl["tokens"] if wl["kind"] != "varlen" else 1024
+    H, D = 16, 80
+    q, k, v = rnd(B, H, N, D), rnd(B, H, N, D), rnd(B, H, N, D)
+    o = torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev)
+    wsb = V.vt_attention_workspace_bytes(B, H, N, D)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    def sdpa(backend):
+        def fn():
+            with sdpa_kernel(backend):
+                F.scaled_dot_product_attention(q, k, v, scale=D ** -0.5)
+        return fn
+
+    # ours: the kernel on operands in its layout (as the tower's QKV epilogue leaves
+    # them: v transposed); "ours_with_prep" adds vt_attention's preparation pass.
+    vt = v.transpose(-1, -2).contiguous()
+    row(f"attention non-causal B={B} H={H} N={N} D={D}", 4.0 * B * H * N * N * D,
+        lambda: V.vt_attention_prepared(q, k, vt, N, o, B, H, N, D, D ** -0.5, stream),
+        {"ours_with_prep": lambda: V.vt_attention(q, k, v, o, B, H, N, D, None, None, 10000.0, D ** -0.5, ws, wsb,
+                                                  stream),
+         "torch_sdpa_flash": sdpa(SDPBackend.FLASH_ATTENTION), "torch_sdpa_cudnn": sdpa(SDPBackend.CUDNN_ATTENTION)})
+    return dict(method="warm L2, 20 back-to-back calls, best of 3 event-timed batches; context only",
+                torch=torch.__version__, rows=rows)
+
+
 def run_gpu(args, wl):
     import torch
     import torch.distributed as dist
@@ -539,6 +625,8 @@ def run_gpu(args, wl):
                    h2d_bytes_per_step=int(img_host.numel()), d2h_bytes_per_step=int(out_h[0].numel() * 2),
                    api="vt_forward_u8 (+ host copies), two streams")
 
+    comp = comparators(V, wl, dev, stream) if args.comparators and rank == 0 else None
+
     if rank == 0:
         # dominant kernel class by device time
         dom = max(("gemm", "attention", "attention_backward"), key=lambda c: prof[c]["ms"])
@@ -583,6 +671,8 @@ def run_gpu(args, wl):
             gpu_launches=int(round(launches_per_step * args.steps)),
             clocks=clk,
         )
+        if comp is not None:
+            line["comparators"] = comp
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -600,6 +690,8 @@ def main():
     ap.add_argument("--profile-steps", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
+    ap.add_argument("--comparators", action="store_true",
+                    help="also time torch's cuBLAS linear and SDPA on the same shapes (context only)")
     args = ap.parse_args()
     wl = workload(args.workload)
     if args.impl == "reference":

@@ -9,8 +9,13 @@
 // comment of CEILING_MAX_PATCHES) builds the full [seq, seq] score matrix per head and
 // notes that larger images need tiled attention; this kernel is that tiled form.
 //
-// CTA = 10 warps.  Warp 0 issues TMA loads (both Q tiles once, then K and V^T tiles
-// shared by the two query tiles).  Warp 1 allocates TMEM and issues the MMAs from one
+// The grid is persistent: at most one CTA per SM, each walking work items (a pair of
+// query tiles of one head of one image) with a stride of the grid size, so barrier
+// setup and TMEM allocation happen once per SM and the next item's first score
+// products run while the current item's last softmax and output are still in flight.
+//
+// CTA = 10 warps.  Warp 0 issues TMA loads (both Q tiles of an item, then K and V^T
+// tiles shared by the two query tiles).  Warp 1 allocates TMEM and issues the MMAs from one
 // thread; for key tile j and query tile t in {0, 1}:
 //     S_t = Q_t K_j^T         -> TMEM columns [256 t, 256 t + 128)        (fp32)
 //     O_t += P_t V_j          -> TMEM columns [256 t + 128, 256 t + 128 + D)
@@ -73,6 +78,27 @@ struct AttnShape {
                 "1024-byte alignment of swizzled tiles");
 };
 
+// One work item: query tiles 2 qp and 2 qp + 1 of head h of image b.
+struct AttnItem {
+  int qp, h, b, N, tok0, nkv, bh;
+};
+
+// Decodes item `it` (query-tile pair fastest, then head, then image, so that items
+// running at the same time share K and V through L2).  False when the pair lies past
+// the end of a smaller image of a packed batch: that item has no work.
+template <int BM, int BN>
+__device__ __forceinline__ bool attn_item(const AttnParams& p, int nqp, int it, AttnItem& w) {
+  w.qp = it % nqp;
+  const int rest = it / nqp;
+  w.h = rest % p.H;
+  w.b = rest / p.H;
+  w.N = p.varlen ? p.vl.tok_off[w.b + 1] - p.vl.tok_off[w.b] : p.N;
+  w.tok0 = p.varlen ? p.vl.tok_off[w.b] : w.b * p.N;
+  w.nkv = (w.N + BN - 1) / BN;
+  w.bh = w.b * p.H + w.h;
+  return w.qp * 2 * BM < w.N;
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
   while (!mbar_test(bar, parity)) {
@@ -111,19 +137,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_free + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* q_empty = drain + 1;  // the last score products of an item have read Q
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* armed = const_cast<int*>(abort_flag + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // qp: pair of query tiles
-  // Tokens of this image and the packed token where they start.
-  const int N = p.varlen ? p.vl.tok_off[b + 1] - p.vl.tok_off[b] : p.N;
-  const int tok0 = p.varlen ? p.vl.tok_off[b] : b * p.N;
-  if (qp * 2 * S::BM >= N) return;  // a smaller image of a packed batch: nothing here
-  const int nkv = (N + S::BN - 1) / S::BN;
-  const int bh = b * p.H + h;
+  const int nqp = (p.N + 2 * S::BM - 1) / (2 * S::BM);  // query-tile pairs of the longest image
+  const int items = nqp * p.H * p.B;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -139,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(q_empty, 1);
     armed[S::STAGES] = -1;  // query tiles
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(&g_attn_err) != 0) ? 1 : 0;
     fence_barrier_init();
@@ -159,30 +182,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ0);
       tma_prefetch_desc(&tmK0);
       tma_prefetch_desc(&tmV);
-      const int qrow = tok0 * p.H + h * N + qp * 2 * S::BM;
-      mbar_arrive_expect_tx(q_full, 2 * S::Q_BYTES);
-      for (int t = 0; t < 2; ++t) {
-        tma_load_2d(sQ + t * S::Q_BYTES, &tmQ0, q_full, 0, qrow + t * S::BM);
-        if (S::C1) tma_load_2d(sQ + t * S::Q_BYTES + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow + t * S::BM);
-      }
-      armed[S::STAGES] = 0;
-      const int krow = tok0 * p.H + h * N;
-      const int vrow = bh * D;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % S::STAGES;
-        const uint32_t ph = (j / S::STAGES) & 1;
-        if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, &g_attn_err)) break;
-        uint8_t* sK = sKV + s * S::KV_BYTES;
-        uint8_t* sV = sK + S::K_BYTES;
-        mbar_arrive_expect_tx(&kv_full[s], S::KV_BYTES);
-        tma_load_2d(sK, &tmK0, &kv_full[s], 0, krow + j * S::BN);
-        if (S::C1) tma_load_2d(sK + S::K1_OFF, &tmK1, &kv_full[s], S::C0, krow + j * S::BN);
-        tma_load_2d(sV, &tmV, &kv_full[s], j * S::BN, vrow);
-        tma_load_2d(sV + S::V1_OFF, &tmV, &kv_full[s], j * S::BN + 64, vrow);
-        armed[s] = static_cast<int>(ph);
+      uint32_t G = 0, I = 0;  // key-tile steps and items loaded so far by this CTA
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+        AttnItem w;
+        if (!attn_item<S::BM, S::BN>(p, nqp, it, w)) continue;
+        // Q is single-buffered: the previous item's score products must have read it.
+        if (I > 0 && !mbar_wait(q_empty, (I - 1) & 1, abort_flag, &g_attn_err)) break;
+        const int qrow = w.tok0 * p.H + w.h * w.N + w.qp * 2 * S::BM;
+        mbar_arrive_expect_tx(q_full, 2 * S::Q_BYTES);
+        for (int t = 0; t < 2; ++t) {
+          tma_load_2d(sQ + t * S::Q_BYTES, &tmQ0, q_full, 0, qrow + t * S::BM);
+          if (S::C1) tma_load_2d(sQ + t * S::Q_BYTES + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow + t * S::BM);
+        }
+        armed[S::STAGES] = static_cast<int>(I & 1);
+        ++I;
+        const int krow = w.tok0 * p.H + w.h * w.N;
+        const int vrow = w.bh * D;
+        for (int j = 0; j < w.nkv; ++j, ++G) {
+          const int s = G % S::STAGES;
+          const uint32_t ph = (G / S::STAGES) & 1;
+          if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, &g_attn_err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sK = sKV + s * S::KV_BYTES;
+          uint8_t* sV = sK + S::K_BYTES;
+          mbar_arrive_expect_tx(&kv_full[s], S::KV_BYTES);
+          tma_load_2d(sK, &tmK0, &kv_full[s], 0, krow + j * S::BN);
+          if (S::C1) tma_load_2d(sK + S::K1_OFF, &tmK1, &kv_full[s], S::C0, krow + j * S::BN);
+          tma_load_2d(sV, &tmV, &kv_full[s], j * S::BN, vrow);
+          tma_load_2d(sV + S::V1_OFF, &tmV, &kv_full[s], j * S::BN + 64, vrow);
+          armed[s] = static_cast<int>(ph);
+        }
       }
       if (*abort_flag) {
-        if (armed[S::STAGES] >= 0) drain_wait(q_full, 0);
+        if (armed[S::STAGES] >= 0) drain_wait(q_full, static_cast<uint32_t>(armed[S::STAGES]));
         for (int s = 0; s < S::STAGES; ++s)
           if (armed[s] >= 0) drain_wait(&kv_full[s], static_cast<uint32_t>(armed[s]));
       }
@@ -192,51 +227,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- MMA
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BN);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D);
-      bool issued = false;
-      bool ok = mbar_wait(q_full, 0, abort_flag, &g_attn_err);
-      // O_t += P_t V_i for query tile t and key tile i.
-      auto issue_pv = [&](int t, int i) -> bool {
-        if (!mbar_wait(&p_full[t], i & 1, abort_flag, &g_attn_err)) return false;
+      bool issued = false, ok = true;
+      // O_t += P_t V for query tile t and the key tile of step g (j-th of its item).
+      auto issue_pv = [&](int t, uint32_t g, int j) -> bool {
+        if (!mbar_wait(&p_full[t], g & 1, abort_flag, &g_attn_err)) return false;
         tc_fence_after();
         const uint32_t p_addr = smem_u32(sP + t * S::P_BYTES);
-        const uint32_t v_addr = smem_u32(sKV + (i % S::STAGES) * S::KV_BYTES + S::K_BYTES);
+        const uint32_t v_addr = smem_u32(sKV + (g % S::STAGES) * S::KV_BYTES + S::K_BYTES);
         const uint32_t tO = tmem + t * 256 + 128;
 #pragma unroll
         for (int ks = 0; ks < S::BN / 16; ++ks) {
           const uint64_t ad = smem_desc(p_addr + (ks >> 2) * (S::BM * 128) + (ks & 3) * 32, 1024, 2);
           const uint64_t bd = smem_desc(v_addr + (ks >> 2) * S::V1_OFF + (ks & 3) * 32, 1024, 2);
-          umma_bf16(tO, ad, bd, idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16(tO, ad, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&o_done[t]);
         return true;
       };
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % S::STAGES;
-        if (!mbar_wait(&kv_full[s], (j / S::STAGES) & 1, abort_flag, &g_attn_err)) {
+      // The P V products of step g are issued after the score products of step g + 1,
+      // which may belong to the next item: the tensor pipe works on those while the
+      // softmax warps finish step g.  pend_j < 0: nothing pending.
+      int pend_j = -1;
+      uint32_t pend_g = 0;
+      uint32_t G = 0, I = 0;
+      for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+        AttnItem w;
+        if (!attn_item<S::BM, S::BN>(p, nqp, it, w)) continue;
+        if (!mbar_wait(q_full, I & 1, abort_flag, &g_attn_err)) {
           ok = false;
           break;
         }
-        const uint32_t k_addr = smem_u32(sKV + s * S::KV_BYTES);
-        for (int t = 0; t < 2 && ok; ++t) {
-          // S_t is single-buffered: the softmax must have read S_t of tile j-1.
-          if (j >= 1 && !mbar_wait(&s_free[t], (j - 1) & 1, abort_flag, &g_attn_err)) {
+        ++I;
+        for (int j = 0; j < w.nkv; ++j, ++G) {
+          const int s = G % S::STAGES;
+          if (!mbar_wait(&kv_full[s], (G / S::STAGES) & 1, abort_flag, &g_attn_err)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(sQ + t * S::Q_BYTES);
+          const uint32_t k_addr = smem_u32(sKV + s * S::KV_BYTES);
+          for (int t = 0; t < 2 && ok; ++t) {
+            // S_t is single-buffered: the softmax must have read S_t of step G - 1.
+            if (G >= 1 && !mbar_wait(&s_free[t], (G - 1) & 1, abort_flag, &g_attn_err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(sQ + t * S::Q_BYTES);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            umma_bf16(tmem + t * 256, qk_desc<D>(q_addr, ks), qk_desc<D>(k_addr, ks), idesc_s, ks > 0 ? 1u : 0u);
-          issued = true;
-          umma_commit(&s_full[t]);
-        }
-        if (ok && j >= 1) {
-          ok = issue_pv(0, j - 1) && issue_pv(1, j - 1);
-          if (ok) umma_commit(&kv_empty[(j - 1) % S::STAGES]);
+            for (int ks = 0; ks < D / 16; ++ks)
+              umma_bf16(tmem + t * 256, qk_desc<D>(q_addr, ks), qk_desc<D>(k_addr, ks), idesc_s, ks > 0 ? 1u : 0u);
+            issued = true;
+            umma_commit(&s_full[t]);
+          }
+          if (!ok) break;
+          if (j == w.nkv - 1) umma_commit(q_empty);
+          if (pend_j >= 0) {
+            if (!(ok = issue_pv(0, pend_g, pend_j) && issue_pv(1, pend_g, pend_j))) break;
+            umma_commit(&kv_empty[pend_g % S::STAGES]);
+          }
+          pend_j = j;
+          pend_g = G;
         }
       }
-      if (ok) ok = issue_pv(0, nkv - 1) && issue_pv(1, nkv - 1);
+      if (ok && pend_j >= 0) ok = issue_pv(0, pend_g, pend_j) && issue_pv(1, pend_g, pend_j);
       if (*abort_flag && issued) {
         umma_commit(drain);
         drain_wait(drain, 0);
@@ -252,107 +305,120 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tS + 128;
     const float sl2 = p.scale * 1.4426950408889634f;  // scale * log2(e)
     uint8_t* pbuf = sP + t * S::P_BYTES;
-    float m_ref = -INFINITY;  // running maximum of s * sl2 used as the exponent origin
-    float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(&s_full[t], j & 1, abort_flag, &g_attn_err)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[S::BN];
+    uint32_t G = 0;  // key-tile steps done by this CTA over all its items
+    for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+      int Nw, nkv;
       {
-        uint32_t raw[S::BN];
-        tmem_ld128(tS, raw);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < S::BN; ++c) s[c] = __uint_as_float(raw[c]);
+        AttnItem w;
+        if (!attn_item<S::BM, S::BN>(p, nqp, it, w)) continue;
+        Nw = w.N;
+        nkv = w.nkv;
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[t]);
-      const int valid = N - j * S::BN;
-      if (valid < S::BN) {
-#pragma unroll
-        for (int c = 0; c < S::BN; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      // Row maximum with 8 independent partial maxima (short dependency chains).
-      float m8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-      for (int c = 8; c < S::BN; c += 8)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      const float m_new = mx * sl2;
-      bool need = false;
-      if (j == 0) {
-        m_ref = m_new;
-      } else {
-        need = m_new > m_ref + 8.0f;
-        // P_t V_{j-1} must be complete before P_t is overwritten and before O_t is
-        // rescaled.
-        if (!mbar_wait(&o_done[t], (j - 1) & 1, abort_flag, &g_attn_err)) {
+      float m_ref = -INFINITY;  // running maximum of s * sl2 used as the exponent origin
+      float l = 0.f;
+      for (int j = 0; j < nkv; ++j, ++G) {
+        if (!mbar_wait(&s_full[t], G & 1, abort_flag, &g_attn_err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-      }
-      const bool any_need = __any_sync(0xffffffffu, need);
-      const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
-      if (need) {
-        m_ref = m_new;
-        l *= alpha;
-      }
-      // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
-      const float neg = -m_ref;
-      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c16 = 0; c16 < S::BN / 8; ++c16) {
-        float e[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          e[i] = fast_exp2(fmaf(s[c16 * 8 + i], sl2, neg));
-          l8[i] += e[i];
-        }
-        const int blk = c16 >> 3, cc = c16 & 7;
-        uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
-        *dst = pack_bf16x8(e);
-      }
-      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-      if (any_need) {
-        // Scale O_t to the new exponent origin before P_t V_j accumulates into it (the
-        // wait on P_t V_{j-1} above made O_t stable).
-#pragma unroll
-        for (int c = 0; c < D; c += 16) {
-          uint32_t o[16];
-          tmem_ld16(tO + c, o);
+        float s[S::BN];
+        {
+          uint32_t raw[S::BN];
+          tmem_ld128(tS, raw);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(tO + c, o);
+          for (int c = 0; c < S::BN; ++c) s[c] = __uint_as_float(raw[c]);
         }
-        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);
+        const int valid = Nw - j * S::BN;
+        if (valid < S::BN) {
+#pragma unroll
+          for (int c = 0; c < S::BN; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        // Row maximum with 8 independent partial maxima (short dependency chains).
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < S::BN; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        const float m_new = mx * sl2;
+        bool need = false;
+        if (j == 0) {
+          m_ref = m_new;
+        } else {
+          need = m_new > m_ref + 8.0f;
+          // P_t V of the previous step must be complete before P_t is overwritten and
+          // before O_t is rescaled (at j = 0 the previous item's output wait did this).
+          if (!mbar_wait(&o_done[t], (G - 1) & 1, abort_flag, &g_attn_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const bool any_need = __any_sync(0xffffffffu, need);
+        const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+        if (need) {
+          m_ref = m_new;
+          l *= alpha;
+        }
+        // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
+        const float neg = -m_ref;
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c16 = 0; c16 < S::BN / 8; ++c16) {
+          float e[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            e[i] = fast_exp2(fmaf(s[c16 * 8 + i], sl2, neg));
+            l8[i] += e[i];
+          }
+          const int blk = c16 >> 3, cc = c16 & 7;
+          uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+          *dst = pack_bf16x8(e);
+        }
+        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        if (any_need) {
+          // Scale O_t to the new exponent origin before P_t V_j accumulates into it (the
+          // wait on P_t V_{j-1} above made O_t stable).
+#pragma unroll
+          for (int c = 0; c < D; c += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(tO + c, o);
+          }
+          tmem_st_wait();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
-    if (ok) ok = mbar_wait(&o_done[t], (nkv - 1) & 1, abort_flag, &g_attn_err);
-    if (ok) {
+      if (!ok) break;
+      // The last P V product of the item; its completion also frees P_t and O_t for
+      // the next item.
+      if (!(ok = mbar_wait(&o_done[t], (G - 1) & 1, abort_flag, &g_attn_err))) break;
       tc_fence_after();
       float o[D];
       load_cols<D>(tO, o);
-      const int n = (qp * 2 + t) * S::BM + r;
-      if (p.lse && n < N) p.lse[static_cast<size_t>(bh) * p.ld_lse + n] = m_ref + __log2f(l);
-      if (n < N) {
+      AttnItem w;  // decoded again rather than kept live through the step loop
+      attn_item<S::BM, S::BN>(p, nqp, it, w);
+      const int n = (w.qp * 2 + t) * S::BM + r;
+      if (p.lse && n < w.N) p.lse[static_cast<size_t>(w.bh) * p.ld_lse + n] = m_ref + __log2f(l);
+      if (n < w.N) {
         const float inv = 1.0f / l;
 #pragma unroll
         for (int i = 0; i < D; ++i) o[i] *= inv;
-        bf16* dst = static_cast<bf16*>(p.o) + (static_cast<size_t>(tok0) + n) * (p.H * D) + h * D;
+        bf16* dst = static_cast<bf16*>(p.o) + (static_cast<size_t>(w.tok0) + n) * (p.H * D) + w.h * D;
 #pragma unroll
         for (int g = 0; g < D / 8; ++g) reinterpret_cast<uint4*>(dst)[g] = pack_bf16x8(o + 8 * g);
       }
@@ -391,7 +457,10 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
   }
   if (!make_tmap_2d(&v, p.vt, static_cast<uint64_t>(p.B) * p.H * D, p.varlen ? p.ld_vt : p.N, p.ld_vt, D, 64, 128))
     return cudaErrorInvalidValue;
-  dim3 grid((p.N + 2 * S::BM - 1) / (2 * S::BM), p.H, p.B);
+  // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no more),
+  // or one per item when there are fewer items.
+  const long items = static_cast<long>((p.N + 2 * S::BM - 1) / (2 * S::BM)) * p.H * p.B;
+  const int grid = static_cast<int>(items < device_sm_count() ? items : device_sm_count());
   attn_fwd_tcgen05<D><<<grid, kThreads, S::SMEM_BYTES, stream>>>(q0, q1, k0, k1, v, p);
   return cudaGetLastError();
 }
