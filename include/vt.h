@@ -29,6 +29,10 @@
  *    failure of the calling thread.  No C++ exception crosses this interface.
  *  - Kernels bound every internal wait (1 s); a wait that runs out records a device
  *    error that vt_check() reports as VT_ERR_TIMEOUT.
+ *  - Devices: one process drives one GPU (the library's deployment model; several GPUs
+ *    run one process each).  Each kernel's shared-memory attribute is set once per
+ *    process, on the device current at its first launch, so a process that switches
+ *    the current device between calls is not supported.
  *  - Token order: activations of one image are t*h*w tokens.  Raster order puts token
  *    (t, row, col) at index (t*h + row)*w + col.  vt_forward keeps tokens internally in
  *    2x2-block order (the four members of a merge group consecutive) and converts at
