@@ -351,9 +351,11 @@ def comparators(V, wl, dev, stream) -> dict:
 
     # ours: the kernel on operands in its layout (as the tower's QKV epilogue leaves
     # them: v transposed); "ours_with_prep" adds vt_attention's preparation pass.
-    vt = v.transpose(-1, -2).contiguous()
+    ld_vt = (N + 7) // 8 * 8  # the kernel's row pitch of v^T: a multiple of 8
+    vt = torch.zeros((B, H, D, ld_vt), dtype=torch.bfloat16, device=dev)
+    vt[..., :N] = v.transpose(-1, -2)
     row(f"attention non-causal B={B} H={H} N={N} D={D}", 4.0 * B * H * N * N * D,
-        lambda: V.vt_attention_prepared(q, k, vt, N, o, B, H, N, D, D ** -0.5, stream),
+        lambda: V.vt_attention_prepared(q, k, vt, ld_vt, o, B, H, N, D, D ** -0.5, stream),
         {"ours_with_prep": lambda: V.vt_attention(q, k, v, o, B, H, N, D, None, None, 10000.0, D ** -0.5, ws, wsb,
                                                   stream),
          "torch_sdpa_flash": sdpa(SDPBackend.FLASH_ATTENTION), "torch_sdpa_cudnn": sdpa(SDPBackend.CUDNN_ATTENTION)})
