@@ -29,6 +29,9 @@
  *    failure of the calling thread.  No C++ exception crosses this interface.
  *  - Kernels bound every internal wait (1 s); a wait that runs out records a device
  *    error that vt_check() reports as VT_ERR_TIMEOUT.
+ *  - Tracing: with the environment variable VT_LOG set (not empty, not "0") when the
+ *    library loads, every kernel launch is written to stderr as it is issued: its
+ *    class, algorithmic FLOPs and bytes, and stream.  vt_profile_* time the launches.
  *  - Devices: one process drives one GPU (the library's deployment model; several GPUs
  *    run one process each).  Each kernel's shared-memory attribute is set once per
  *    process, on the device current at its first launch, so a process that switches

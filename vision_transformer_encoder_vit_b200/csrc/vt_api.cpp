@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -86,13 +87,28 @@ struct Profiler {
 };
 Profiler g_prof;
 
-// Brackets one launch with events when profiling is on.
+// Launch trace: with VT_LOG set to anything but empty or "0" when the library loads,
+// every launch is written to stderr as it is issued (kernel class, algorithmic FLOPs
+// and bytes, stream).  Host side only, so it also traces launches recorded into a CUDA
+// graph; off, it costs one branch per launch.
+const char* const kClassNames[CLS_COUNT] = {"gemm",           "attention",          "layernorm",
+                                            "patch_unfold",   "reorder",            "attention_prep",
+                                            "attention_backward", "backward_misc"};
+const bool g_log = [] {
+  const char* v = std::getenv("VT_LOG");
+  return v != nullptr && v[0] != '\0' && !(v[0] == '0' && v[1] == '\0');
+}();
+
+// Brackets one launch with events when profiling is on; traces it when VT_LOG is set.
 struct ProfScope {
   int cls;
   double flops, bytes;
   cudaStream_t st;
   cudaEvent_t a = nullptr;
   ProfScope(int c, double f, double b, cudaStream_t s) : cls(c), flops(f), bytes(b), st(s) {
+    if (g_log)
+      std::fprintf(stderr, "vt: launch %s flops=%.6g bytes=%.6g stream=%p\n", kClassNames[c], f, b,
+                   static_cast<void*>(s));
     if (g_prof.on) {
       std::lock_guard<std::mutex> l(g_prof.mu);
       a = g_prof.get();
