@@ -201,6 +201,19 @@ class ClockSampler:
 _ORACLE_WEIGHTS: dict = {}
 
 
+def oracle_threads() -> int:
+    """Threads the oracle's numpy arithmetic runs on: the largest BLAS pool numpy has
+    loaded (its matrix products dominate), else the host's logical CPUs."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") or 0 for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n and max(n) > 0:
+            return int(max(n))
+    except Exception:  # threadpoolctl missing or unable to inspect: fall back
+        pass
+    return os.cpu_count() or 1
+
+
 def oracle_images_per_s(cfg: dict, budget_s: float = 15.0) -> dict:
     """Times the fp64 oracle on one image: patch embedding, as many layers as fit in the
     budget (at least one), and the projector; extrapolates to all layers.  The weights
@@ -230,7 +243,7 @@ def oracle_images_per_s(cfg: dict, budget_s: float = 15.0) -> dict:
     R.projector(x, w, cfg, t, gh, gw)
     t_proj = time.perf_counter() - t0
     per_image = t_embed + cfg["layers"] * statistics.mean(layer_times) + t_proj
-    return dict(value=1.0 / per_image, unit="images/s", cores=os.cpu_count(), kind="oracle",
+    return dict(value=1.0 / per_image, unit="images/s", cores=oracle_threads(), kind="oracle",
                 sample=f"one {cfg['image'][0]}x{cfg['image'][1]} image: patch embedding, {len(layer_times)} of "
                        f"{cfg['layers']} layers (mean layer time x {cfg['layers']}), projector; numpy float64",
                 seconds=per_image)
@@ -249,7 +262,7 @@ def oracle_attention(wl: dict, budget_s: float = 15.0) -> dict:
         n_heads += 1
     dt = time.perf_counter() - t0
     per_call = dt / (n_heads * len(rows)) * N * H
-    return dict(value=1.0 / per_call, unit="calls/s", cores=os.cpu_count(), kind="oracle",
+    return dict(value=1.0 / per_call, unit="calls/s", cores=oracle_threads(), kind="oracle",
                 sample=f"{len(rows)} query rows x {n_heads} heads of the {N}-token attention, scaled to all rows "
                        f"and {H} heads", seconds=per_call)
 

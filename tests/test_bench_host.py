@@ -79,3 +79,13 @@ def test_workload_token_counts():
     assert bench.workload("attn65536")["tokens"] == 256 * 256
     with pytest.raises(SystemExit):
         bench.workload("no_such_workload")
+
+
+def test_cpu_baseline_reports_the_blas_threads():
+    import os
+    n = bench.oracle_threads()
+    assert isinstance(n, int) and 1 <= n <= max(os.cpu_count() or 1, n)
+    from threadpoolctl import threadpool_info
+    blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+    if blas:
+        assert n == max(blas)
