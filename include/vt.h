@@ -123,7 +123,10 @@ typedef struct vt_handle vt_handle;
  * merge != 2 or a head layout without a kernel. */
 VT_API vt_status vt_create(const vt_config* cfg, vt_handle** out);
 
-/* Frees the handle and the device memory it owns.  Synchronises the device. */
+/* Frees the handle and the device memory it owns.  Synchronises the device.
+ * Library-defined (the pages have no user API; this is the counterpart of dropping the
+ * encoder that VisionEncoder::new of "spark_model/layers/vision_encoder/enc_impl/
+ * init.rs" builds). */
 VT_API vt_status vt_destroy(vt_handle* h);
 
 /* Registers the n weights (all of them, in any order) on the current device, packs
@@ -135,7 +138,9 @@ VT_API vt_status vt_load_weights(vt_handle* h, const vt_weight* w, int n);
 /* Bytes of caller workspace vt_forward / vt_forward_video / vt_tower_layer /
  * vt_merge_project need for B images or clips of grid grid_thw (host int32[3] = t, h, w
  * in patches, t <= 4096).  Affine in B*t*h*w: no term grows with the square of the
- * sequence.  Host only. */
+ * sequence.  Host only.  Library-defined: it replaces the capacity policy of
+ * "spark_model/layers/vision_encoder/enc_impl/init.rs" (derive_max_patches and the
+ * [seq, seq] buffers of build_scratch) with a size that is linear in the tokens. */
 VT_API vt_status vt_workspace_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* out);
 
 /* Full forward: patch unfold -> patch embedding -> layers -> 2x2 merge -> projector.
@@ -267,6 +272,18 @@ VT_API vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32
 VT_API vt_status vt_backward(vt_handle* h, const void* saved, const int32_t* grid_thw, int B, const void* d_tower,
                              float* d_pixels, void* ws, size_t ws_bytes, void* stream);
 
+/* One tower layer backward on raster-ordered tokens: dx = J^T dy for x_out = layer_i(x_in),
+ * x_in, dy and dx device bf16 [B, h*w, hidden] (dx may equal dy).  Runs the layer's
+ * forward with saved activations and its backward with the same kernels as
+ * vt_forward_saved / vt_backward, so that a single layer of the tower's backward can be
+ * checked on its own.  Workspace: vt_tower_layer_backward_bytes (it holds the one
+ * layer's saved activations).  Still images (t = 1); VT_ERR_NOT_LOADED before
+ * vt_enable_backward.  Source as for vt_backward; the layer is the ViTBlock of
+ * "metrale_model_arch/weight_loader/qwen3_vl.rs". */
+VT_API vt_status vt_tower_layer_backward_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* ws_bytes);
+VT_API vt_status vt_tower_layer_backward(vt_handle* h, int layer, const void* x_in, const void* dy, void* dx,
+                                         const int32_t* grid_thw, int B, void* ws, size_t ws_bytes, void* stream);
+
 /* Attention backward alone, no rotary embedding: q, k, v device bf16 [B, H, N, D] (q, k
  * as the scores use them), dO device bf16 [B*N, H*D] (gradient of the output
  * [B, N, H, D]); writes dqkv device bf16 [B*N, 3*H*D] = [dq | dk | dv], each in the
@@ -364,11 +381,16 @@ VT_API vt_status vt_patch_unfold(const float* pixels, void* out, int B, int H, i
  *   pos_thw     [t*h*w, 3] (t, row, col) of each raster token, the RoPE positions
  *   merge_src   [t*h*w/4, 4] raster indices gathered by each merged token, in the
  *               member order (0,0), (0,1), (1,0), (1,1)
- * Any output pointer may be NULL. */
+ * Any output pointer may be NULL.  Library-defined debugging aid: it exposes the
+ * readings of the 2x2 merge (model card, Architecture table) and of the 3D RoPE
+ * positions ("v2_loaders" findings, section 3) for exact tests. */
 VT_API vt_status vt_index_maps(const int32_t* grid_thw, int32_t* token_order, int32_t* pos_thw, int32_t* merge_src);
 
 /* Synchronises the stream and reports device-side errors recorded by the kernels
- * (VT_ERR_TIMEOUT), clearing them, and pending launch errors (VT_ERR_CUDA). */
+ * (VT_ERR_TIMEOUT), clearing them, and pending launch errors (VT_ERR_CUDA).
+ * Library-defined: the pages' loader checks extents only with a debug assertion that
+ * release builds compile out (init.rs, build_scratch doc comment); here every wait is
+ * bounded and its failure is reported through this call. */
 VT_API vt_status vt_check(void* stream);
 
 /* Diagnostic of the failure-detection path.  Launches one CTA whose only waiting
@@ -378,7 +400,9 @@ VT_API vt_status vt_check(void* stream);
  * the CUDA context stays usable.  Nothing faults, traps or hangs. */
 VT_API vt_status vt_selftest_wait_timeout(void* stream);
 
-/* Message of the calling thread's last failed call ("" if none). */
+/* Message of the calling thread's last failed call ("" if none).  Library-defined.
+ * Thread-local rather than per handle, because several entry points (vt_attention,
+ * vt_linear, vt_layernorm, ...) take no handle. */
 VT_API const char* vt_last_error(void);
 
 /* Per-kernel-class device time of the calls made between vt_profile_begin and

@@ -263,3 +263,23 @@ def test_launch_trace_follows_vt_log():
         r = subprocess.run([sys.executable, "-c", _TRACE_CALL], cwd=root, env=env, capture_output=True, text=True,
                            timeout=120)
         assert "vt: launch" not in r.stderr
+
+
+def test_static_attention_limit_is_exact_on_the_host():
+    # vt_attention_static needs 3 * align256(B*H*D*ceil8(N)*2) bytes of its 32 MiB array.
+    # The largest accepted single part is 11184640 bytes (43690 * 256): D = 80, one head,
+    # N = 69904 tokens.  One token more rounds up to 69912 and must be rejected before
+    # anything touches the device (so fake, aligned pointers are safe here).
+    limit = V.vt_attention_static_max_bytes()
+    assert limit == 32 << 20
+    assert V.vt_attention_workspace_bytes(1, 1, 69904, 80) == 3 * 11184640 <= limit
+    assert V.vt_attention_workspace_bytes(1, 1, 69905, 80) > limit
+    fake = 1 << 20
+    for N in (69905, 69912, 1 << 20):
+        with pytest.raises(V.VtError) as e:
+            V.vt_attention_static(fake, fake, fake, fake, 1, 1, N, 80, None, None, 0.0, 80 ** -0.5)
+        assert _status(e) == "VT_ERR_WORKSPACE"
+    # the row limit of the workspace entry point holds here too (B * H * N < 2^31)
+    with pytest.raises(V.VtError) as e:
+        V.vt_attention_static(fake, fake, fake, fake, 1 << 25, 1 << 25, 256, 32, None, None, 0.0, 32 ** -0.5)
+    assert _status(e) == "VT_ERR_SHAPE"

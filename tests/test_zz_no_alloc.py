@@ -58,3 +58,20 @@ def test_static_scratch_rejects_oversized_problem():
     with pytest.raises(V.VtError) as e:
         V.vt_attention_static(q, q, q, q, 1, 16, N, 80, None, None, 0.0, 80 ** -0.5)
     assert e.value.name == "VT_ERR_WORKSPACE"
+
+
+def test_static_scratch_accepts_the_exact_limit():
+    # The largest problem the array holds: D = 80, one head, N = 69904 tokens, i.e.
+    # 3 parts of 11184640 bytes (43690 * 256), within 32 MiB.  It runs and matches
+    # vt_attention; one token more (69905, rounded up to 69912) is rejected.
+    B, H, N, D = 1, 1, 69904, 80
+    q, k, v = (dev_bf16(a) for a in S.make_qkv(B, H, N, D, 7))
+    ref = _reference(q, k, v, B, H, N, D, None, None)
+    o = empty_bf16(B, N, H * D)
+    V.vt_attention_static(q, k, v, o, B, H, N, D, None, None, 0.0, D ** -0.5)
+    V.vt_check()
+    assert_close(host_f64(o), ref, what="static-scratch attention at the exact size limit")
+    q1 = empty_bf16(B, H, N + 1, D)
+    with pytest.raises(V.VtError) as e:
+        V.vt_attention_static(q1, q1, q1, q1, B, H, N + 1, D, None, None, 0.0, D ** -0.5)
+    assert e.value.name == "VT_ERR_WORKSPACE"

@@ -13,7 +13,6 @@
 // caller.
 #include <mutex>
 
-#include "../../include/vt.h"
 #include "internal.h"
 
 namespace {
@@ -73,17 +72,11 @@ vt_status vt_attention_static_max_bytes(size_t* out) {
 vt_status vt_attention_static(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
                               const int32_t* pos_thw, const int32_t* sections, float theta, float scale,
                               void* stream) {
+  vt_status s = vt::check_attention_dims(B, H, N, D, scale);
+  if (s != VT_OK) return s;
   if (!q || !k || !v || !o) {
     vt::set_error_message("vt_attention_static: NULL operand");
     return VT_ERR_INVALID_ARG;
-  }
-  if (B <= 0 || H <= 0 || N <= 0 || !(scale > 0.f)) {
-    vt::set_error_message("vt_attention_static: B, H, N and scale must be positive");
-    return VT_ERR_INVALID_ARG;
-  }
-  if (D != 32 && D != 64 && D != 80 && D != 96) {
-    vt::set_error_message("vt_attention_static: head_dim has no kernel (32, 64, 80 or 96)");
-    return VT_ERR_UNSUPPORTED;
   }
   if (((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
         reinterpret_cast<uintptr_t>(o)) & 15u) != 0) {
@@ -108,31 +101,22 @@ vt_status vt_attention_static(const void* q, const void* k, const void* v, void*
       return VT_ERR_INVALID_ARG;
     }
   }
+  // B * H * N < 2^31 (checked above) keeps these products far inside 64 bits.
   const int ldv = (N + 7) & ~7;
   const size_t part = round_up256(static_cast<size_t>(B) * H * D * ldv * 2);
-  if (3 * part > kStaticScratchBytes) {
+  if (part > kStaticScratchBytes / 3) {
     vt::set_error_message("vt_attention_static: problem needs more scratch than the 32 MiB static array "
                           "(3 * B*H*D*ceil8(N) * 2 bytes); use vt_attention with a workspace");
     return VT_ERR_WORKSPACE;
   }
   void* base = nullptr;
-  vt_status s = scratch_address(&base);
-  if (s != VT_OK) return s;
+  if ((s = scratch_address(&base)) != VT_OK) return s;
   char* w = static_cast<char*>(base);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = vt::launch_attention_prep(q, k, v, w, w + part, w + 2 * part, B, H, N, D, ldv, pos_thw, sec,
-                                            theta, st);
-  if (e != cudaSuccess) {
-    vt::set_error_message("vt_attention_static: preparation launch failed");
-    return VT_ERR_CUDA;
-  }
+  if ((s = vt::run_attention_prep(q, k, v, w, w + part, w + 2 * part, B, H, N, D, ldv, pos_thw, sec, theta, st)))
+    return s;
   vt::AttnParams a{w, w + part, w + 2 * part, o, B, H, N, D, ldv, scale};
-  e = vt::launch_attention(a, st);
-  if (e != cudaSuccess) {
-    vt::set_error_message("vt_attention_static: attention launch failed");
-    return VT_ERR_CUDA;
-  }
-  return VT_OK;
+  return vt::run_attention(a, st);
 }
 
 }  // extern "C"

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "vt.h"
+
 namespace vt {
 
 // Token order of the activations of one image.
@@ -122,6 +124,10 @@ struct AttnParams {
   // lse[(b*H + h) * ld_lse + n] = log2(sum_j 2^(s_nj * scale * log2 e)), for the backward.
   float* lse;
   int ld_lse;
+  // Work schedule (set by launch_attention; callers leave it zero): the first sched_full
+  // items run whole in rounds of the grid, then sched_tail_pairs items form a tail of one
+  // unit per CTA, sched_tail_split of them cut into two single-tile units.
+  int sched_full, sched_tail_pairs, sched_tail_split;
 };
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream);
 unsigned int attention_read_clear_error(cudaStream_t stream);
@@ -220,5 +226,15 @@ unsigned int selftest_read_clear_error(cudaStream_t stream);
 
 // Sets the calling thread's message returned by vt_last_error().
 void set_error_message(const char* msg);
+
+// Host side of the stand-alone attention, shared by the entry points that take a
+// workspace and the one with static scratch: argument checks (positive sizes and
+// scale, a head_dim with a kernel, B * H * N rows within the 32-bit index range), and
+// the two launches, each bracketed for the launch trace and the profiler.
+vt_status check_attention_dims(int B, int H, int N, int D, float scale);
+vt_status run_attention_prep(const void* q, const void* k, const void* v, void* qr, void* kr, void* vt_, int B, int H,
+                             int N, int D, int ld_vt, const int32_t* pos, const int sections[3], float theta,
+                             cudaStream_t st);
+vt_status run_attention(const AttnParams& p, cudaStream_t st);
 
 }  // namespace vt

@@ -162,7 +162,9 @@ vt_status run_layernorm(const void* x, const void* g, const void* b, void* y, in
   return VT_OK;
 }
 
-vt_status run_attention(const AttnParams& p, cudaStream_t st) {
+}  // namespace
+
+vt_status vt::run_attention(const AttnParams& p, cudaStream_t st) {
   double n2 = static_cast<double>(p.B) * p.N * p.N, n1 = static_cast<double>(p.B) * p.N;
   if (p.varlen) {  // per-image token counts of a packed batch
     n2 = n1 = 0;
@@ -178,7 +180,22 @@ vt_status run_attention(const AttnParams& p, cudaStream_t st) {
   return VT_OK;
 }
 
-}  // namespace
+vt_status vt::run_attention_prep(const void* q, const void* k, const void* v, void* qr, void* kr, void* vt_, int B,
+                                 int H, int N, int D, int ld_vt, const int32_t* pos, const int sections[3],
+                                 float theta, cudaStream_t st) {
+  ProfScope ps(CLS_PREP, 0, 12.0 * B * H * static_cast<double>(N) * D, st);
+  cudaError_t e = launch_attention_prep(q, k, v, qr, kr, vt_, B, H, N, D, ld_vt, pos, sections, theta, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention preparation launch");
+  return VT_OK;
+}
+
+vt_status vt::check_attention_dims(int B, int H, int N, int D, float scale) {
+  if (B <= 0 || H <= 0 || N <= 0) return fail(VT_ERR_INVALID_ARG, "B, H, N must be positive");
+  if (!(scale > 0.f)) return fail(VT_ERR_INVALID_ARG, "scale must be positive");
+  if (D != 32 && D != 64 && D != 80 && D != 96) return fail(VT_ERR_UNSUPPORTED, "head_dim %d has no kernel", D);
+  if (static_cast<long long>(B) * H * N > (1ll << 31) - 256) return fail(VT_ERR_SHAPE, "too many rows");
+  return VT_OK;
+}
 
 void vt::set_error_message(const char* msg) { g_last_error = msg ? msg : ""; }
 
@@ -291,7 +308,13 @@ vt_status check_still(int t, const char* entry) {
   return VT_OK;
 }
 
-// One pre-LN layer over M tokens stored at x (in place).
+// The patch-embedding product: patch vectors U [M, K0] -> tokens x [M, hidden].
+vt_status run_patch_embed(vt_handle* h, const void* U, void* x, const Plan& pl, cudaStream_t st) {
+  const vt_config& c = h->cfg;
+  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
+  return run_gemm(gemm_params(U, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0, ACT_NONE), st);
+}
+
 // One pre-LN layer over the M tokens at x_in (written to x, which may equal x_in).  With
 // vl non-null the tokens are a packed batch of images of different grids.
 vt_status run_layer(vt_handle* h, int i, const void* x_in, void* x, int B, int gt, int gh, int gw, int order,
@@ -558,12 +581,8 @@ static vt_status forward_embedded(vt_handle* h, int B, int t, int gh, int gw, vo
                                   const Plan& pl, cudaStream_t st) {
   const vt_config& c = h->cfg;
   void* x = w + pl.x;
-  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
   vt_status s;
-  if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0,
-                                ACT_NONE),
-                    st)))
-    return s;
+  if ((s = run_patch_embed(h, w + pl.unfold, x, pl, st))) return s;
   for (int i = 0; i < c.layers; ++i)
     if ((s = run_layer(h, i, x, x, B, t, gh, gw, ORDER_BLOCK, w, pl, st))) return s;
   if (tower_out) {
@@ -823,10 +842,7 @@ vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int32_t* gr
     cudaError_t e = launch_patch_unfold_varlen(pixels, w + pl.unfold, vl, c.patch, c.temporal_patch, st);
     if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
   }
-  if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0,
-                                ACT_NONE),
-                    st)))
-    return s;
+  if ((s = run_patch_embed(h, w + pl.unfold, x, pl, st))) return s;
   // The QKV epilogue writes only each image's own v^T columns; the rest of the common
   // stride must read as zeros in the attention's P.V (P is zero there).
   {
@@ -932,13 +948,10 @@ vt_status vt_patch_embed(vt_handle* h, const float* pixels, const int32_t* grid_
   if (ws_bytes < pl.total) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, pl.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
   cudaError_t e = launch_patch_unfold(pixels, w + pl.unfold, B, gh * c.patch, gw * c.patch, c.patch, c.temporal_patch,
                                       ORDER_RASTER, st);
   if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
-  return run_gemm(
-      gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x_out, c.hidden, pl.M, c.hidden, K0, ACT_NONE),
-      st);
+  return run_patch_embed(h, w + pl.unfold, x_out, pl, st);
 }
 
 vt_status vt_merge_project(vt_handle* h, const void* tower, const int32_t* grid_thw, int B, void* out, void* ws,
@@ -969,17 +982,9 @@ vt_status vt_attention_workspace_bytes(int B, int H, int N, int D, size_t* out) 
   return VT_OK;
 }
 
-static vt_status check_attn_dims(int B, int H, int N, int D, float scale) {
-  if (B <= 0 || H <= 0 || N <= 0) return fail(VT_ERR_INVALID_ARG, "B, H, N must be positive");
-  if (!(scale > 0.f)) return fail(VT_ERR_INVALID_ARG, "scale must be positive");
-  if (D != 32 && D != 64 && D != 80 && D != 96) return fail(VT_ERR_UNSUPPORTED, "head_dim %d has no kernel", D);
-  if (static_cast<long long>(B) * H * N > (1ll << 31) - 256) return fail(VT_ERR_SHAPE, "too many rows");
-  return VT_OK;
-}
-
 vt_status vt_attention_prepared(const void* q, const void* k, const void* vt_, int ld_vt, void* o, int B, int H, int N,
                                 int D, float scale, void* stream) {
-  vt_status s = check_attn_dims(B, H, N, D, scale);
+  vt_status s = check_attention_dims(B, H, N, D, scale);
   if (s) return s;
   if (!q || !k || !vt_ || !o) return fail(VT_ERR_INVALID_ARG, "NULL operand");
   if (!aligned16(q) || !aligned16(k) || !aligned16(vt_) || !aligned16(o))
@@ -992,7 +997,7 @@ vt_status vt_attention_prepared(const void* q, const void* k, const void* vt_, i
 vt_status vt_attention(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
                        const int32_t* pos_thw, const int32_t* sections, float theta, float scale, void* ws,
                        size_t ws_bytes, void* stream) {
-  vt_status s = check_attn_dims(B, H, N, D, scale);
+  vt_status s = check_attention_dims(B, H, N, D, scale);
   if (s) return s;
   if (!q || !k || !v || !o || !ws) return fail(VT_ERR_INVALID_ARG, "NULL operand or workspace");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws))
@@ -1017,11 +1022,7 @@ vt_status vt_attention(const void* q, const void* k, const void* v, void* o, int
   void* kr = w + part;
   void* vt_ = w + 2 * part;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  {
-    ProfScope ps(CLS_PREP, 0, 12.0 * B * H * static_cast<double>(N) * D, st);
-    cudaError_t e = launch_attention_prep(q, k, v, qr, kr, vt_, B, H, N, D, ldv, pos_thw, sec, theta, st);
-    if (e != cudaSuccess) return cuda_fail(e, "attention preparation launch");
-  }
+  if ((s = run_attention_prep(q, k, v, qr, kr, vt_, B, H, N, D, ldv, pos_thw, sec, theta, st))) return s;
   AttnParams a{qr, kr, vt_, o, B, H, N, D, ldv, scale};
   return run_attention(a, st);
 }
@@ -1494,10 +1495,7 @@ vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* gri
     if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
   }
   void* x0 = c.layers > 0 ? static_cast<void*>(block(0) + sl.x) : static_cast<void*>(w + pl.x);
-  if ((s = run_gemm(gemm_params(w + pl.unfold, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x0, c.hidden, pl.M, c.hidden,
-                                K0, ACT_NONE),
-                    st)))
-    return s;
+  if ((s = run_patch_embed(h, w + pl.unfold, x0, pl, st))) return s;
   for (int i = 0; i < c.layers; ++i) {
     void* out = i + 1 < c.layers ? static_cast<void*>(block(i + 1) + sl.x) : static_cast<void*>(w + pl.x);
     if ((s = run_layer_saving(h, i, block(i), sl, out, B, gh, gw, w, pl, st))) return s;
@@ -1544,6 +1542,58 @@ vt_status vt_backward(vt_handle* h, const void* saved, const int32_t* grid_thw, 
   cudaError_t e = launch_patch_fold(w + bp.hmid, d_pixels, B, gh * c.patch, gw * c.patch, c.patch, c.temporal_patch,
                                     ORDER_BLOCK, st);
   if (e != cudaSuccess) return cuda_fail(e, "patch fold launch");
+  return VT_OK;
+}
+
+vt_status vt_tower_layer_backward_bytes(const vt_handle* h, int B, const int32_t* grid_thw, size_t* ws_bytes) {
+  if (!h || !ws_bytes) return fail(VT_ERR_INVALID_ARG, "handle and output must not be NULL");
+  int gh, gw;
+  vt_status s = check_backward_grid(h, B, grid_thw, &gh, &gw);
+  if (s) return s;
+  const vt_config& c = h->cfg;
+  *ws_bytes = align256(saved_layout(c, B, gh * gw).per_layer) +
+              std::max(make_plan(c, B, 1, gh, gw).total, make_bwd_plan(c, B, gh * gw).total);
+  return VT_OK;
+}
+
+vt_status vt_tower_layer_backward(vt_handle* h, int layer, const void* x_in, const void* dy, void* dx,
+                                  const int32_t* grid_thw, int B, void* ws, size_t ws_bytes, void* stream) {
+  vt_status s = check_loaded(h);
+  if (s) return s;
+  if (!h->bwd_pack) return fail(VT_ERR_NOT_LOADED, "call vt_enable_backward before vt_tower_layer_backward");
+  if (layer < 0 || layer >= h->cfg.layers) return fail(VT_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (!x_in || !dy || !dx || !ws) return fail(VT_ERR_INVALID_ARG, "pointers must not be NULL");
+  if (!aligned16(x_in) || !aligned16(dy) || !aligned16(dx) || !aligned16(ws))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  int gh, gw;
+  if ((s = check_backward_grid(h, B, grid_thw, &gh, &gw))) return s;
+  size_t need;
+  vt_tower_layer_backward_bytes(h, B, grid_thw, &need);
+  if (ws_bytes < need) return fail(VT_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, need);
+  const vt_config& c = h->cfg;
+  const int N = gh * gw, d = c.hidden;
+  const SavedLayout sl = saved_layout(c, B, N);
+  const Plan pl = make_plan(c, B, 1, gh, gw);
+  const BwdPlan bp = make_bwd_plan(c, B, N);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* sv = static_cast<char*>(ws);                  // the layer's saved activations
+  char* w = sv + align256(sl.per_layer);              // forward, then backward scratch
+  cudaError_t e;
+  {  // the layer runs on 2x2-block-ordered tokens, as inside the tower
+    ProfScope ps(CLS_REORDER, 0, 4.0 * pl.M * d, st);
+    if ((e = launch_reorder_rows(x_in, sv + sl.x, B, 1, gh, gw, d, 1, st)) != cudaSuccess)
+      return cuda_fail(e, "reorder launch");
+  }
+  if ((s = run_layer_saving(h, layer, sv, sl, w + pl.x, B, gh, gw, w, pl, st))) return s;
+  {
+    ProfScope ps(CLS_REORDER, 0, 4.0 * bp.M * d, st);
+    if ((e = launch_reorder_rows(dy, w + bp.dx, B, 1, gh, gw, d, 1, st)) != cudaSuccess)
+      return cuda_fail(e, "reorder launch");
+  }
+  if ((s = run_layer_backward(h, layer, sv, sl, B, gh, gw, w, bp, st))) return s;
+  ProfScope ps(CLS_REORDER, 0, 4.0 * bp.M * d, st);
+  if ((e = launch_reorder_rows(w + bp.dx, dx, B, 1, gh, gw, d, 0, st)) != cudaSuccess)
+    return cuda_fail(e, "reorder launch");
   return VT_OK;
 }
 

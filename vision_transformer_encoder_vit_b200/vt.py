@@ -79,6 +79,8 @@ _SIGS = {
     "vt_layernorm_backward": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp]),
     "vt_forward_u8": ([_vp, _vp, _i32p, _i, _i32p, _fp, _fp, _vp, _vp, _vp, _sz, _vp]),
     "vt_tower_layer": ([_vp, _i, _vp, _vp, _i32p, _i, _vp, _sz, _vp]),
+    "vt_tower_layer_backward_bytes": ([_vp, _i, _i32p, ctypes.POINTER(_sz)]),
+    "vt_tower_layer_backward": ([_vp, _i, _vp, _vp, _vp, _i32p, _i, _vp, _sz, _vp]),
     "vt_patch_embed": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_merge_project": ([_vp, _vp, _i32p, _i, _vp, _vp, _sz, _vp]),
     "vt_attention_workspace_bytes": ([_i, _i, _i, _i, ctypes.POINTER(_sz)]),
@@ -305,6 +307,18 @@ def vt_forward_host_async(h, pixels_host, grid_thw, B, out_host, ws, ws_bytes, s
 def vt_tower_layer(h, layer, x_in, x_out, grid_thw, B, ws, ws_bytes, stream=None) -> None:
     _check(lib.vt_tower_layer(h, layer, _ptr(x_in), _ptr(x_out), _grid(grid_thw), B, _ptr(ws), ws_bytes,
                               _stream(stream)), "vt_tower_layer")
+
+
+def vt_tower_layer_backward_bytes(h, B, grid_thw) -> int:
+    out = _sz()
+    _check(lib.vt_tower_layer_backward_bytes(h, B, _grid(grid_thw), ctypes.byref(out)),
+           "vt_tower_layer_backward_bytes")
+    return out.value
+
+
+def vt_tower_layer_backward(h, layer, x_in, dy, dx, grid_thw, B, ws, ws_bytes, stream=None) -> None:
+    _check(lib.vt_tower_layer_backward(h, layer, _ptr(x_in), _ptr(dy), _ptr(dx), _grid(grid_thw), B, _ptr(ws),
+                                       ws_bytes, _stream(stream)), "vt_tower_layer_backward")
 
 
 def vt_patch_embed(h, pixels, grid_thw, B, x_out, ws, ws_bytes, stream=None) -> None:
