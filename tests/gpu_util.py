@@ -6,7 +6,10 @@ Tolerances (written here once, used by every parity test):
     single kernels, <= 2e-2 for the final projected tokens;
   * element-wise |g - o| <= ELEM_RTOL * |o| + ELEM_ATOL * rms(o), a bound a few bf16
     half-ulps wide (bf16 keeps 8 significant bits, so rounding one result costs up to
-    2^-9 relative), which catches a single wrong tile that an L2 norm could average away.
+    2^-9 relative), which catches a single wrong tile that an L2 norm could average away;
+  * for outputs that crossed many bf16 layers (free-running towers), where single
+    elements drift further than a few half-ulps, a relative L2 gate on every token row
+    (assert_rows_close), which still catches a single wrong token or tile.
 """
 from __future__ import annotations
 
@@ -79,4 +82,22 @@ def assert_close(g, o, rel=REL_L2_LAYER, rtol=ELEM_RTOL, atol=ELEM_ATOL, what=""
         idx = np.unravel_index(np.argmax(np.abs(g - o) - bound), g.shape)
         raise AssertionError(f"{what}: {int(bad.sum())} elements outside the element-wise bound; worst at {idx}: "
                              f"got {g[idx]:.6g}, expected {o[idx]:.6g}")
+    return r
+
+
+def assert_rows_close(g, o, rel, rel_row, what=""):
+    """Relative L2 over the whole tensor <= rel and over every row (last axis) <= rel_row;
+    reports the worst row."""
+    g = np.asarray(g, np.float64)
+    o = np.asarray(o, np.float64)
+    assert g.shape == o.shape, f"{what}: shape {g.shape} != {o.shape}"
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    r = rel_l2(g, o)
+    g2 = g.reshape(-1, g.shape[-1])
+    o2 = o.reshape(-1, o.shape[-1])
+    per = np.linalg.norm(g2 - o2, axis=1) / np.maximum(np.linalg.norm(o2, axis=1), 1e-300)
+    worst = int(np.argmax(per))
+    report(what, rel_l2=r, gate=rel, worst_row=worst, worst_row_rel_l2=float(per[worst]), row_gate=rel_row)
+    assert r <= rel, f"{what}: relative L2 error {r:.3e} > {rel:.1e}"
+    assert per[worst] <= rel_row, f"{what}: row {worst} has relative L2 error {per[worst]:.3e} > {rel_row:.1e}"
     return r

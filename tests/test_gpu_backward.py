@@ -110,6 +110,36 @@ def test_tower_backward_full_width_two_layers_448():
     _tower_backward(S.get_config("tower448"), (448, 448), 1, affine=False, layers=2, seed=4)
 
 
+def test_tower_layer_backward_448_every_layer_teacher_forced():
+    # Every layer of the 32-layer, 1280-wide tower at 448x448 (1024 tokens) on its own:
+    # the oracle's layer input (its forward of one image, rounded to bf16) and a seeded
+    # upstream gradient go through one GPU layer backward (forward with saved
+    # activations, then backward, as in vt_forward_saved / vt_backward); the input
+    # gradient is compared with the oracle's layer backward on the same bf16 input.
+    cfg = S.get_config("tower448")
+    bits = S.make_weights(cfg, affine=True)
+    w = S.weights_f64(bits)
+    tw = V.Tower(cfg, bits)
+    V.vt_enable_backward(tw.h)
+    t, gh, gw = S.token_grid(cfg)
+    grid = (1, gh, gw)
+    N, d = gh * gw, cfg["hidden"]
+    px = S.make_pixels(cfg, batch=1)
+    ref = R.forward(px.astype(np.float64), w, cfg, keep_layers=True)
+    pos = R.positions_raster(1, gh, gw)
+    ws_bytes = V.vt_tower_layer_backward_bytes(tw.h, 1, grid)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    dx = empty_bf16(1, N, d)
+    for i in range(cfg["layers"]):
+        xin = S.bf16_bits(ref["layer_in"][i][0].astype(np.float32))
+        dy = S.make_matrix((N, d), 500 + i)
+        V.vt_tower_layer_backward(tw.h, i, dev_bf16(xin), dev_bf16(dy), dx, grid, 1, ws, ws_bytes)
+        V.vt_check()
+        refdx = R.tower_layer_backward(S.bf16_to_f64(xin), w, i, cfg, pos, S.bf16_to_f64(dy))
+        assert_close(host_f64(dx)[0], refdx, rel=REL_L2_FINAL, what=f"448 layer {i} backward (teacher-forced)")
+    tw.close()
+
+
 def test_backward_needs_enable_and_still_images():
     cfg = S.get_config("tiny")
     tw = V.Tower(cfg, S.make_weights(cfg, affine=True))
