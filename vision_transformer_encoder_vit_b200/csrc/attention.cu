@@ -99,6 +99,32 @@ __device__ __forceinline__ bool attn_item(const AttnParams& p, int nqp, int it, 
   return w.qp * 2 * BM < w.N;
 }
 
+// The CTA's work units.  Its first units are whole items (both query tiles), taken
+// with a stride of the grid over the first sched_full items; the items left after the
+// last full round form a tail of one unit per CTA, in which sched_tail_split items are
+// cut into two single-tile units (tmask 1 or 2), so that the tail spreads over more SMs
+// (a CTA with one query tile finishes its unit sooner: its softmax does not share the
+// SM).  k-th unit of this CTA: 0 none left, 1 a unit, 2 an empty unit (an item past the
+// end of a smaller image of a packed batch).
+template <int BM, int BN>
+__device__ __forceinline__ int attn_unit(const AttnParams& p, int nqp, int k, AttnItem& w, int& tmask) {
+  const int c = blockIdx.x;
+  int it = c + k * static_cast<int>(gridDim.x);
+  tmask = 3;
+  if (it >= p.sched_full) {
+    const int kt = (p.sched_full - c + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+    const int s = p.sched_tail_split;
+    if (k != kt || c >= p.sched_tail_pairs + s) return 0;
+    if (c < 2 * s) {
+      it = p.sched_full + (c >> 1);
+      tmask = 1 << (c & 1);
+    } else {
+      it = p.sched_full + s + (c - 2 * s);
+    }
+  }
+  return attn_item<BM, BN>(p, nqp, it, w) ? 1 : 2;
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
   while (!mbar_test(bar, parity)) {
@@ -145,7 +171,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nqp = (p.N + 2 * S::BM - 1) / (2 * S::BM);  // query-tile pairs of the longest image
-  const int items = nqp * p.H * p.B;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -182,16 +207,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ0);
       tma_prefetch_desc(&tmK0);
       tma_prefetch_desc(&tmV);
-      uint32_t G = 0, I = 0;  // key-tile steps and items loaded so far by this CTA
+      uint32_t G = 0, I = 0;  // key-tile steps and units loaded so far by this CTA
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+      for (int k = 0; ok; ++k) {
         AttnItem w;
-        if (!attn_item<S::BM, S::BN>(p, nqp, it, w)) continue;
-        // Q is single-buffered: the previous item's score products must have read it.
+        int tmask;
+        const int ru = attn_unit<S::BM, S::BN>(p, nqp, k, w, tmask);
+        if (ru == 0) break;
+        if (ru == 2) continue;
+        // Q is single-buffered: the previous unit's score products must have read it.
         if (I > 0 && !mbar_wait(q_empty, (I - 1) & 1, abort_flag, &g_attn_err)) break;
         const int qrow = w.tok0 * p.H + w.h * w.N + w.qp * 2 * S::BM;
-        mbar_arrive_expect_tx(q_full, 2 * S::Q_BYTES);
+        mbar_arrive_expect_tx(q_full, (tmask == 3 ? 2 : 1) * S::Q_BYTES);
         for (int t = 0; t < 2; ++t) {
+          if (!((tmask >> t) & 1)) continue;
           tma_load_2d(sQ + t * S::Q_BYTES, &tmQ0, q_full, 0, qrow + t * S::BM);
           if (S::C1) tma_load_2d(sQ + t * S::Q_BYTES + S::Q1_OFF, &tmQ1, q_full, S::C0, qrow + t * S::BM);
         }
@@ -228,9 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, S::BN);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D);
       bool issued = false, ok = true;
-      // O_t += P_t V for query tile t and the key tile of step g (j-th of its item).
-      auto issue_pv = [&](int t, uint32_t g, int j) -> bool {
-        if (!mbar_wait(&p_full[t], g & 1, abort_flag, &g_attn_err)) return false;
+      // O_t += P_t V for query tile t and the key tile of step g (j-th of its unit); c:
+      // the number of earlier steps in which tile t took part (its barrier phases).
+      auto issue_pv = [&](int t, uint32_t g, uint32_t c, int j) -> bool {
+        if (!mbar_wait(&p_full[t], c & 1, abort_flag, &g_attn_err)) return false;
         tc_fence_after();
         const uint32_t p_addr = smem_u32(sP + t * S::P_BYTES);
         const uint32_t v_addr = smem_u32(sKV + (g % S::STAGES) * S::KV_BYTES + S::K_BYTES);
@@ -245,14 +275,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       // The P V products of step g are issued after the score products of step g + 1,
-      // which may belong to the next item: the tensor pipe works on those while the
+      // which may belong to the next unit: the tensor pipe works on those while the
       // softmax warps finish step g.  pend_j < 0: nothing pending.
-      int pend_j = -1;
-      uint32_t pend_g = 0;
+      int pend_j = -1, pend_mask = 0;
+      uint32_t pend_g = 0, pend_c[2] = {0, 0};
       uint32_t G = 0, I = 0;
-      for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+      uint32_t C[2] = {0, 0};  // steps in which query tile t took part
+      auto flush = [&]() -> bool {
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (((pend_mask >> t) & 1) && !issue_pv(t, pend_g, pend_c[t], pend_j)) return false;
+        umma_commit(&kv_empty[pend_g % S::STAGES]);
+        return true;
+      };
+      for (int k = 0; ok; ++k) {
         AttnItem w;
-        if (!attn_item<S::BM, S::BN>(p, nqp, it, w)) continue;
+        int tmask;
+        const int ru = attn_unit<S::BM, S::BN>(p, nqp, k, w, tmask);
+        if (ru == 0) break;
+        if (ru == 2) continue;
+        // Unit boundary: the previous unit's last P V products go first unless this unit's
+        // query tiles have already arrived (then its first score products run while the
+        // softmax finishes the last step).
+        if (pend_j >= 0 && !mbar_test(q_full, I & 1)) {
+          if (!(ok = flush())) break;
+          pend_j = -1;
+        }
         if (!mbar_wait(q_full, I & 1, abort_flag, &g_attn_err)) {
           ok = false;
           break;
@@ -265,9 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t k_addr = smem_u32(sKV + s * S::KV_BYTES);
-          for (int t = 0; t < 2 && ok; ++t) {
-            // S_t is single-buffered: the softmax must have read S_t of step G - 1.
-            if (G >= 1 && !mbar_wait(&s_free[t], (G - 1) & 1, abort_flag, &g_attn_err)) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || !((tmask >> t) & 1)) continue;
+            // S_t is single-buffered: the softmax must have read S_t of tile t's last step.
+            if (C[t] >= 1 && !mbar_wait(&s_free[t], (C[t] - 1) & 1, abort_flag, &g_attn_err)) {
               ok = false;
               break;
             }
@@ -278,18 +328,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_bf16(tmem + t * 256, qk_desc<D>(q_addr, ks), qk_desc<D>(k_addr, ks), idesc_s, ks > 0 ? 1u : 0u);
             issued = true;
             umma_commit(&s_full[t]);
+            ++C[t];
           }
           if (!ok) break;
           if (j == w.nkv - 1) umma_commit(q_empty);
-          if (pend_j >= 0) {
-            if (!(ok = issue_pv(0, pend_g, pend_j) && issue_pv(1, pend_g, pend_j))) break;
-            umma_commit(&kv_empty[pend_g % S::STAGES]);
-          }
+          if (pend_j >= 0 && !(ok = flush())) break;
           pend_j = j;
           pend_g = G;
+          pend_mask = tmask;
+          pend_c[0] = C[0] - 1;
+          pend_c[1] = C[1] - 1;
         }
       }
-      if (ok && pend_j >= 0) ok = issue_pv(0, pend_g, pend_j) && issue_pv(1, pend_g, pend_j);
+      if (ok && pend_j >= 0) ok = flush();
       if (*abort_flag && issued) {
         umma_commit(drain);
         drain_wait(drain, 0);
@@ -306,12 +357,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale * 1.4426950408889634f;  // scale * log2(e)
     uint8_t* pbuf = sP + t * S::P_BYTES;
     bool ok = true;
-    uint32_t G = 0;  // key-tile steps done by this CTA over all its items
-    for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
+    uint32_t G = 0;  // steps in which this warpgroup's query tile took part
+    for (int k = 0; ok; ++k) {
       int Nw, nkv;
       {
         AttnItem w;
-        if (!attn_item<S::BM, S::BN>(p, nqp, it, w)) continue;
+        int tmask;
+        const int ru = attn_unit<S::BM, S::BN>(p, nqp, k, w, tmask);
+        if (ru == 0) break;
+        if (ru == 2 || !((tmask >> t) & 1)) continue;
         Nw = w.N;
         nkv = w.nkv;
       }
@@ -339,16 +393,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < S::BN; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
-        // Row maximum with 8 independent partial maxima (short dependency chains).
-        float m8[8];
+        // Row maximum: four independent chains of three-input maxima.
+        float a4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+        for (int c = 4; c + 8 <= S::BN; c += 8)
 #pragma unroll
-        for (int c = 8; c < S::BN; c += 8)
+          for (int i = 0; i < 4; ++i) a4[i] = fmax3(a4[i], s[c + i], s[c + 4 + i]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int i = 0; i < 4; ++i) a4[i] = fmaxf(a4[i], s[S::BN - 4 + i]);
+        const float mx = fmax3(a4[0], a4[1], fmaxf(a4[2], a4[3]));
         const float m_new = mx * sl2;
         bool need = false;
         if (j == 0) {
@@ -370,21 +423,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
         }
         // P = exp2(s * sl2 - m_ref), written bf16 in the 128-byte-swizzled K-major layout.
-        const float neg = -m_ref;
-        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float2 sl2x2 = make_float2(sl2, sl2), negx2 = make_float2(-m_ref, -m_ref);
+        float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c16 = 0; c16 < S::BN / 8; ++c16) {
           float e[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            e[i] = fast_exp2(fmaf(s[c16 * 8 + i], sl2, neg));
-            l8[i] += e[i];
+          for (int q = 0; q < 4; ++q) {
+            const float2 x = ffma2(make_float2(s[c16 * 8 + 2 * q], s[c16 * 8 + 2 * q + 1]), sl2x2, negx2);
+            const float2 y = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            e[2 * q] = y.x;
+            e[2 * q + 1] = y.y;
+            l4[q] = fadd2(l4[q], y);
           }
           const int blk = c16 >> 3, cc = c16 & 7;
           uint4* dst = reinterpret_cast<uint4*>(pbuf + blk * (S::BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
           *dst = pack_bf16x8(e);
         }
-        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        const float2 l2 = fadd2(fadd2(l4[0], l4[1]), fadd2(l4[2], l4[3]));
+        l += l2.x + l2.y;
         if (any_need) {
           // Scale O_t to the new exponent origin before P_t V_j accumulates into it (the
           // wait on P_t V_{j-1} above made O_t stable).
@@ -411,7 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float o[D];
       load_cols<D>(tO, o);
       AttnItem w;  // decoded again rather than kept live through the step loop
-      attn_item<S::BM, S::BN>(p, nqp, it, w);
+      int tmask;
+      attn_unit<S::BM, S::BN>(p, nqp, k, w, tmask);
       const int n = (w.qp * 2 + t) * S::BM + r;
       if (p.lse && n < w.N) p.lse[static_cast<size_t>(w.bh) * p.ld_lse + n] = m_ref + __log2f(l);
       if (n < w.N) {
@@ -457,11 +515,28 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
   }
   if (!make_tmap_2d(&v, p.vt, static_cast<uint64_t>(p.B) * p.H * D, p.varlen ? p.ld_vt : p.N, p.ld_vt, D, 64, 128))
     return cudaErrorInvalidValue;
-  // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no more),
-  // or one per item when there are fewer items.
+  // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no more).
+  // Full rounds of whole items, then a tail in which as many of the remaining items as
+  // there are otherwise idle SMs are cut into single-tile units.  Packed batches of
+  // mixed sizes (which have empty items) run whole items only.
+  AttnParams ps = p;
   const long items = static_cast<long>((p.N + 2 * S::BM - 1) / (2 * S::BM)) * p.H * p.B;
-  const int grid = static_cast<int>(items < device_sm_count() ? items : device_sm_count());
-  attn_fwd_tcgen05<D><<<grid, kThreads, S::SMEM_BYTES, stream>>>(q0, q1, k0, k1, v, p);
+  const int sms = device_sm_count();
+  int grid;
+  if (p.varlen) {
+    ps.sched_full = static_cast<int>(items);
+    ps.sched_tail_pairs = ps.sched_tail_split = 0;
+    grid = static_cast<int>(items < sms ? items : sms);
+  } else {
+    const long full = items / sms * sms, rest = items - full;
+    const long split = rest < sms - rest ? rest : sms - rest;
+    ps.sched_full = static_cast<int>(full);
+    ps.sched_tail_pairs = static_cast<int>(rest);
+    ps.sched_tail_split = static_cast<int>(split);
+    grid = full > 0 ? sms : static_cast<int>(rest + split);
+  }
+  if (grid <= 0) return cudaSuccess;
+  attn_fwd_tcgen05<D><<<grid, kThreads, S::SMEM_BYTES, stream>>>(q0, q1, k0, k1, v, ps);
   return cudaGetLastError();
 }
 
