@@ -52,55 +52,73 @@ __device__ __forceinline__ typename VecT<VEC>::T pack_vec(const float* f) {
   return u;
 }
 
-// The row stays packed as bf16 in registers (VEC/2 words per vector) and is unpacked
-// on the fly in each pass, which keeps register use low enough for many warps per SM:
-// the kernel is latency-bound otherwise.
+// The rows stay packed as bf16 in registers (VEC/2 words per vector) and are unpacked
+// on the fly in each pass.  A warp walks rows with a stride of all warps of the grid
+// (a few rows each, the grid sized to the SMs) and loads its next row while it
+// normalises the current one, so that reading and writing overlap in every warp; gamma
+// and beta are read through L1, where they stay for all rows of the SM.
 template <int VEC, int NV>
-__global__ void __launch_bounds__(128) layernorm_warp(const bf16* __restrict__ x, const bf16* __restrict__ gamma,
-                                                      const bf16* __restrict__ beta, bf16* __restrict__ y, int rows,
-                                                      float eps) {
+__global__ void __launch_bounds__(256, 2) layernorm_warp(const bf16* __restrict__ x, const bf16* __restrict__ gamma,
+                                                         const bf16* __restrict__ beta, bf16* __restrict__ y,
+                                                         int rows, float eps) {
   typedef typename VecT<VEC>::T V;
   constexpr int COLS = 32 * VEC * NV;
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * (blockDim.x >> 5);
+  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
-  const V* xr = reinterpret_cast<const V*>(x + static_cast<size_t>(row) * COLS);
-  V xv[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) xv[i] = xr[i * 32 + lane];
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    float f[VEC];
-    unpack_vec<VEC>(xv[i], f);
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) s += f[e];
-  }
-  const float mean = warp_sum(s) * (1.0f / COLS);
-  float q = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    float f[VEC];
-    unpack_vec<VEC>(xv[i], f);
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const float d = f[e] - mean;
-      q += d * d;
-    }
-  }
-  const float rstd = rsqrtf(warp_sum(q) * (1.0f / COLS) + eps);
   const V* gr = reinterpret_cast<const V*>(gamma);
   const V* br = reinterpret_cast<const V*>(beta);
-  V* yr = reinterpret_cast<V*>(y + static_cast<size_t>(row) * COLS);
+  V xv[NV];
+  {
+    const V* xr = reinterpret_cast<const V*>(x + static_cast<size_t>(row) * COLS);
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    float f[VEC], g[VEC], bb[VEC], o[VEC];
-    unpack_vec<VEC>(xv[i], f);
-    unpack_vec<VEC>(__ldg(gr + i * 32 + lane), g);
-    unpack_vec<VEC>(__ldg(br + i * 32 + lane), bb);
+    for (int i = 0; i < NV; ++i) xv[i] = xr[i * 32 + lane];
+  }
+  for (; row < rows; row += stride) {
+    const int next = row + stride;
+    V xn[NV];
+    if (next < rows) {
+      const V* xr = reinterpret_cast<const V*>(x + static_cast<size_t>(next) * COLS);
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) o[e] = (f[e] - mean) * rstd * g[e] + bb[e];
-    yr[i * 32 + lane] = pack_vec<VEC>(o);
+      for (int i = 0; i < NV; ++i) xn[i] = xr[i * 32 + lane];
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      float f[VEC];
+      unpack_vec<VEC>(xv[i], f);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) s += f[e];
+    }
+    const float mean = warp_sum(s) * (1.0f / COLS);
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      float f[VEC];
+      unpack_vec<VEC>(xv[i], f);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float d = f[e] - mean;
+        q += d * d;
+      }
+    }
+    const float rstd = rsqrtf(warp_sum(q) * (1.0f / COLS) + eps);
+    V* yr = reinterpret_cast<V*>(y + static_cast<size_t>(row) * COLS);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      float f[VEC], g[VEC], bb[VEC], o[VEC];
+      unpack_vec<VEC>(xv[i], f);
+      unpack_vec<VEC>(__ldg(gr + i * 32 + lane), g);
+      unpack_vec<VEC>(__ldg(br + i * 32 + lane), bb);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) o[e] = (f[e] - mean) * rstd * g[e] + bb[e];
+      yr[i * 32 + lane] = pack_vec<VEC>(o);
+    }
+    if (next < rows) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) xv[i] = xn[i];
+    }
   }
 }
 
@@ -293,14 +311,16 @@ cudaError_t launch_layernorm(const void* x, const void* gamma, const void* beta,
   const bf16* G = static_cast<const bf16*>(gamma);
   const bf16* Bt = static_cast<const bf16*>(beta);
   bf16* Y = static_cast<bf16*>(y);
-  const int blocks = (rows + 3) / 4;  // 4 warps (rows) per 128-thread block
-  if (cols == 1280) layernorm_warp<8, 5><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
-  else if (cols == 1024) layernorm_warp<8, 4><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
-  else if (cols == 768) layernorm_warp<8, 3><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
-  else if (cols == 512) layernorm_warp<8, 2><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
-  else if (cols == 256) layernorm_warp<8, 1><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
-  else if (cols == 128) layernorm_warp<4, 1><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
-  else if (cols == 64) layernorm_warp<2, 1><<<blocks, 128, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  // 8 warps (rows at a time) per block, at most two blocks per SM
+  const int need = (rows + 7) / 8, cap = 2 * device_sm_count();
+  const int blocks = need < cap ? need : cap;
+  if (cols == 1280) layernorm_warp<8, 5><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  else if (cols == 1024) layernorm_warp<8, 4><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  else if (cols == 768) layernorm_warp<8, 3><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  else if (cols == 512) layernorm_warp<8, 2><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  else if (cols == 256) layernorm_warp<8, 1><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  else if (cols == 128) layernorm_warp<4, 1><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
+  else if (cols == 64) layernorm_warp<2, 1><<<blocks, 256, 0, stream>>>(X, G, Bt, Y, rows, eps);
   else layernorm_block<<<rows, 256, 0, stream>>>(X, G, Bt, Y, cols, eps);
   return cudaGetLastError();
 }
