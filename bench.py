@@ -214,6 +214,18 @@ def oracle_threads() -> int:
     return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first entry of /proc/cpuinfo), or the platform's."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def oracle_images_per_s(cfg: dict, budget_s: float = 15.0) -> dict:
     """Times the fp64 oracle on one image: patch embedding, as many layers as fit in the
     budget (at least one), and the projector; extrapolates to all layers.  The weights
@@ -227,6 +239,7 @@ def oracle_images_per_s(cfg: dict, budget_s: float = 15.0) -> dict:
     px = S.make_pixels(cfg, batch=1)[0].astype(np.float64)
     t, gh, gw = S.token_grid(cfg)
     pos = R.positions_raster(t, gh, gw)
+    t_sample = time.perf_counter()
     t0 = time.perf_counter()
     x = R.patch_embed(R.patch_unfold(px, cfg["patch"], cfg["temporal_patch"]), w["embeddings.proj.weight"],
                       w["embeddings.proj.bias"])
@@ -243,7 +256,8 @@ def oracle_images_per_s(cfg: dict, budget_s: float = 15.0) -> dict:
     R.projector(x, w, cfg, t, gh, gw)
     t_proj = time.perf_counter() - t0
     per_image = t_embed + cfg["layers"] * statistics.mean(layer_times) + t_proj
-    return dict(value=1.0 / per_image, unit="images/s", cores=oracle_threads(), kind="oracle",
+    return dict(value=1.0 / per_image, unit="images/s", cores=oracle_threads(), cpu_model=cpu_model(), kind="oracle",
+                timed_s=time.perf_counter() - t_sample,
                 sample=f"one {cfg['image'][0]}x{cfg['image'][1]} image: patch embedding, {len(layer_times)} of "
                        f"{cfg['layers']} layers (mean layer time x {cfg['layers']}), projector; numpy float64",
                 seconds=per_image)
@@ -262,7 +276,8 @@ def oracle_attention(wl: dict, budget_s: float = 15.0) -> dict:
         n_heads += 1
     dt = time.perf_counter() - t0
     per_call = dt / (n_heads * len(rows)) * N * H
-    return dict(value=1.0 / per_call, unit="calls/s", cores=oracle_threads(), kind="oracle",
+    return dict(value=1.0 / per_call, unit="calls/s", cores=oracle_threads(), cpu_model=cpu_model(), kind="oracle",
+                timed_s=dt,
                 sample=f"{len(rows)} query rows x {n_heads} heads of the {N}-token attention, scaled to all rows "
                        f"and {H} heads", seconds=per_call)
 
@@ -295,8 +310,11 @@ def run_reference(args, wl):
                 impl="reference",
                 config=dict(workload=wl["name"], description=wl["desc"], global_batch=wl["batch"],
                             tokens_per_image=wl["tokens"]),
-                cpu_baseline=dict(value=value, unit=unit, cores=steps[0]["cores"], kind="oracle",
-                                  sample=steps[0]["sample"]),
+                cpu_baseline=dict(value=value, unit=unit, cores=steps[0]["cores"], cpu_model=steps[0]["cpu_model"],
+                                  kind="oracle", sample=steps[0]["sample"]),
+                # each step times a bounded sample and scales it to the whole workload:
+                # ms_per_step is that extrapolation, timed_seconds what was actually timed
+                extrapolated=True, timed_seconds=sum(s["timed_s"] for s in steps),
                 e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
 
@@ -391,25 +409,15 @@ def comparators(V, wl, dev, stream) -> dict:
                 torch=torch.__version__, rows=rows)
 
 
-def run_gpu(args, wl):
-    import torch
-    import torch.distributed as dist
-
-    rank, world, local = REP.rank_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    from vision_transformer_encoder_vit_b200 import vt as V
-
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
-    peaks, peaks_kind = load_peaks()
+def setup_step(wl, V, torch, dev, rank):
+    """Synthetic inputs and buffers of one step of workload `wl` on this rank, and the
+    launch of that step on a given stream.  Returns every local of the set-up (the
+    end-to-end leg reuses the host buffers)."""
+    import types
     B = wl["batch"]
     grid = wl.get("grid")
     N = wl["tokens"]
     extra_cfg = {}  # workload-specific config entries of the JSON line
-
     if wl["kind"] == "tower":
         cfg = wl["cfg"]
         tower = V.Tower(cfg, S.make_weights(cfg))
@@ -528,6 +536,15 @@ def run_gpu(args, wl):
         step_flops = 4.0 * H * N * N * D
         units_per_step = 1
         unit = "calls/s"
+    return types.SimpleNamespace(**locals())
+
+def time_steps(args, ctx, V, torch, dist, dev, stream, world, local, steps, warmup, profile_steps):
+    """Warm-up, optional CUDA graph of one step, then `steps` timed steps (CUDA events on
+    the launching stream, L2 flushed between steps outside the events, clocks sampled,
+    maximum over ranks), then `profile_steps` steps with every launch bracketed by
+    events for the per-kernel-class times."""
+    import types
+    launch = ctx.launch
 
     def step():
         launch(stream)
@@ -535,7 +552,7 @@ def run_gpu(args, wl):
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     # warm-up (also compiles nothing: the library is prebuilt; first calls set kernel attributes)
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         step()
     V.vt_check(stream)
 
@@ -570,9 +587,9 @@ def run_gpu(args, wl):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for i in range(args.steps):
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
         timed_step()
@@ -584,30 +601,86 @@ def run_gpu(args, wl):
     V.vt_check(stream)
     ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms = REP.max_over_ranks(ms, dev)
-    ms_per_step = ms / args.steps
-    value = REP.job_throughput(units_per_step, args.steps, ms, world)
+    ms_per_step = ms / steps
+    value = REP.job_throughput(ctx.units_per_step, steps, ms, world)
 
     # ---------------- per-kernel-class times of one profiled step (events around each launch)
     V.vt_profile_begin(stream)
-    for _ in range(args.profile_steps):
+    for _ in range(profile_steps):
         flush.fill_(1)
         step()
     V.vt_profile_end(stream)
     prof = V.vt_profile_read()
-    launches_per_step = sum(v["launches"] for v in prof.values()) / args.profile_steps
+    launches_per_step = sum(v["launches"] for v in prof.values()) / profile_steps
+    return types.SimpleNamespace(value=value, ms=ms, ms_per_step=ms_per_step, prof=prof, graph=graph, clk=clk,
+                                 launches_per_step=launches_per_step, flush=flush)
 
+
+def summarize(prof, profile_steps, peaks, peaks_kind, wl_name):
+    """Roofline of the dominant kernel class (against the measured burst bf16 peak: the
+    kernels run inside steps of milliseconds to a tenth of a second, at burst clocks) and
+    the per-class times of the profiled steps."""
+    dom = max(("gemm", "attention", "attention_backward"), key=lambda c: prof[c]["ms"])
+    p = prof[dom]
+    achieved = p["flops"] / (p["ms"] / 1000.0) / 1e12 if p["ms"] > 0 else 0.0
+    peak = peaks["bf16_tflops"]
+    roofline = dict(bound="tensor", kernel={"gemm": "gemm_bf16_tcgen05 (all linear layers)",
+                                            "attention": "attn_fwd_tcgen05",
+                                            "attention_backward": "attn_bwd_dq + attn_bwd_dkdv"}[dom],
+                    achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
+                    peak_source=f"{peaks_kind} bf16 burst",
+                    frac_of_sustained=achieved / peaks["bf16_tflops_sustained"],
+                    frac_of_nominal=achieved / NOMINAL_BF16_TFLOPS,
+                    traffic=recorded_traffic(dom, {"tower448": "tower448_b8"}.get(wl_name, wl_name)),
+                    traffic_unit="bytes per launch (ncu dram read + write)",
+                    per_launch_flops=p["flops"] / max(p["launches"], 1),
+                    avg_launch_us=1000.0 * p["ms"] / max(p["launches"], 1))
+    classes = {k: dict(ms_per_step=v["ms"] / profile_steps,
+                       launches_per_step=v["launches"] / profile_steps,
+                       tflops=(v["flops"] / (v["ms"] / 1000.0) / 1e12) if v["ms"] > 0 and v["flops"] else None,
+                       gbs=(v["bytes"] / (v["ms"] / 1000.0) / 1e9) if v["ms"] > 0 and v["bytes"] and
+                       not v["flops"] else None)
+               for k, v in prof.items() if v["launches"]}
+    return roofline, classes
+
+
+def run_gpu(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = REP.rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    from vision_transformer_encoder_vit_b200 import vt as V
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks, peaks_kind = load_peaks()
+    ctx = setup_step(wl, V, torch, dev, rank)
+    B, grid, N, unit = ctx.B, ctx.grid, ctx.N, ctx.unit
+    tm = time_steps(args, ctx, V, torch, dist, dev, stream, world, local, args.steps, args.warmup,
+                    args.profile_steps)
+    value, ms, ms_per_step, prof, graph, clk = tm.value, tm.ms, tm.ms_per_step, tm.prof, tm.graph, tm.clk
+    launches_per_step = tm.launches_per_step
+    flush = tm.flush
+
+
+    # ---------------- end to end through the C ABI with host buffers
+    e2e = None
     # ---------------- end to end through the C ABI with host buffers
     e2e = None
     if wl["kind"] == "tower":
         # A serving pipeline: batches alternate between two streams, each with its own
         # workspace and pinned output, so one batch's copies overlap the other's forward.
         # Every step still copies its pixels in and its projected tokens out.
-        wsb_h = V.vt_forward_host_workspace_bytes(tower.h, B, grid)
+        wsb_h = V.vt_forward_host_workspace_bytes(ctx.tower.h, B, grid)
         ws_h = [torch.empty(wsb_h, dtype=torch.uint8, device=dev) for _ in range(2)]
-        out_h = [torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        out_h = [torch.empty((B, N // 4, ctx.cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         streams = [stream, torch.cuda.Stream(device=dev)]
         for i in range(2):
-            V.vt_forward_host(tower.h, px_host, grid, B, out_h[i], ws_h[i], wsb_h, streams[i])
+            V.vt_forward_host(ctx.tower.h, ctx.px_host, grid, B, out_h[i], ws_h[i], wsb_h, streams[i])
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -616,28 +689,29 @@ def run_gpu(args, wl):
         e_s.record(stream)
         streams[1].wait_event(e_s)
         for i in range(args.steps):
-            V.vt_forward_host_async(tower.h, px_host, grid, B, out_h[i % 2], ws_h[i % 2], wsb_h, streams[i % 2])
+            V.vt_forward_host_async(ctx.tower.h, ctx.px_host, grid, B, out_h[i % 2], ws_h[i % 2], wsb_h, streams[i % 2])
         stream.wait_stream(streams[1])
         e_e.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e_s.elapsed_time(e_e)
         e2e_ms = REP.max_over_ranks(e2e_ms, dev)
         e2e = dict(value=REP.job_throughput(B, args.steps, e2e_ms, world), unit=unit,
-                   h2d_bytes_per_step=int(px_host.numel() * 4), d2h_bytes_per_step=int(out_h[0].numel() * 2),
+                   h2d_bytes_per_step=int(ctx.px_host.numel() * 4), d2h_bytes_per_step=int(out_h[0].numel() * 2),
                    api="vt_forward_host_async, two streams")
         del ws_h
     elif wl["kind"] == "u8":
         # decoded images from pinned host memory -> device, forward, projected tokens back;
         # batches alternate between two streams with their own buffers (serving pipeline)
         streams = [stream, torch.cuda.Stream(device=dev)]
-        bufs = [(img, ws, out), (torch.empty_like(img), torch.empty_like(ws), torch.empty_like(out))]
-        out_h = [torch.empty((B, N // 4, cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        bufs = [(ctx.img, ctx.ws, ctx.out),
+                (torch.empty_like(ctx.img), torch.empty_like(ctx.ws), torch.empty_like(ctx.out))]
+        out_h = [torch.empty((B, N // 4, ctx.cfg["proj_out"]), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
 
         def e2e_step(i):
             im, w_, o_ = bufs[i % 2]
             with torch.cuda.stream(streams[i % 2]):
-                im.copy_(img_host, non_blocking=True)
-                V.vt_forward_u8(tower.h, im, sizes, grid, o_, None, w_, w_.numel(), stream=streams[i % 2])
+                im.copy_(ctx.img_host, non_blocking=True)
+                V.vt_forward_u8(ctx.tower.h, im, ctx.sizes, grid, o_, None, w_, w_.numel(), stream=streams[i % 2])
                 out_h[i % 2].copy_(o_, non_blocking=True)
 
         e2e_step(0)
@@ -656,38 +730,35 @@ def run_gpu(args, wl):
         torch.cuda.synchronize()
         e2e_ms = REP.max_over_ranks(e_s.elapsed_time(e_e), dev)
         e2e = dict(value=REP.job_throughput(B, args.steps, e2e_ms, world), unit=unit,
-                   h2d_bytes_per_step=int(img_host.numel()), d2h_bytes_per_step=int(out_h[0].numel() * 2),
+                   h2d_bytes_per_step=int(ctx.img_host.numel()), d2h_bytes_per_step=int(out_h[0].numel() * 2),
                    api="vt_forward_u8 (+ host copies), two streams")
+
+    # The second headline configuration: one 2016x2016 image (20736 tokens) through the
+    # same path, timed the same way after the main workload (its buffers released).
+    secondary = None
+    if wl["name"] == "tower448" and args.secondary_steps > 0:
+        wl2 = workload("tower2016")
+        ctx2 = setup_step(wl2, V, torch, dev, rank)
+        tm2 = time_steps(args, ctx2, V, torch, dist, dev, stream, world, local, args.secondary_steps, 3, 1)
+        if rank == 0:
+            roof2, classes2 = summarize(tm2.prof, 1, peaks, peaks_kind, wl2["name"])
+            secondary = dict(workload=wl2["name"], description=wl2["desc"], value=tm2.value, unit=ctx2.unit,
+                             steps=args.secondary_steps, warmup=3, ms_per_step=tm2.ms_per_step,
+                             tokens_per_s=tm2.value * wl2["tokens"], output_tokens_per_s=tm2.value * wl2["tokens"] / 4,
+                             tflops=world * ctx2.step_flops * args.secondary_steps / (tm2.ms / 1000.0) / 1e12,
+                             launch="cuda graph" if tm2.graph else "eager", roofline=roof2, kernel_classes=classes2,
+                             clocks=tm2.clk)
+        del ctx2, tm2
 
     comp = comparators(V, wl, dev, stream) if args.comparators and rank == 0 else None
 
     if rank == 0:
-        # dominant kernel class by device time
-        dom = max(("gemm", "attention", "attention_backward"), key=lambda c: prof[c]["ms"])
-        p = prof[dom]
-        achieved = p["flops"] / (p["ms"] / 1000.0) / 1e12 if p["ms"] > 0 else 0.0
-        peak = peaks["bf16_tflops_sustained"]
-        roofline = dict(bound="tensor", kernel={"gemm": "gemm_bf16_tcgen05 (all linear layers)",
-                                                "attention": "attn_fwd_tcgen05",
-                                                "attention_backward": "attn_bwd_dq + attn_bwd_dkdv"}[dom],
-                        achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
-                        peak_source=f"{peaks_kind} bf16 sustained",
-                        frac_of_burst=achieved / peaks["bf16_tflops"], frac_of_nominal=achieved / NOMINAL_BF16_TFLOPS,
-                        traffic=recorded_traffic(dom, {"tower448": "tower448_b8"}.get(wl["name"], wl["name"])),
-                        traffic_unit="bytes per launch (ncu dram read + write)",
-                        per_launch_flops=p["flops"] / max(p["launches"], 1),
-                        avg_launch_us=1000.0 * p["ms"] / max(p["launches"], 1))
-        classes = {k: dict(ms_per_step=v["ms"] / args.profile_steps,
-                           launches_per_step=v["launches"] / args.profile_steps,
-                           tflops=(v["flops"] / (v["ms"] / 1000.0) / 1e12) if v["ms"] > 0 and v["flops"] else None,
-                           gbs=(v["bytes"] / (v["ms"] / 1000.0) / 1e9) if v["ms"] > 0 and v["bytes"] and
-                           not v["flops"] else None)
-                   for k, v in prof.items() if v["launches"]}
+        roofline, classes = summarize(prof, args.profile_steps, peaks, peaks_kind, wl["name"])
         cpu = None
         if world == 1 and not args.no_cpu_baseline and wl["kind"] in ("tower", "attn"):
-            cpu = (oracle_images_per_s(wl["cfg"], args.cpu_budget) if wl["kind"] == "tower"
+            cpu = (oracle_images_per_s(ctx.cfg, args.cpu_budget) if wl["kind"] == "tower"
                    else oracle_attention(wl, args.cpu_budget))
-            cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            cpu = {k: cpu[k] for k in ("value", "unit", "cores", "cpu_model", "kind", "sample")}
         # tokens of one image (clip); a packed varlen batch reports its mean image
         per_unit = N / B if wl["kind"] == "varlen" else N
         line = dict(
@@ -697,15 +768,17 @@ def run_gpu(args, wl):
             config=dict(workload=wl["name"], description=wl["desc"], per_gpu_batch=B, global_batch=B * world,
                         tokens_per_image=per_unit, merged_tokens_per_image=per_unit / 4,
                         l2="flushed (512 MB write) between timed steps", launch="cuda graph" if graph else "eager",
-                        parallelism=f"replicas x{world}", **extra_cfg),
+                        parallelism=f"replicas x{world}", **ctx.extra_cfg),
             tokens_per_s=value * per_unit if wl["kind"] not in ("attn", "attn_bwd") else None,
             output_tokens_per_s=value * per_unit / 4 if wl["kind"] not in ("attn", "attn_bwd") else None,
-            tflops=world * step_flops * args.steps / (ms / 1000.0) / 1e12,
+            tflops=world * ctx.step_flops * args.steps / (ms / 1000.0) / 1e12,
             roofline=roofline, kernel_classes=classes,
             cpu_baseline=cpu, e2e=e2e,
             gpu_launches=int(round(launches_per_step * args.steps)),
             clocks=clk,
         )
+        if secondary is not None:
+            line["secondary"] = secondary
         if comp is not None:
             line["comparators"] = comp
         print(json.dumps(line), flush=True)
@@ -723,6 +796,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=2)
+    ap.add_argument("--secondary-steps", type=int, default=5,
+                    help="timed steps of the 2016x2016 configuration measured after tower448 (0: skip)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--comparators", action="store_true",
