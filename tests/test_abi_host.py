@@ -117,6 +117,9 @@ def test_workspace_is_affine_in_tokens():
     b = (ws[-1] - ws[-3]) / (ns[-1] - ns[-3])
     a = ws[-1] - b * ns[-1]
     assert np.all(np.abs(ws - (a + b * ns)) <= 16 * 256), (a, b)
+    # the constant part is the linear layers' split-K scratch: one 256 x 256 fp32 tile
+    # per pair of SMs (the host falls back to 148 SMs without a device)
+    assert 0 < a <= 74 * 256 * 256 * 4 + 16 * 256
     # per token: the residual stream x (2d bytes) plus the larger of the tower phase
     # (LN out, q, k, v^T, o: 5 x 2d, MLP hidden 2m) and the projector phase (two
     # P-wide activations and a quarter-row merged hidden: 2P + 2P + 2P/4)
@@ -137,7 +140,10 @@ def test_varlen_workspace_and_argument_checks():
     assert V.vt_workspace_bytes_varlen(h, [(1, 32, 32)]) == one
     mixed = V.vt_workspace_bytes_varlen(h, [(1, 32, 32), (1, 16, 24), (1, 2, 2)])
     tokens = 1024 + 384 + 4
-    assert one < mixed <= 30208 * tokens + 64 * 256  # affine in the packed token count
+    # affine in the packed token count: the fixed split-K scratch plus 30208 bytes per token
+    fixed = one - 30208 * 1024
+    assert 0 < fixed <= 74 * 256 * 256 * 4 + 16 * 256
+    assert one < mixed <= fixed + 30208 * tokens + 64 * 256
     with pytest.raises(V.VtError) as e:
         V.vt_workspace_bytes_varlen(h, [(1, 32, 32), (1, 15, 24)])
     assert _status(e) == "VT_ERR_SHAPE"

@@ -108,6 +108,31 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Work item i (0, 1, ...) of CTA pair `pair` of P: output tile `tile` over K steps
+// [kb0, kb1).  Whole tiles come in rounds of P; with a split-K tail (p.sk_part) the
+// tiles from p.sk_full on are cut into p.sk_split K ranges each, and pair u takes range
+// u % sk_split of tile sk_full + u / sk_split as its last item (unit = u; -1 for a whole
+// tile).  Every role of the kernel walks the same items.
+__device__ __forceinline__ bool pair_work(const GemmParams& p, int pair, int P, int T, int nk, int i, int& tile,
+                                          int& kb0, int& kb1, int& unit) {
+  const int F = p.sk_part ? p.sk_full : T;
+  const int whole = pair < F ? (F - pair + P - 1) / P : 0;
+  if (i < whole) {
+    tile = pair + i * P;
+    kb0 = 0;
+    kb1 = nk;
+    unit = -1;
+    return true;
+  }
+  if (!p.sk_part || i != whole || pair >= (T - F) * p.sk_split) return false;
+  const int sp = pair % p.sk_split;
+  tile = F + pair / p.sk_split;
+  kb0 = sp * nk / p.sk_split;
+  kb1 = (sp + 1) * nk / p.sk_split;
+  unit = pair;
+  return true;
+}
+
 // Drains one accumulator: this thread's row `row`, columns [col0, col0 + BN), the
 // warp's TMEM lane quadrant at t_row.  Waits for the accumulator (tfull, phase
 // `parity`) itself, after issuing the loads it can issue early.  Returns false on abort.
@@ -514,10 +539,11 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       // full[stage], armed by the even CTA for the bytes of both.
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      int tile, kb0, kb1, unit;
+      for (int i = 0; pair_work(p, pair, num_pairs, num_tiles, nk, i, tile, kb0, kb1, unit); ++i) {
         const int mb = tile % m_tiles, nb = tile / m_tiles;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) {
             ok = false;
             break;
@@ -558,13 +584,14 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       uint32_t phase = 0;
       int it = 0;
       bool issued_any = false;
-      for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+      int tile, kb0, kb1, unit;
+      for (; pair_work(p, pair, num_pairs, num_tiles, nk, it, tile, kb0, kb1, unit); ++it) {
         const int acc = it & 1;
         if (!mbar_wait_cluster(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, &g_gemm_err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_cluster(&full[stage], phase, abort_flag, &g_gemm_err)) {
             ok = false;
             break;
@@ -575,7 +602,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             umma_bf16_pair(d_tmem, smem_desc(a_addr + kk * 32, 1024, 2), smem_desc(b_addr + kk * 32, 1024, 2),
-                           idesc, (kb | kk) != 0 ? 1u : 0u);
+                           idesc, (kb > kb0 || kk != 0) ? 1u : 0u);
           }
           issued_any = true;
           const uint32_t e_local = smem_u32(&empty[stage]);
@@ -604,14 +631,29 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     uint8_t* stage = sEpi + (warp - 2) * 2 * S::EPI_BOX;
     int sbuf = 0;
     int it = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+    int tile, kb0, kb1, unit;
+    for (; pair_work(p, pair, num_pairs, num_tiles, nk, it, tile, kb0, kb1, unit); ++it) {
       const int acc = it & 1;
       const int mb = tile % m_tiles, nb = tile / m_tiles;
       const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-      if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp, &tmC,
-                                       &tmZ, stage, sbuf))
+      if (unit >= 0) {
+        // A K range of a split tile: its fp32 partial sums go to scratch, column-major
+        // [BN][256] per unit so that a warp's 32 rows store 128 contiguous bytes.
+        if (!mbar_wait_cluster(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
+        tc_fence_after();
+        float* part = p.sk_part + static_cast<size_t>(unit) * (2 * kBM) * BN + rank * kBM + quad * 32 + lane;
+#pragma unroll 1
+        for (int c0 = 32 * grp; c0 < BN; c0 += 32 * Epi<RL>::GROUPS) {
+          float v[32];
+          load_cols<32>(t_row + c0, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) part[static_cast<size_t>(c0 + i) * (2 * kBM)] = v[i];
+        }
+      } else if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp,
+                                              &tmC, &tmZ, stage, sbuf)) {
         break;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -632,7 +674,76 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
   }
 }
 
+// --------------------------------------------------------- split-K tail sum
+constexpr int kMaxSplit = 8;  // K ranges per split tile at most
+
+// out = epilogue(sum over s of part[tile's unit s]) for the split tiles of a pair
+// product: the partials are added in unit order (the same order on every run), then
+// bias, activation and residual as in epilogue_tile.  One thread per 8 consecutive
+// columns of one row; a warp covers 32 consecutive rows, so every partial load is a
+// contiguous 128-byte line.
+template <int BN>
+__global__ void __launch_bounds__(256) gemm_split_sum(const GemmParams p) {
+  const int m_tiles = (p.M + 2 * kBM - 1) / (2 * kBM);
+  const int groups = BN / 8;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int r = static_cast<int>(i % (2 * kBM));
+  const long long rest = i / (2 * kBM);
+  const int g = static_cast<int>(rest % groups);
+  const int t = static_cast<int>(rest / groups);  // split tile, 0-based after sk_full
+  const int tile = p.sk_full + t;
+  if (tile >= m_tiles * ((p.N + BN - 1) / BN)) return;
+  const int row = (tile % m_tiles) * 2 * kBM + r;
+  const int col = (tile / m_tiles) * BN + 8 * g;
+  if (row >= p.M || col >= p.N) return;
+  // every partial is loaded before the first add, so that the loads overlap
+  float pv[kMaxSplit][8];
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s) {
+    if (s >= p.sk_split) break;
+    const float* part = p.sk_part + static_cast<size_t>(t * p.sk_split + s) * (2 * kBM) * BN +
+                        static_cast<size_t>(8 * g) * (2 * kBM) + r;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) pv[s][c] = part[c * (2 * kBM)];
+  }
+  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s) {
+    if (s >= p.sk_split) break;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[c] += pv[s][c];
+  }
+  if (p.bias) add_bf16x8(v, __ldg(reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.bias) + col)));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    if (p.act == ACT_GELU_TANH) v[c] = gelu_tanh(v[c]);
+    else if (p.act == ACT_GELU_ERF) v[c] = gelu_erf(v[c]);
+  }
+  if (p.resid)
+    add_bf16x8(v, *reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.resid) + static_cast<size_t>(row) * p.ldr +
+                                                  col));
+  *reinterpret_cast<uint4*>(static_cast<bf16*>(p.out) + static_cast<size_t>(row) * p.ldo + col) = pack_bf16x8(v);
+}
+
 // ------------------------------------------------------------------- launch
+
+// K ranges per tile for the split-K tail of a plain pair product, 1 for none.  Used when
+// the tiles of the last round fill at most half of the pairs and K is long (at least 32
+// steps: below that the tail sum costs about what the split saves, measured on B200 for
+// the 1280-deep output projection), with at least eight K steps per range and an
+// epilogue that the tail sum reproduces.
+int split_factor(const GemmParams& p, int tiles, int pairs, int bn) {
+  if (!p.sk_part || p.pre_out || p.act > ACT_GELU_ERF || p.N % 8) return 1;
+  const int rem = tiles % pairs;
+  if (rem == 0 || 2 * rem > pairs) return 1;
+  const int nk = (p.K + kBK - 1) / kBK;
+  if (nk < 32) return 1;
+  int s = pairs / rem;
+  if (s > nk / 8) s = nk / 8;
+  if (s > kMaxSplit) s = kMaxSplit;
+  if (static_cast<size_t>(rem) * s * 2 * kBM * bn * sizeof(float) > gemm_split_bytes()) return 1;
+  return s > 1 ? s : 1;
+}
 
 template <int BN, class RL>
 cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
@@ -676,7 +787,16 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   const int tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + BN - 1) / BN);
   const int max_pairs = device_sm_count() / 2;
-  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  int pairs = tiles < max_pairs ? tiles : max_pairs;
+  GemmParams q = p;
+  const int split = split_factor(p, tiles, max_pairs, BN);
+  if (split > 1) {
+    q.sk_full = tiles - tiles % max_pairs;
+    q.sk_split = split;
+    pairs = max_pairs;
+  } else {
+    q.sk_part = nullptr;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(Epi<RL>::THREADS, 1, 1);
@@ -689,12 +809,18 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, tc, tz, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, tc, tz, q);
   if (e != cudaSuccess) return e;
+  if (split > 1) {
+    const long long threads = static_cast<long long>(tiles - q.sk_full) * (BN / 8) * (2 * kBM);
+    gemm_split_sum<BN><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(q);
+  }
   return cudaGetLastError();
 }
 
 }  // namespace
+
+size_t gemm_split_bytes() { return static_cast<size_t>(device_sm_count() / 2) * 2 * kBM * 256 * sizeof(float); }
 
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return cudaSuccess;
@@ -708,12 +834,14 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) 
     return cudaErrorNotSupported;
   }
   if (pair) {
-    // 224-wide tiles when they fill the last wave of CTA pairs clearly better than
-    // 256-wide ones (measured on B200 for short-K, 1280-wide outputs such as the
-    // attention output projection of 8 images at 448x448).
+    const int pairs = device_sm_count() / 2;
+    const int mt = (p.M + 2 * kBM - 1) / (2 * kBM);
+    // 256-wide tiles whose last round a split-K tail fills
+    if (split_factor(p, mt * ((p.N + 255) / 256), pairs, 256) > 1) return launch_pair<256, Rope0>(p, stream);
+    // otherwise 224-wide tiles when they fill the last round of CTA pairs clearly better
+    // than 256-wide ones (measured on B200 for short-K, 1280-wide outputs such as the
+    // attention output projection of 8 images at 448x448)
     if (p.K <= 2048) {
-      const int pairs = device_sm_count() / 2;
-      const int mt = (p.M + 2 * kBM - 1) / (2 * kBM);
       auto eff = [&](int bn) {
         const int nt = (p.N + bn - 1) / bn;
         const long tiles = static_cast<long>(mt) * nt;

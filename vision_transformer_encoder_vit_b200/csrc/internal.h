@@ -98,7 +98,18 @@ struct GemmParams {
   // v^T of image b is [heads, head_dim, ld_vt[b]] at vt_off[b].
   int varlen;
   VarlenTable vl;
+  // Split-K tail of plain products on CTA pairs (sk_part null: off).  The caller gives
+  // sk_part, gemm_split_bytes() bytes of fp32 scratch; launch_gemm sets the rest when
+  // the output tiles leave the last round of the grid mostly idle: the first sk_full
+  // tiles run whole, each remaining tile's K steps are cut into sk_split ranges, one per
+  // idle CTA pair, and a second kernel adds their fp32 partial sums in a fixed order and
+  // applies the epilogue.
+  float* sk_part;
+  int sk_full, sk_split;
 };
+
+// Bytes of split-K scratch a product may use (one 256 x 256 fp32 tile per CTA pair).
+size_t gemm_split_bytes();
 
 // Returns a CUDA error code (cudaSuccess on success); host-side shape checks are the
 // caller's job.

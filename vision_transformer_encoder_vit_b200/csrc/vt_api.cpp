@@ -134,6 +134,12 @@ vt_status run_gemm(GemmParams p, cudaStream_t st) {
   return VT_OK;
 }
 
+// The same product with a split-K tail allowed, on `scratch` (gemm_split_bytes()).
+GemmParams split_k(GemmParams p, char* scratch) {
+  p.sk_part = reinterpret_cast<float*>(scratch);
+  return p;
+}
+
 GemmParams gemm_params(const void* A, int lda, const void* W, int ldw, const void* bias, const void* resid,
                        int ldr, void* out, int ldo, int M, int N, int K, int act) {
   GemmParams p;
@@ -232,7 +238,7 @@ bool qkv_layout_supported(const vt_config& c) {
 
 struct Plan {
   int N, M, Mm, ld_vt;
-  size_t x, xn, q, k, vt, o, hmid, unfold, y1, y2, z1, total;
+  size_t x, sk, xn, q, k, vt, o, hmid, unfold, y1, y2, z1, total;
 };
 
 // Workspace layout for M packed tokens whose transposed v blocks take vt_elems elements.
@@ -247,6 +253,8 @@ Plan make_plan_core(const vt_config& c, int M_, size_t vt_elems) {
   size_t off = 0;
   p.x = off;
   off += align256(M * d * 2);
+  p.sk = off;  // split-K scratch of the linear layers (fixed size)
+  off += align256(gemm_split_bytes());
   const size_t base = off;
   // tower phase
   size_t o2 = base;
@@ -309,10 +317,12 @@ vt_status check_still(int t, const char* entry) {
 }
 
 // The patch-embedding product: patch vectors U [M, K0] -> tokens x [M, hidden].
-vt_status run_patch_embed(vt_handle* h, const void* U, void* x, const Plan& pl, cudaStream_t st) {
+vt_status run_patch_embed(vt_handle* h, const void* U, void* x, char* ws, const Plan& pl, cudaStream_t st) {
   const vt_config& c = h->cfg;
   const int K0 = 3 * c.temporal_patch * c.patch * c.patch;
-  return run_gemm(gemm_params(U, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0, ACT_NONE), st);
+  return run_gemm(
+      split_k(gemm_params(U, K0, h->pe_w, K0, h->pe_b, nullptr, 0, x, c.hidden, pl.M, c.hidden, K0, ACT_NONE), ws + pl.sk),
+      st);
 }
 
 // One pre-LN layer over the M tokens at x_in (written to x, which may equal x_in).  With
@@ -376,12 +386,16 @@ vt_status run_layer(vt_handle* h, int i, const void* x_in, void* x, int B, int g
     }
     if ((s = run_attention(a, st))) return s;
   }
-  if ((s = run_gemm(gemm_params(ws + pl.o, d, L.o_w, d, L.o_b, x_in, d, x, d, M, d, d, ACT_NONE), st))) return s;
+  if ((s = run_gemm(split_k(gemm_params(ws + pl.o, d, L.o_w, d, L.o_b, x_in, d, x, d, M, d, d, ACT_NONE), ws + pl.sk),
+                    st)))
+    return s;
   if ((s = run_layernorm(x, L.ln2_w, L.ln2_b, xn, M, d, c.ln_eps, st))) return s;
   const int act = c.gelu_tanh ? ACT_GELU_TANH : ACT_GELU_ERF;
   if ((s = run_gemm(gemm_params(xn, d, L.fc1_w, d, L.fc1_b, nullptr, 0, ws + pl.hmid, c.mlp, M, c.mlp, d, act), st)))
     return s;
-  return run_gemm(gemm_params(ws + pl.hmid, c.mlp, L.fc2_w, c.mlp, L.fc2_b, x, d, x, d, M, d, c.mlp, ACT_NONE), st);
+  return run_gemm(
+      split_k(gemm_params(ws + pl.hmid, c.mlp, L.fc2_w, c.mlp, L.fc2_b, x, d, x, d, M, d, c.mlp, ACT_NONE), ws + pl.sk),
+      st);
 }
 
 // Projector on block-ordered tokens x [M, d] -> out [M/4, proj_out].
@@ -389,18 +403,16 @@ vt_status run_projector(vt_handle* h, const void* x, void* out, char* ws, const 
   const vt_config& c = h->cfg;
   const int d = c.hidden, P = c.proj_hidden, M = pl.M, Mm = pl.Mm;
   const int act = c.proj_gelu_tanh ? ACT_GELU_TANH : ACT_GELU_ERF;
+  auto gemm = [&](const void* A, int lda, const void* W, const void* b, void* o, int ldo, int rows, int n, int k,
+                  int a) { return run_gemm(split_k(gemm_params(A, lda, W, lda, b, nullptr, 0, o, ldo, rows, n, k, a),
+                                                   ws + pl.sk),
+                                           st); };
   vt_status s;
-  if ((s = run_gemm(gemm_params(x, d, h->pa1_w, d, h->pa1_b, nullptr, 0, ws + pl.y1, P, M, P, d, act), st))) return s;
-  if ((s = run_gemm(gemm_params(ws + pl.y1, P, h->pa2_w, P, h->pa2_b, nullptr, 0, ws + pl.y2, P, M, P, P, ACT_NONE),
-                    st)))
-    return s;
+  if ((s = gemm(x, d, h->pa1_w, h->pa1_b, ws + pl.y1, P, M, P, d, act))) return s;
+  if ((s = gemm(ws + pl.y1, P, h->pa2_w, h->pa2_b, ws + pl.y2, P, M, P, P, ACT_NONE))) return s;
   // Four consecutive block-ordered rows of y2 are one merged token: a [M/4, 4P] view.
-  if ((s = run_gemm(gemm_params(ws + pl.y2, 4 * P, h->pb1_w, 4 * P, h->pb1_b, nullptr, 0, ws + pl.z1, P, Mm, P, 4 * P,
-                                act),
-                    st)))
-    return s;
-  return run_gemm(
-      gemm_params(ws + pl.z1, P, h->pb2_w, P, h->pb2_b, nullptr, 0, out, c.proj_out, Mm, c.proj_out, P, ACT_NONE), st);
+  if ((s = gemm(ws + pl.y2, 4 * P, h->pb1_w, h->pb1_b, ws + pl.z1, P, Mm, P, 4 * P, act))) return s;
+  return gemm(ws + pl.z1, P, h->pb2_w, h->pb2_b, out, c.proj_out, Mm, c.proj_out, P, ACT_NONE);
 }
 
 vt_status check_loaded(const vt_handle* h) {
@@ -582,7 +594,7 @@ static vt_status forward_embedded(vt_handle* h, int B, int t, int gh, int gw, vo
   const vt_config& c = h->cfg;
   void* x = w + pl.x;
   vt_status s;
-  if ((s = run_patch_embed(h, w + pl.unfold, x, pl, st))) return s;
+  if ((s = run_patch_embed(h, w + pl.unfold, x, w, pl, st))) return s;
   for (int i = 0; i < c.layers; ++i)
     if ((s = run_layer(h, i, x, x, B, t, gh, gw, ORDER_BLOCK, w, pl, st))) return s;
   if (tower_out) {
@@ -842,7 +854,7 @@ vt_status vt_forward_varlen(vt_handle* h, const float* pixels, const int32_t* gr
     cudaError_t e = launch_patch_unfold_varlen(pixels, w + pl.unfold, vl, c.patch, c.temporal_patch, st);
     if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
   }
-  if ((s = run_patch_embed(h, w + pl.unfold, x, pl, st))) return s;
+  if ((s = run_patch_embed(h, w + pl.unfold, x, w, pl, st))) return s;
   // The QKV epilogue writes only each image's own v^T columns; the rest of the common
   // stride must read as zeros in the attention's P.V (P is zero there).
   {
@@ -951,7 +963,7 @@ vt_status vt_patch_embed(vt_handle* h, const float* pixels, const int32_t* grid_
   cudaError_t e = launch_patch_unfold(pixels, w + pl.unfold, B, gh * c.patch, gw * c.patch, c.patch, c.temporal_patch,
                                       ORDER_RASTER, st);
   if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
-  return run_patch_embed(h, w + pl.unfold, x_out, pl, st);
+  return run_patch_embed(h, w + pl.unfold, x_out, w, pl, st);
 }
 
 vt_status vt_merge_project(vt_handle* h, const void* tower, const int32_t* grid_thw, int B, void* out, void* ws,
@@ -1237,7 +1249,7 @@ SavedLayout saved_layout(const vt_config& c, int B, int N) {
 // the [M, 3d] qkv gradient and the per-query delta.
 struct BwdPlan {
   int N, M, ld, lds;
-  size_t dx, xn, hmid, dO, dqkv, delta, total;
+  size_t dx, xn, hmid, dO, dqkv, delta, sk, total;
 };
 
 BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
@@ -1261,6 +1273,7 @@ BwdPlan make_bwd_plan(const vt_config& c, int B, int N) {
   p.dO = take(M * d * 2);
   p.dqkv = take(M * 3 * d * 2);
   p.delta = take(stats * 4);
+  p.sk = take(gemm_split_bytes());
   p.total = off;
   return p;
 }
@@ -1330,7 +1343,9 @@ vt_status run_layer_saving(vt_handle* h, int i, char* sv, const SavedLayout& sl,
     a.ld_lse = sl.lds;
     if ((s = run_attention(a, st))) return s;
   }
-  if ((s = run_gemm(gemm_params(sv + sl.a, d, L.o_w, d, L.o_b, sv + sl.x, d, sv + sl.x1, d, M, d, d, ACT_NONE), st)))
+  if ((s = run_gemm(
+           split_k(gemm_params(sv + sl.a, d, L.o_w, d, L.o_b, sv + sl.x, d, sv + sl.x1, d, M, d, d, ACT_NONE), w + pl.sk),
+           st)))
     return s;
   if ((s = run_layernorm(sv + sl.x1, L.ln2_w, L.ln2_b, xn, M, d, c.ln_eps, st))) return s;
   {
@@ -1339,7 +1354,8 @@ vt_status run_layer_saving(vt_handle* h, int i, char* sv, const SavedLayout& sl,
     p.pre_out = sv + sl.z;  // the pre-activation, for the GELU derivative
     if ((s = run_gemm(p, st))) return s;
   }
-  return run_gemm(gemm_params(hmid, m, L.fc2_w, m, L.fc2_b, sv + sl.x1, d, x_out, d, M, d, m, ACT_NONE), st);
+  return run_gemm(
+      split_k(gemm_params(hmid, m, L.fc2_w, m, L.fc2_b, sv + sl.x1, d, x_out, d, M, d, m, ACT_NONE), w + pl.sk), st);
 }
 
 // One layer backward on block-ordered tokens: dx (in: d loss / d layer output; out:
@@ -1357,10 +1373,14 @@ vt_status run_layer_backward(vt_handle* h, int i, const char* sv, const SavedLay
   // ---- MLP branch: dz = (dx W2) * gelu'(z), dg = dz W1, dx += LN2^T(dg)
   const int dact = c.gelu_tanh ? ACT_DGELU_TANH : ACT_DGELU_ERF;
   if ((s = run_gemm(gemm_params(dx, d, T.fc2_t, d, nullptr, sv + sl.z, m, hmid, m, M, m, d, dact), st))) return s;
-  if ((s = run_gemm(gemm_params(hmid, m, T.fc1_t, m, nullptr, nullptr, 0, xn, d, M, d, m, ACT_NONE), st))) return s;
+  if ((s = run_gemm(split_k(gemm_params(hmid, m, T.fc1_t, m, nullptr, nullptr, 0, xn, d, M, d, m, ACT_NONE), w + bp.sk),
+                    st)))
+    return s;
   if ((s = run_layernorm_backward(sv + sl.x1, L.ln2_w, xn, dx, dx, M, d, c.ln_eps, st))) return s;
   // ---- attention branch: dO = dx Wo, attention backward, dh = dqkv Wqkv, dx += LN1^T(dh)
-  if ((s = run_gemm(gemm_params(dx, d, T.o_t, d, nullptr, nullptr, 0, w + bp.dO, d, M, d, d, ACT_NONE), st))) return s;
+  if ((s = run_gemm(
+           split_k(gemm_params(dx, d, T.o_t, d, nullptr, nullptr, 0, w + bp.dO, d, M, d, d, ACT_NONE), w + bp.sk), st)))
+    return s;
   {
     ProfScope ps(CLS_BWD_MISC, 0, 4.0 * M * d + 4.0 * M * H, st);
     cudaError_t e = launch_attention_delta(w + bp.dO, sv + sl.a, reinterpret_cast<float*>(w + bp.delta), B, N, H, D,
@@ -1392,8 +1412,9 @@ vt_status run_layer_backward(vt_handle* h, int i, const char* sv, const SavedLay
     a.order = ORDER_BLOCK;
     if ((s = run_attention_backward(a, st))) return s;
   }
-  if ((s = run_gemm(gemm_params(w + bp.dqkv, 3 * d, T.qkv_t, 3 * d, nullptr, nullptr, 0, xn, d, M, d, 3 * d,
-                                ACT_NONE),
+  if ((s = run_gemm(split_k(gemm_params(w + bp.dqkv, 3 * d, T.qkv_t, 3 * d, nullptr, nullptr, 0, xn, d, M, d, 3 * d,
+                                        ACT_NONE),
+                            w + bp.sk),
                     st)))
     return s;
   return run_layernorm_backward(sv + sl.x, L.ln1_w, xn, dx, dx, M, d, c.ln_eps, st);
@@ -1495,7 +1516,7 @@ vt_status vt_forward_saved(vt_handle* h, const float* pixels, const int32_t* gri
     if (e != cudaSuccess) return cuda_fail(e, "patch unfold launch");
   }
   void* x0 = c.layers > 0 ? static_cast<void*>(block(0) + sl.x) : static_cast<void*>(w + pl.x);
-  if ((s = run_patch_embed(h, w + pl.unfold, x0, pl, st))) return s;
+  if ((s = run_patch_embed(h, w + pl.unfold, x0, w, pl, st))) return s;
   for (int i = 0; i < c.layers; ++i) {
     void* out = i + 1 < c.layers ? static_cast<void*>(block(i + 1) + sl.x) : static_cast<void*>(w + pl.x);
     if ((s = run_layer_saving(h, i, block(i), sl, out, B, gh, gw, w, pl, st))) return s;
