@@ -409,7 +409,8 @@ VT_API const char* vt_last_error(void);
  * vt_profile_end on one stream, measured with CUDA events around each launch.
  * Classes: 0 gemm, 1 attention, 2 layernorm, 3 patch unfold, 4 reorder, 5 attention
  * preparation.  vt_profile_read synchronises and returns, per class, the summed
- * milliseconds, launch count and algorithmic FLOPs (GEMM: 2MNK; attention: 4 N^2 D
+ * milliseconds, kernel launch count (a linear layer with a split-K tail launches two
+ * kernels) and algorithmic FLOPs (GEMM: 2MNK; attention: 4 N^2 D
  * per head and image) and bytes (memory-bound classes). */
 VT_API vt_status vt_profile_begin(void* stream);
 VT_API vt_status vt_profile_end(void* stream);

@@ -638,17 +638,19 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
       if (unit >= 0) {
-        // A K range of a split tile: its fp32 partial sums go to scratch, column-major
-        // [BN][256] per unit so that a warp's 32 rows store 128 contiguous bytes.
+        // A K range of a split tile: its fp32 partial sums go to scratch, row-major
+        // [256][BN] per unit (each thread writes its row's 128 contiguous bytes per chunk),
+        // so that the sum kernel reads and writes whole rows.
         if (!mbar_wait_cluster(&tfull[acc], (it >> 1) & 1, abort_flag, &g_gemm_err)) break;
         tc_fence_after();
-        float* part = p.sk_part + static_cast<size_t>(unit) * (2 * kBM) * BN + rank * kBM + quad * 32 + lane;
+        float* part = p.sk_part + (static_cast<size_t>(unit) * (2 * kBM) + rank * kBM + quad * 32 + lane) * BN;
 #pragma unroll 1
         for (int c0 = 32 * grp; c0 < BN; c0 += 32 * Epi<RL>::GROUPS) {
           float v[32];
           load_cols<32>(t_row + c0, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) part[static_cast<size_t>(c0 + i) * (2 * kBM)] = v[i];
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(part + c0)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
       } else if (!epilogue_tile<BN, RL, true>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp,
                                               &tmC, &tmZ, stage, sbuf)) {
@@ -679,50 +681,57 @@ constexpr int kMaxSplit = 8;  // K ranges per split tile at most
 
 // out = epilogue(sum over s of part[tile's unit s]) for the split tiles of a pair
 // product: the partials are added in unit order (the same order on every run), then
-// bias, activation and residual as in epilogue_tile.  One thread per 8 consecutive
-// columns of one row; a warp covers 32 consecutive rows, so every partial load is a
-// contiguous 128-byte line.
+// bias, activation and residual as in epilogue_tile.  One thread per 4 consecutive
+// columns of one row; a warp covers 128 contiguous columns, so its partial loads are
+// 512 contiguous bytes and its residual loads and output stores 256.
 template <int BN>
 __global__ void __launch_bounds__(256) gemm_split_sum(const GemmParams p) {
   const int m_tiles = (p.M + 2 * kBM - 1) / (2 * kBM);
-  const int groups = BN / 8;
+  constexpr int QUADS = BN / 4;  // four columns per thread: a warp covers 128 contiguous columns
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int r = static_cast<int>(i % (2 * kBM));
-  const long long rest = i / (2 * kBM);
-  const int g = static_cast<int>(rest % groups);
-  const int t = static_cast<int>(rest / groups);  // split tile, 0-based after sk_full
+  const int g = static_cast<int>(i % QUADS);
+  const long long rest = i / QUADS;
+  const int r = static_cast<int>(rest % (2 * kBM));
+  const int t = static_cast<int>(rest / (2 * kBM));  // split tile, 0-based after sk_full
   const int tile = p.sk_full + t;
   if (tile >= m_tiles * ((p.N + BN - 1) / BN)) return;
   const int row = (tile % m_tiles) * 2 * kBM + r;
-  const int col = (tile / m_tiles) * BN + 8 * g;
+  const int col = (tile / m_tiles) * BN + 4 * g;
   if (row >= p.M || col >= p.N) return;
   // every partial is loaded before the first add, so that the loads overlap
-  float pv[kMaxSplit][8];
+  float4 pv[kMaxSplit];
 #pragma unroll
   for (int s = 0; s < kMaxSplit; ++s) {
     if (s >= p.sk_split) break;
-    const float* part = p.sk_part + static_cast<size_t>(t * p.sk_split + s) * (2 * kBM) * BN +
-                        static_cast<size_t>(8 * g) * (2 * kBM) + r;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) pv[s][c] = part[c * (2 * kBM)];
+    pv[s] = *reinterpret_cast<const float4*>(p.sk_part + (static_cast<size_t>(t * p.sk_split + s) * (2 * kBM) + r) * BN +
+                                             4 * g);
   }
-  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int s = 0; s < kMaxSplit; ++s) {
     if (s >= p.sk_split) break;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) v[c] += pv[s][c];
+    v[0] += pv[s].x;
+    v[1] += pv[s].y;
+    v[2] += pv[s].z;
+    v[3] += pv[s].w;
   }
-  if (p.bias) add_bf16x8(v, __ldg(reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.bias) + col)));
+  auto add4 = [&](uint2 u) {
+    const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+    v[0] += a.x;
+    v[1] += a.y;
+    v[2] += b.x;
+    v[3] += b.y;
+  };
+  if (p.bias) add4(__ldg(reinterpret_cast<const uint2*>(static_cast<const bf16*>(p.bias) + col)));
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < 4; ++c) {
     if (p.act == ACT_GELU_TANH) v[c] = gelu_tanh(v[c]);
     else if (p.act == ACT_GELU_ERF) v[c] = gelu_erf(v[c]);
   }
   if (p.resid)
-    add_bf16x8(v, *reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.resid) + static_cast<size_t>(row) * p.ldr +
-                                                  col));
-  *reinterpret_cast<uint4*>(static_cast<bf16*>(p.out) + static_cast<size_t>(row) * p.ldo + col) = pack_bf16x8(v);
+    add4(*reinterpret_cast<const uint2*>(static_cast<const bf16*>(p.resid) + static_cast<size_t>(row) * p.ldr + col));
+  *reinterpret_cast<uint2*>(static_cast<bf16*>(p.out) + static_cast<size_t>(row) * p.ldo + col) =
+      make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
 
 // ------------------------------------------------------------------- launch
@@ -769,7 +778,7 @@ cudaError_t launch_one(const GemmParams& p, cudaStream_t stream) {
 }
 
 template <int BN, class RL>
-cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
+cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream, int* kernels = nullptr) {
   using S = GemmShape<BN, true>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -811,8 +820,9 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_bf16_tcgen05_pair<BN, RL>, ta, tb, tc, tz, q);
   if (e != cudaSuccess) return e;
+  if (kernels) *kernels = split > 1 ? 2 : 1;
   if (split > 1) {
-    const long long threads = static_cast<long long>(tiles - q.sk_full) * (BN / 8) * (2 * kBM);
+    const long long threads = static_cast<long long>(tiles - q.sk_full) * (BN / 4) * (2 * kBM);
     gemm_split_sum<BN><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(q);
   }
   return cudaGetLastError();
@@ -822,7 +832,8 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream) {
 
 size_t gemm_split_bytes() { return static_cast<size_t>(device_sm_count() / 2) * 2 * kBM * 256 * sizeof(float); }
 
-cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) {
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode, int* kernels) {
+  if (kernels) *kernels = 1;
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return cudaSuccess;
   // Pairs of CTAs (256-row tiles) once there are enough rows to keep them busy.
   const bool pair = p.M >= 1024;
@@ -837,7 +848,7 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) 
     const int pairs = device_sm_count() / 2;
     const int mt = (p.M + 2 * kBM - 1) / (2 * kBM);
     // 256-wide tiles whose last round a split-K tail fills
-    if (split_factor(p, mt * ((p.N + 255) / 256), pairs, 256) > 1) return launch_pair<256, Rope0>(p, stream);
+    if (split_factor(p, mt * ((p.N + 255) / 256), pairs, 256) > 1) return launch_pair<256, Rope0>(p, stream, kernels);
     // otherwise 224-wide tiles when they fill the last round of CTA pairs clearly better
     // than 256-wide ones (measured on B200 for short-K, 1280-wide outputs such as the
     // attention output projection of 8 images at 448x448)
@@ -848,9 +859,9 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode) 
         const long waves = (tiles + pairs - 1) / pairs;
         return (static_cast<double>(tiles) / (waves * pairs)) * (static_cast<double>(p.N) / (nt * bn));
       };
-      if (eff(224) * 0.93 > eff(256)) return launch_pair<224, Rope0>(p, stream);
+      if (eff(224) * 0.93 > eff(256)) return launch_pair<224, Rope0>(p, stream, kernels);
     }
-    return launch_pair<256, Rope0>(p, stream);
+    return launch_pair<256, Rope0>(p, stream, kernels);
   }
   // Wide tiles when they still fill the SMs; narrower ones for small problems.
   const int sms = device_sm_count();

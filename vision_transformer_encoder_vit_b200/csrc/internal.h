@@ -113,7 +113,8 @@ size_t gemm_split_bytes();
 
 // Returns a CUDA error code (cudaSuccess on success); host-side shape checks are the
 // caller's job.
-cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode);
+// *kernels (if given) receives the number of kernels launched (2 with a split-K tail sum).
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode, int* kernels = nullptr);
 unsigned int gemm_read_clear_error(cudaStream_t stream);
 
 // ------------------------------------------------------------- attention

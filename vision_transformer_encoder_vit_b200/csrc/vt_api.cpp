@@ -59,6 +59,7 @@ struct ProfRec {
   int cls;
   cudaEvent_t a, b;
   double flops, bytes;
+  int kernels;  // kernels the bracketed call launched
 };
 
 struct DoneRec {
@@ -105,6 +106,7 @@ struct ProfScope {
   double flops, bytes;
   cudaStream_t st;
   cudaEvent_t a = nullptr;
+  int kernels = 1;
   ProfScope(int c, double f, double b, cudaStream_t s) : cls(c), flops(f), bytes(b), st(s) {
     if (g_log)
       std::fprintf(stderr, "vt: launch %s flops=%.6g bytes=%.6g stream=%p\n", kClassNames[c], f, b,
@@ -120,7 +122,7 @@ struct ProfScope {
       std::lock_guard<std::mutex> l(g_prof.mu);
       cudaEvent_t b = g_prof.get();
       cudaEventRecord(b, st);
-      g_prof.recs.push_back({cls, a, b, flops, bytes});
+      g_prof.recs.push_back({cls, a, b, flops, bytes, kernels});
     }
   }
 };
@@ -129,7 +131,7 @@ struct ProfScope {
 
 vt_status run_gemm(GemmParams p, cudaStream_t st) {
   ProfScope ps(CLS_GEMM, 2.0 * p.M * static_cast<double>(p.N) * p.K, 0, st);
-  cudaError_t e = launch_gemm(p, st, 0);
+  cudaError_t e = launch_gemm(p, st, 0, &ps.kernels);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return VT_OK;
 }
@@ -1154,7 +1156,7 @@ vt_status resolve_profile() {
     g_prof.ms[r.cls] += t;
     g_prof.flops[r.cls] += r.flops;
     g_prof.bytes[r.cls] += r.bytes;
-    g_prof.n[r.cls] += 1;
+    g_prof.n[r.cls] += r.kernels;
     g_prof.done.push_back({r.cls, static_cast<double>(t), r.flops, r.bytes});
     g_prof.pool.push_back(r.a);
     g_prof.pool.push_back(r.b);
