@@ -363,6 +363,16 @@ VT_API vt_status vt_attention_static_max_bytes(size_t* out);
  * Architecture table). */
 VT_API vt_status vt_linear(const void* A, const void* W, const void* bias, const void* resid, void* out, int M, int N,
                     int K, int act, void* stream);
+/* The same product with device scratch ws (ws_bytes >= vt_linear_workspace_bytes(),
+ * 16-byte aligned) for a split-K tail: when M >= 1024 and the output tiles leave most
+ * pairs of SMs idle in the last round of the grid, with K at least 2048, the K steps of
+ * the remaining tiles are shared out and summed in fp32 by a second kernel in a fixed
+ * order (the result does not depend on timing).  The forward uses this form for every
+ * linear layer.  Library-defined; ws NULL or too small: runs as vt_linear. */
+VT_API vt_status vt_linear_ws(const void* A, const void* W, const void* bias, const void* resid, void* out, int M,
+                              int N, int K, int act, void* ws, size_t ws_bytes, void* stream);
+/* Bytes of the split-K scratch (one 256 x 256 fp32 tile per pair of SMs).  Host only. */
+VT_API vt_status vt_linear_workspace_bytes(size_t* out);
 
 /* LayerNorm over rows: y = (x - mean) / sqrt(var + eps) * gamma + beta; x, y device
  * bf16 [rows, cols]; statistics in fp32 (CLIP-style pre-LN block). */

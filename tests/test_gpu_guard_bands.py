@@ -178,6 +178,23 @@ def test_attention_guard_bands(B, H, N, D):
         unchanged(b, a, f"vt_attention {shape}: {what}")
 
 
+def test_linear_split_k_guard_bands():
+    # ragged split-K tail: 5 x 4 tiles of 256 on the pairs, K = 4104 (a partial K step)
+    M, N, K = 1100, 1000, 4104
+    A, W = S.make_matrix((M, K), 80), S.make_matrix((N, K), 81, 0.01)
+    bias, resid = S.make_matrix((N,), 82, 0.1), S.make_matrix((M, N), 83)
+    ab, wb, bb, rb = banded_from(A), banded_from(W), banded_from(bias), banded_from(resid)
+    ws = Banded(V.vt_linear_workspace_bytes())
+    out = Banded(M * N * 2)
+    V.vt_linear_ws(ab.typed(torch.bfloat16, M, K), wb.typed(torch.bfloat16, N, K), bb.typed(torch.bfloat16, N),
+                   rb.typed(torch.bfloat16, M, N), out.typed(torch.bfloat16, M, N), M, N, K, 0, ws.body, ws.nbytes)
+    V.vt_check()
+    ws.check("vt_linear_ws: split-K scratch")
+    out.check("vt_linear_ws: output")
+    for b, a, what in ((ab, A, "A"), (wb, W, "W"), (bb, bias, "bias"), (rb, resid, "resid")):
+        unchanged(b, a, f"vt_linear_ws: {what}")
+
+
 def test_backward_guard_bands():
     tw, cfg = _tower("tiny")
     V.vt_enable_backward(tw.h)

@@ -59,6 +59,66 @@ def test_linear_parity(M, N, K, use_bias, use_resid, act):
     assert_close(host_f64(out), ref, what=f"linear {M}x{N}x{K}")
 
 
+# Shapes whose last round of CTA-pair tiles leaves most pairs idle with K >= 2048: the
+# product shares out the K steps of those tiles and a second kernel sums the fp32
+# partials (vt_linear_ws).  Ragged M, N and K (a partial K step) included.
+SPLIT_CASES = [
+    # M, N, K, bias, resid, act
+    (1100, 1000, 4104, True, True, 0),
+    (8192, 1280, 5120, True, True, 0),    # fc2 at 448 x 448 x 8
+    (2048, 640, 2048, True, False, 1),    # GELU (tanh)
+    (1024, 256, 8192, False, True, 2),    # GELU (erf), one column of tiles, 8 ranges
+]
+
+
+def _expected_split(M, N, K, sms):
+    """K ranges per tile the library picks for 256-wide pair tiles (1: no split)."""
+    pairs, tiles = sms // 2, -(-M // 256) * -(-N // 256)
+    rem, nk = tiles % pairs, -(-K // 64)
+    if M < 1024 or rem == 0 or 2 * rem > pairs or nk < 32:
+        return 1
+    return max(1, min(pairs // rem, nk // 8, 8))
+
+
+@pytest.mark.parametrize("M,N,K,use_bias,use_resid,act", SPLIT_CASES)
+def test_linear_split_k_tail(M, N, K, use_bias, use_resid, act):
+    seed = M * 5 + N * 11 + K
+    A = S.make_matrix((M, K), seed)
+    W = S.make_matrix((N, K), seed + 1, scale=0.02 * 50 / math.sqrt(K))
+    bias = S.make_matrix((N,), seed + 2, 0.1) if use_bias else None
+    resid = S.make_matrix((M, N), seed + 3) if use_resid else None
+    dA, dW = dev_bf16(A), dev_bf16(W)
+    dB = dev_bf16(bias) if use_bias else None
+    dR = dev_bf16(resid) if use_resid else None
+    ws_bytes = V.vt_linear_workspace_bytes()
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    out = empty_bf16(M, N)
+    V.vt_profile_begin()
+    V.vt_linear_ws(dA, dW, dB, dR, out, M, N, K, act, ws, ws_bytes)
+    V.vt_profile_end()
+    prof = V.vt_profile_read()
+    V.vt_check()
+    split = _expected_split(M, N, K, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert split > 1, "the case should take the split-K path"
+    assert prof["gemm"]["launches"] == 2  # the product and the tail sum
+    # rows checked: all of them for small M, else a sample that includes the last tile
+    rows = np.arange(M) if M <= 2048 else np.unique(np.concatenate(
+        [np.random.default_rng(seed).choice(M, 256, replace=False), np.arange(M - 64, M)]))
+    ref = S.bf16_to_f64(A)[rows] @ S.bf16_to_f64(W).T
+    if use_bias:
+        ref = ref + S.bf16_to_f64(bias)
+    if act:
+        ref = R.gelu(ref, tanh_form=(act == 1))
+    if use_resid:
+        ref = ref + S.bf16_to_f64(resid)[rows]
+    got = host_f64(out)[rows]
+    assert_close(got, ref, what=f"split-K linear {M}x{N}x{K}")
+    # the same call again gives the same bits (fixed summation order)
+    out2 = empty_bf16(M, N)
+    V.vt_linear_ws(dA, dW, dB, dR, out2, M, N, K, act, ws, ws_bytes)
+    assert torch.equal(out, out2)
+
+
 def test_linear_residual_in_place():
     M, N, K = 384, 512, 256
     A, W = S.make_matrix((M, K), 1), S.make_matrix((N, K), 2, 0.05)

@@ -1052,6 +1052,26 @@ vt_status vt_linear(const void* A, const void* W, const void* bias, const void* 
   return run_gemm(gemm_params(A, K, W, K, bias, resid, N, out, N, M, N, K, act), static_cast<cudaStream_t>(stream));
 }
 
+vt_status vt_linear_ws(const void* A, const void* W, const void* bias, const void* resid, void* out, int M, int N,
+                       int K, int act, void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < gemm_split_bytes()) return vt_linear(A, W, bias, resid, out, M, N, K, act, stream);
+  if (!aligned16(ws)) return fail(VT_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+  if (!A || !W || !out) return fail(VT_ERR_INVALID_ARG, "A, W and out must not be NULL");
+  if (M <= 0 || N <= 0 || K <= 0) return fail(VT_ERR_INVALID_ARG, "M, N, K must be positive");
+  if (N % 8 || K % 8) return fail(VT_ERR_INVALID_ARG, "N and K must be multiples of 8");
+  if (act < 0 || act > 2) return fail(VT_ERR_INVALID_ARG, "act must be 0, 1 or 2");
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out) || (bias && !aligned16(bias)) || (resid && !aligned16(resid)))
+    return fail(VT_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  return run_gemm(split_k(gemm_params(A, K, W, K, bias, resid, N, out, N, M, N, K, act), static_cast<char*>(ws)),
+                  static_cast<cudaStream_t>(stream));
+}
+
+vt_status vt_linear_workspace_bytes(size_t* out) {
+  if (!out) return fail(VT_ERR_INVALID_ARG, "out is NULL");
+  *out = gemm_split_bytes();
+  return VT_OK;
+}
+
 vt_status vt_layernorm(const void* x, const void* gamma, const void* beta, void* y, int rows, int cols, float eps,
                        void* stream) {
   if (!x || !gamma || !beta || !y) return fail(VT_ERR_INVALID_ARG, "NULL operand");

@@ -89,6 +89,8 @@ _SIGS = {
     "vt_attention_static": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i32p, _f, _f, _vp]),
     "vt_attention_static_max_bytes": ([ctypes.POINTER(_sz)]),
     "vt_linear": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "vt_linear_ws": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "vt_linear_workspace_bytes": ([ctypes.POINTER(_sz)]),
     "vt_layernorm": ([_vp, _vp, _vp, _vp, _i, _i, _f, _vp]),
     "vt_patch_unfold": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "vt_index_maps": ([_i32p, _i32p, _i32p, _i32p]),
@@ -365,6 +367,17 @@ def vt_attention_prepared(q, k, vt, ld_vt, o, B, H, N, D, scale, stream=None) ->
 def vt_linear(A, W, bias, resid, out, M, N, K, act=0, stream=None) -> None:
     _check(lib.vt_linear(_ptr(A), _ptr(W), _ptr(bias), _ptr(resid), _ptr(out), M, N, K, act, _stream(stream)),
            "vt_linear")
+
+
+def vt_linear_ws(A, W, bias, resid, out, M, N, K, act, ws, ws_bytes, stream=None) -> None:
+    _check(lib.vt_linear_ws(_ptr(A), _ptr(W), _ptr(bias), _ptr(resid), _ptr(out), M, N, K, act, _ptr(ws), ws_bytes,
+                            _stream(stream)), "vt_linear_ws")
+
+
+def vt_linear_workspace_bytes() -> int:
+    n = _sz()
+    _check(lib.vt_linear_workspace_bytes(ctypes.byref(n)), "vt_linear_workspace_bytes")
+    return n.value
 
 
 def vt_layernorm(x, gamma, beta, y, rows, cols, eps, stream=None) -> None:
