@@ -108,6 +108,14 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Row and column tile of output tile `tile` in the order p.n_fastest selects.
+__host__ __device__ __forceinline__ int tile_row(const GemmParams& p, int tile, int m_tiles, int n_tiles) {
+  return p.n_fastest ? tile / n_tiles : tile % m_tiles;
+}
+__host__ __device__ __forceinline__ int tile_col(const GemmParams& p, int tile, int m_tiles, int n_tiles) {
+  return p.n_fastest ? tile % n_tiles : tile / m_tiles;
+}
+
 // Work item i (0, 1, ...) of CTA pair `pair` of P: output tile `tile` over K steps
 // [kb0, kb1).  Whole tiles come in rounds of P; with a split-K tail (p.sk_part) the
 // tiles from p.sk_full on are cut into p.sk_split K ranges each, and pair u takes range
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int mb = tile % m_tiles, nb = tile / m_tiles;
+        const int mb = tile_row(p, tile, m_tiles, n_tiles), nb = tile_col(p, tile, m_tiles, n_tiles);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) {
@@ -449,7 +457,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
-      const int mb = tile % m_tiles, nb = tile / m_tiles;
+      const int mb = tile_row(p, tile, m_tiles, n_tiles), nb = tile_col(p, tile, m_tiles, n_tiles);
       const int row = mb * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
       if (!epilogue_tile<BN, RL, false>(p, row, nb * BN, t_row, &tfull[acc], (it >> 1) & 1, abort_flag, grp, &tmC,
@@ -541,7 +549,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
       uint32_t phase = 0;
       int tile, kb0, kb1, unit;
       for (int i = 0; pair_work(p, pair, num_pairs, num_tiles, nk, i, tile, kb0, kb1, unit); ++i) {
-        const int mb = tile % m_tiles, nb = tile / m_tiles;
+        const int mb = tile_row(p, tile, m_tiles, n_tiles), nb = tile_col(p, tile, m_tiles, n_tiles);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, abort_flag, &g_gemm_err)) {
@@ -634,7 +642,7 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     int tile, kb0, kb1, unit;
     for (; pair_work(p, pair, num_pairs, num_tiles, nk, it, tile, kb0, kb1, unit); ++it) {
       const int acc = it & 1;
-      const int mb = tile % m_tiles, nb = tile / m_tiles;
+      const int mb = tile_row(p, tile, m_tiles, n_tiles), nb = tile_col(p, tile, m_tiles, n_tiles);
       const int row = mb * 2 * kBM + rank * kBM + quad * 32 + lane;
       const uint32_t t_row = tmem_base + acc * S::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
       if (unit >= 0) {
@@ -695,8 +703,9 @@ __global__ void __launch_bounds__(256) gemm_split_sum(const GemmParams p) {
   const int t = static_cast<int>(rest / (2 * kBM));  // split tile, 0-based after sk_full
   const int tile = p.sk_full + t;
   if (tile >= m_tiles * ((p.N + BN - 1) / BN)) return;
-  const int row = (tile % m_tiles) * 2 * kBM + r;
-  const int col = (tile / m_tiles) * BN + 4 * g;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int row = tile_row(p, tile, m_tiles, n_tiles) * 2 * kBM + r;
+  const int col = tile_col(p, tile, m_tiles, n_tiles) * BN + 4 * g;
   if (row >= p.M || col >= p.N) return;
   // every partial is loaded before the first add, so that the loads overlap
   float4 pv[kMaxSplit];
@@ -832,9 +841,18 @@ cudaError_t launch_pair(const GemmParams& p, cudaStream_t stream, int* kernels =
 
 size_t gemm_split_bytes() { return static_cast<size_t>(device_sm_count() / 2) * 2 * kBM * 256 * sizeof(float); }
 
-cudaError_t launch_gemm(const GemmParams& p, cudaStream_t stream, int qkv_mode, int* kernels) {
+cudaError_t launch_gemm(const GemmParams& p_in, cudaStream_t stream, int qkv_mode, int* kernels) {
   if (kernels) *kernels = 1;
-  if (p.M <= 0 || p.N <= 0 || p.K <= 0) return cudaSuccess;
+  if (p_in.M <= 0 || p_in.N <= 0 || p_in.K <= 0) return cudaSuccess;
+  // Row tiles fastest (CTAs running together share W's tiles through L2), unless A is
+  // both the larger operand and too large to stay in L2 between column tiles (above
+  // 48 MB): then column tiles run fastest, so that A is read from memory once.  On the
+  // fc2 product at 448x448 x 8 (A = 84 MB) this takes DRAM traffic from 223 to 130 MB
+  // per launch at the same time (ncu); smaller A keeps the other order, which measured
+  // 1-2% faster there.
+  GemmParams p = p_in;
+  const double a_bytes = 2.0 * p.M * p.K, w_bytes = 2.0 * p.N * p.K;
+  p.n_fastest = a_bytes > w_bytes && a_bytes > 48e6 ? 1 : 0;
   // Pairs of CTAs (256-row tiles) once there are enough rows to keep them busy.
   const bool pair = p.M >= 1024;
   if (qkv_mode) {

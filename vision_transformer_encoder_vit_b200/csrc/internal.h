@@ -106,6 +106,11 @@ struct GemmParams {
   // applies the epilogue.
   float* sk_part;
   int sk_full, sk_split;
+  // Tile order (set by launch_gemm): 0 walks the row tiles of A fastest, so that the CTAs
+  // running together share each tile of W through L2; 1 walks the column tiles fastest,
+  // so that they share each row tile of A (used when A is the larger operand, which is
+  // then read from memory once).
+  int n_fastest;
 };
 
 // Bytes of split-K scratch a product may use (one 256 x 256 fp32 tile per CTA pair).
