@@ -119,6 +119,22 @@ def test_linear_split_k_tail(M, N, K, use_bias, use_resid, act):
     assert torch.equal(out, out2)
 
 
+def test_linear_large_a_ragged_column_tiles_fastest():
+    # A above 48 MB and larger than W: the CTA pairs walk column tiles fastest.  Ragged M
+    # (40 rows in the last 256-row tile), ragged N (232 columns in the last tile), a
+    # partial K step; rows checked at a sample that includes the last tile.
+    M, N, K = 9000, 1000, 4104
+    A = S.make_matrix((M, K), 91)
+    W = S.make_matrix((N, K), 92, scale=0.02 * 50 / math.sqrt(K))
+    bias, resid = S.make_matrix((N,), 93, 0.1), S.make_matrix((M, N), 94)
+    out = empty_bf16(M, N)
+    V.vt_linear(dev_bf16(A), dev_bf16(W), dev_bf16(bias), dev_bf16(resid), out, M, N, K, 0)
+    V.vt_check()
+    rows = np.unique(np.concatenate([np.random.default_rng(95).choice(M, 256, replace=False), np.arange(M - 64, M)]))
+    ref = S.bf16_to_f64(A)[rows] @ S.bf16_to_f64(W).T + S.bf16_to_f64(bias) + S.bf16_to_f64(resid)[rows]
+    assert_close(host_f64(out)[rows], ref, what=f"linear {M}x{N}x{K}, column tiles fastest")
+
+
 def test_linear_residual_in_place():
     M, N, K = 384, 512, 256
     A, W = S.make_matrix((M, K), 1), S.make_matrix((N, K), 2, 0.05)
