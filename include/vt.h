@@ -321,7 +321,9 @@ VT_API vt_status vt_merge_project(vt_handle* h, const void* tower, const int32_t
  * attention).
  *   q, k, v  device bf16 [B, H, N, D];  o  device bf16 [B, N, H*D]
  *   pos_thw  device int32 [N, 3] token positions (t, h, w) for 3D RoPE of q and k, or
- *            NULL for none; sections / theta as in vt_config (ignored when NULL)
+ *            NULL for none; sections / theta as in vt_config (ignored when NULL).  The
+ *            rotation's cos and sin are single precision, taken of the angle after an
+ *            exact double-precision reduction to within half a turn (a few 1e-7 off).
  *   scale    > 0, usually 1/sqrt(D)
  *   ws       device workspace of vt_attention_workspace_bytes() (rotated q, k and the
  *            transposed v): 3 * B*H*D*ceil8(N) * 2 bytes, linear in N.

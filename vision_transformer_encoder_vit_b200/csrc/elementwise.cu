@@ -238,68 +238,212 @@ __global__ void __launch_bounds__(256) reorder_rows_kernel(const uint4* __restri
 }
 
 // ------------------------------------------------------ attention preparation
-// Rotates q and k by the 3D RoPE of each token's position (pairs (off+j, off+j+s/2)
-// of each axis block, angle pos_axis * theta^(-2j/s)) and copies them; one thread per
-// (token, pair), looping over batch and heads.
-__global__ void __launch_bounds__(256) rope_qk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
-                                                      bf16* __restrict__ qr, bf16* __restrict__ kr, int B, int H,
-                                                      int N, int D, const int32_t* __restrict__ pos, int s0, int s1,
-                                                      int s2, float theta) {
-  const int half = D / 2;
-  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long>(N) * half) return;
-  const int n = static_cast<int>(idx / half);
-  const int pi = static_cast<int>(idx - static_cast<long>(n) * half);
-  int axis, j, off, s;
-  if (pi < s0 / 2) {
-    axis = 0; j = pi; off = 0; s = s0;
-  } else if (pi < (s0 + s1) / 2) {
-    axis = 1; j = pi - s0 / 2; off = s0; s = s1;
-  } else {
-    axis = 2; j = pi - (s0 + s1) / 2; off = s0 + s1; s = s2;
-  }
-  const double inv_freq = pow(static_cast<double>(theta), -2.0 * j / s);
-  const double ang = static_cast<double>(pos[n * 3 + axis]) * inv_freq;
-  double sd, cd;
-  sincos(ang, &sd, &cd);
-  const float c = static_cast<float>(cd), sn = static_cast<float>(sd);
-  const int c1 = off + j, c2 = off + j + s / 2;
-  for (int bh = 0; bh < B * H; ++bh) {
-    const size_t base = (static_cast<size_t>(bh) * N + n) * D;
-    float a = __bfloat162float(q[base + c1]), bb = __bfloat162float(q[base + c2]);
-    qr[base + c1] = __float2bfloat16_rn(a * c - bb * sn);
-    qr[base + c2] = __float2bfloat16_rn(bb * c + a * sn);
-    a = __bfloat162float(k[base + c1]);
-    bb = __bfloat162float(k[base + c2]);
-    kr[base + c1] = __float2bfloat16_rn(a * c - bb * sn);
-    kr[base + c2] = __float2bfloat16_rn(bb * c + a * sn);
-  }
-}
+// q and k are rotated by the 3D RoPE of each token's position: within the axis block
+// [off, off + s) of an axis, channels (off + j, off + j + s/2) form pair j, turned by
+// the angle pos_axis * theta^(-2j/s).  v is transposed to vt [B*H, D, ld_vt].
+//
+// Persistent kernel over items (token tile of kPrepTok tokens, (image, head) pair),
+// the pair index fastest; each block takes one contiguous, balanced range of items
+// and recomputes its tokens' (cos, sin) only when the tile changes.  A block has
+// kPrepTok * D / 8 threads, so that each thread owns one task of each kind per item:
+//  - q and k (kMode 0: copy, 1: RoPE when every half section is a multiple of 8
+//    channels): one pair of 16-byte chunks (channels c..c+7 and their partners) of one
+//    token, rotated in registers;
+//  - v: one 16-byte chunk staged in shared memory (rows an odd number of words apart,
+//    so the column reads fall on distinct banks), then one eight-token run of one vt
+//    column written with a 16-byte store.
+// The next item's 16-byte loads are issued before the current item's stores.  kMode 2
+// (other section widths) rotates q and k one channel pair at a time.
+constexpr int kPrepTok = 32;
 
-// v [B*H, N, D] -> vt [B*H, D, ld_vt] through a 64-token shared tile.
-__global__ void __launch_bounds__(256) transpose_v_kernel(const bf16* __restrict__ v, bf16* __restrict__ vt, int N,
-                                                          int D, int ld_vt) {
-  __shared__ bf16 tile[64][128 + 2];
-  const int n0 = blockIdx.x * 64;
-  const size_t bh = blockIdx.y;
-  const bf16* src = v + bh * N * static_cast<size_t>(D);
-  for (int e = threadIdx.x; e < 64 * D; e += blockDim.x) {
-    const int r = e / D, c = e - (e / D) * D;
-    if (n0 + r < N) tile[r][c] = src[static_cast<size_t>(n0 + r) * D + c];
+template <int D, int kMode>
+__global__ void __launch_bounds__(kPrepTok * D / 8) attention_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
+                                                               const bf16* __restrict__ v, bf16* __restrict__ qr,
+                                                               bf16* __restrict__ kr, bf16* __restrict__ vt,
+                                                               long long BH, int N, int ld_vt,
+                                                               const int32_t* __restrict__ pos, int s0, int s1, int s2,
+                                                               float theta) {
+  constexpr int kThreads = kPrepTok * D / 8, kC8 = D / 8, kPC = D / 16, kHalf = D / 2, kRowWords = D / 2 + 1;
+  constexpr int kRuns = kPrepTok / 8;  // eight-token runs of a vt column
+  constexpr bool kRope = kMode != 0;
+  __shared__ uint32_t vtile[kPrepTok][kRowWords];
+  __shared__ __align__(16) float2 cs[kRope ? kPrepTok : 1][kHalf];  // (cos, sin) per token and pair
+  __shared__ double freq[kRope ? kHalf : 1];  // theta^(-2j/s) / pi per pair
+  __shared__ int freq_axis[kRope ? kHalf : 1];
+  __shared__ int chunk_map[kPC];  // first chunk | partner chunk << 8 | first pair << 16
+  const int tid = threadIdx.x;
+  const long long tiles = (N + kPrepTok - 1) / kPrepTok, items = tiles * BH;
+  const long long per = items / gridDim.x, extra = items % gridDim.x;
+  const long long it0 = blockIdx.x * per + min(static_cast<long long>(blockIdx.x), extra);
+  const long long it1 = it0 + per + (blockIdx.x < extra ? 1 : 0);
+  if (it0 >= it1) return;
+  if (tid == 0) {
+    if (kMode == 1) {
+      int n = 0;
+      const int sec[3] = {s0, s1, s2};
+      for (int a = 0, off = 0; a < 3; off += sec[a], ++a)
+        for (int c = 0; c < sec[a] / 16; ++c)
+          chunk_map[n++] = (off / 8 + c) | ((off / 8 + sec[a] / 16 + c) << 8) | ((off / 2 + 8 * c) << 16);
+    } else {
+      for (int c = 0; c < kPC; ++c) chunk_map[c] = 2 * c | ((2 * c + 1) << 8);
+    }
   }
+  if (kRope) {
+    for (int pi = tid; pi < kHalf; pi += kThreads) {
+      int axis, j, s;
+      if (pi < s0 / 2) {
+        axis = 0; j = pi; s = s0;
+      } else if (pi < (s0 + s1) / 2) {
+        axis = 1; j = pi - s0 / 2; s = s1;
+      } else {
+        axis = 2; j = pi - (s0 + s1) / 2; s = s2;
+      }
+      freq[pi] = pow(static_cast<double>(theta), -2.0 * j / s) / 3.141592653589793;
+      freq_axis[pi] = axis;
+    }
+  }
+  // This thread's tasks: q/k chunk pair (matrix qm, token qt, chunk pair qc); v chunk
+  // (token vt_t, chunk vc); vt run (channel td, tokens 8 * tc ..).
+  const int qm = tid >= kThreads / 2, qi = tid - qm * (kThreads / 2), qt = qi / kPC, qc = qi - qt * kPC;
+  const int vt_t = tid / kC8, vc = tid - vt_t * kC8;
+  const int td = tid / kRuns, tc = tid - td * kRuns;
+  const bf16* qsrc = qm ? k : q;
+  bf16* qdst = qm ? kr : qr;
   __syncthreads();
-  bf16* dst = vt + bh * D * static_cast<size_t>(ld_vt);
-  for (int e = threadIdx.x; e < 64 * D; e += blockDim.x) {
-    const int c = e / 64, r = e - (e / 64) * 64;
-    if (n0 + r < N) dst[static_cast<size_t>(c) * ld_vt + n0 + r] = tile[r][c];
+  const int cm = chunk_map[qc];
+  uint4 na = make_uint4(0, 0, 0, 0), nb = na, nv = na;  // the next item's chunks
+  auto load = [&](long long it) {
+    const long long tl = it / BH, bh = it - tl * BH;
+    const int n0 = static_cast<int>(tl) * kPrepTok, rows = min(kPrepTok, N - n0);
+    const size_t row0 = (static_cast<size_t>(bh) * N + n0) * D;
+    if (kMode != 2 && qt < rows) {
+      const uint4* src = reinterpret_cast<const uint4*>(qsrc + row0 + static_cast<size_t>(qt) * D);
+      na = __ldg(src + (cm & 255));
+      nb = __ldg(src + ((cm >> 8) & 255));
+    }
+    if (vt_t < rows) nv = __ldg(reinterpret_cast<const uint4*>(v + row0) + tid);
+  };
+  load(it0);
+  long long table_tile = -1;
+  for (long long it = it0; it < it1; ++it) {
+    const long long tl = it / BH, bh = it - tl * BH;
+    const int n0 = static_cast<int>(tl) * kPrepTok, rows = min(kPrepTok, N - n0);
+    const size_t row0 = (static_cast<size_t>(bh) * N + n0) * D;
+    __syncthreads();  // the previous item's vt columns and (cos, sin) read
+    if (kRope && tl != table_tile) {
+      // Angle in half-turns, reduced exactly (in double) to [-1, 1] before the
+      // single-precision sincospi: cos and sin within a few 1e-7 of exact.
+      for (int e = tid; e < kPrepTok * kHalf; e += kThreads) {
+        const int t = e / kHalf, pi = e - t * kHalf;
+        if (t < rows) {
+          double x = static_cast<double>(pos[static_cast<size_t>(n0 + t) * 3 + freq_axis[pi]]) * freq[pi];
+          x -= 2.0 * rint(0.5 * x);
+          float sn, c;
+          sincospif(static_cast<float>(x), &sn, &c);
+          cs[t][pi] = make_float2(c, sn);
+        }
+      }
+      table_tile = tl;
+    }
+    if (vt_t < rows) {
+      uint32_t* w = &vtile[vt_t][4 * vc];
+      w[0] = nv.x; w[1] = nv.y; w[2] = nv.z; w[3] = nv.w;
+    }
+    const uint4 ca = na, cb = nb;
+    __syncthreads();
+    if (it + 1 < it1) load(it + 1);  // in flight while this item is written
+    if (kMode != 2) {
+      if (qt < rows) {
+        uint4* dst = reinterpret_cast<uint4*>(qdst + row0 + static_cast<size_t>(qt) * D);
+        if (kMode == 0) {
+          dst[cm & 255] = ca;
+          dst[(cm >> 8) & 255] = cb;
+        } else {
+          const float4* c4 = reinterpret_cast<const float4*>(&cs[qt][cm >> 16]);
+          const uint32_t* wa = reinterpret_cast<const uint32_t*>(&ca);
+          const uint32_t* wb = reinterpret_cast<const uint32_t*>(&cb);
+          uint32_t oa[4], ob[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 r = c4[i];  // (cos, sin) of pairs 2i, 2i+1 of the chunk
+            const float2 x = unpack_bf16x2(wa[i]), y = unpack_bf16x2(wb[i]);
+            oa[i] = pack_bf16x2(x.x * r.x - y.x * r.y, x.y * r.z - y.y * r.w);
+            ob[i] = pack_bf16x2(y.x * r.x + x.x * r.y, y.y * r.z + x.y * r.w);
+          }
+          dst[cm & 255] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+          dst[(cm >> 8) & 255] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        }
+      }
+    } else {
+      for (int e = tid; e < 2 * kPrepTok * kHalf; e += kThreads) {
+        const int m = e / (kPrepTok * kHalf), r = e - m * (kPrepTok * kHalf);
+        const int t = r / kHalf, pi = r - t * kHalf;
+        if (t >= rows) continue;
+        int c1, s;
+        if (pi < s0 / 2) {
+          c1 = pi; s = s0;
+        } else if (pi < (s0 + s1) / 2) {
+          c1 = s0 + pi - s0 / 2; s = s1;
+        } else {
+          c1 = s0 + s1 + pi - (s0 + s1) / 2; s = s2;
+        }
+        const int c2 = c1 + s / 2;
+        const size_t base = row0 + static_cast<size_t>(t) * D;
+        const bf16* src = m ? k : q;
+        bf16* dst = m ? kr : qr;
+        const float x = __bfloat162float(src[base + c1]), y = __bfloat162float(src[base + c2]);
+        const float2 a = cs[t][pi];
+        dst[base + c1] = __float2bfloat16_rn(x * a.x - y * a.y);
+        dst[base + c2] = __float2bfloat16_rn(y * a.x + x * a.y);
+      }
+    }
+    if (8 * tc < rows) {
+      const int t0 = 8 * tc;
+      uint32_t x[4];  // tokens t0 .. t0+7 of channel td, two per word
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint16_t lo = reinterpret_cast<const uint16_t*>(&vtile[t0 + 2 * i][0])[td];
+        const uint16_t hi = reinterpret_cast<const uint16_t*>(&vtile[t0 + 2 * i + 1][0])[td];
+        x[i] = lo | (static_cast<uint32_t>(hi) << 16);
+      }
+      bf16* dst = vt + (static_cast<size_t>(bh) * D + td) * ld_vt + n0 + t0;
+      if (t0 + 8 <= rows) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(x[0], x[1], x[2], x[3]);
+      } else {
+        uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (i < rows - t0) d16[i] = static_cast<uint16_t>(x[i >> 1] >> (16 * (i & 1)));
+      }
+    }
   }
 }
 
-// Plain copy of q or k when no rotation is requested.
-__global__ void copy_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, size_t n16) {
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n16;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    out[i] = in[i];
+template <int D, int kMode>
+cudaError_t launch_prep(const bf16* q, const bf16* k, const bf16* v, bf16* qr, bf16* kr, bf16* vt, long long BH, int N,
+                        int ld_vt, const int32_t* pos, const int* sec, float theta, cudaStream_t stream) {
+  static int resident = 0;  // blocks of this kernel one SM holds
+  if (!resident) {
+    int r = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, attention_prep_kernel<D, kMode>, kPrepTok * D / 8, 0);
+    resident = r < 1 ? 1 : r;
+  }
+  const long long items = (N + kPrepTok - 1) / kPrepTok * BH;
+  const long long cap = static_cast<long long>(resident) * device_sm_count();
+  const unsigned grid = static_cast<unsigned>(items < cap ? items : cap);
+  attention_prep_kernel<D, kMode><<<grid, kPrepTok * D / 8, 0, stream>>>(q, k, v, qr, kr, vt, BH, N, ld_vt, pos,
+                                                              sec ? sec[0] : 0, sec ? sec[1] : 0, sec ? sec[2] : 0,
+                                                              theta);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_prep_d(const bf16* q, const bf16* k, const bf16* v, bf16* qr, bf16* kr, bf16* vt, long long BH,
+                          int N, int ld_vt, const int32_t* pos, const int* sec, float theta, cudaStream_t stream) {
+  if (!pos) return launch_prep<D, 0>(q, k, v, qr, kr, vt, BH, N, ld_vt, nullptr, nullptr, 0.f, stream);
+  if (sec[0] % 16 == 0 && sec[1] % 16 == 0 && sec[2] % 16 == 0)
+    return launch_prep<D, 1>(q, k, v, qr, kr, vt, BH, N, ld_vt, pos, sec, theta, stream);
+  return launch_prep<D, 2>(q, k, v, qr, kr, vt, BH, N, ld_vt, pos, sec, theta, stream);
 }
 
 }  // namespace
@@ -363,21 +507,16 @@ cudaError_t launch_attention_prep(const void* q, const void* k, const void* v, v
                                   int H, int N, int D, int ld_vt, const int32_t* pos, const int sections[3],
                                   float theta, cudaStream_t stream) {
   if (B <= 0 || H <= 0 || N <= 0) return cudaSuccess;
-  if (pos) {
-    const long threads = static_cast<long>(N) * (D / 2);
-    rope_qk_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-        static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<bf16*>(qr), static_cast<bf16*>(kr), B,
-        H, N, D, pos, sections[0], sections[1], sections[2], theta);
-  } else {
-    const size_t n16 = static_cast<size_t>(B) * H * N * D / 8;
-    copy_kernel<<<1184, 256, 0, stream>>>(static_cast<const uint4*>(q), static_cast<uint4*>(qr), n16);
-    copy_kernel<<<1184, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<uint4*>(kr), n16);
+  const long long BH = static_cast<long long>(B) * H;
+  const bf16 *Q = static_cast<const bf16*>(q), *K = static_cast<const bf16*>(k), *V = static_cast<const bf16*>(v);
+  bf16 *QR = static_cast<bf16*>(qr), *KR = static_cast<bf16*>(kr), *VT = static_cast<bf16*>(vt);
+  switch (D) {
+    case 32: return launch_prep_d<32>(Q, K, V, QR, KR, VT, BH, N, ld_vt, pos, sections, theta, stream);
+    case 64: return launch_prep_d<64>(Q, K, V, QR, KR, VT, BH, N, ld_vt, pos, sections, theta, stream);
+    case 80: return launch_prep_d<80>(Q, K, V, QR, KR, VT, BH, N, ld_vt, pos, sections, theta, stream);
+    case 96: return launch_prep_d<96>(Q, K, V, QR, KR, VT, BH, N, ld_vt, pos, sections, theta, stream);
+    default: return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dim3 grid((N + 63) / 64, B * H);
-  transpose_v_kernel<<<grid, 256, 0, stream>>>(static_cast<const bf16*>(v), static_cast<bf16*>(vt), N, D, ld_vt);
-  return cudaGetLastError();
 }
 
 }  // namespace vt
