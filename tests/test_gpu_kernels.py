@@ -186,7 +186,7 @@ def test_patch_unfold_is_exact(B, H, W, order):
 
 # -------------------------------------------------------------- attention
 
-def _attn_case(B, H, N, D, rope, seed, sections=None, grid=None, rows=None):
+def _attn_case(B, H, N, D, rope, seed, sections=None, grid=None, rows=None, t_axis=False):
     q, k, v = S.make_qkv(B, H, N, D, seed)
     dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
     o = empty_bf16(B, N, H * D)
@@ -196,7 +196,8 @@ def _attn_case(B, H, N, D, rope, seed, sections=None, grid=None, rows=None):
     if rope:
         if grid is None:
             pos = np.random.default_rng(seed).integers(0, 200, size=(N, 3)).astype(np.int32)
-            pos[:, 0] = 0
+            if not t_axis:
+                pos[:, 0] = 0
         else:
             pos = R.positions_raster(*grid).astype(np.int32)
         dpos = torch.from_numpy(pos).cuda()
@@ -223,6 +224,25 @@ def test_attention_d80_ragged(N):
 @pytest.mark.parametrize("N", [64, 200, 2304])
 def test_attention_d32(N):
     _attn_case(2, 4, N, 32, True, N + 1, sections=(8, 12, 12))
+
+
+# The preparation pass of vt_attention has three forms: a plain copy (no RoPE), the
+# rotation of 16-byte channel chunks (every section a multiple of 16) and the rotation
+# one channel pair at a time (other sections).  Ragged token counts leave a partial
+# 32-token tile; positions include the t axis.
+@pytest.mark.parametrize("B,H,N,D,sections", [
+    (3, 5, 1001, 80, (16, 32, 32)),
+    (1, 4, 250, 64, (16, 16, 32)),
+    (2, 4, 777, 64, (16, 24, 24)),
+    (2, 3, 517, 96, (32, 32, 32)),
+    (1, 3, 333, 96, (32, 16, 48)),
+    (1, 3, 45, 96, (24, 36, 36)),
+    (2, 2, 70, 32, (0, 16, 16)),
+    (1, 2, 300, 64, None),
+    (1, 2, 301, 96, None),
+])
+def test_attention_prep_forms(B, H, N, D, sections):
+    _attn_case(B, H, N, D, sections is not None, B * N + D, sections=sections, t_axis=True)
 
 
 def test_attention_rope_raster_grid_448():
