@@ -410,6 +410,9 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     if (lane == 0) {
       // ----------------------------------------------------------------- MMA
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      // Descriptors of stage 0, computed once: later stages and K steps add to the
+      // start-address field (address / 16; shared addresses stay below 256 KB).
+      const uint64_t a_desc0 = smem_desc(smem_u32(sA), 1024, 2), b_desc0 = smem_desc(smem_u32(sB), 1024, 2);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -426,13 +429,10 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * S::A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * S::B_BYTES);
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage * (S::A_BYTES >> 4));
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage * (S::B_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            umma_bf16(d_tmem, smem_desc(a_addr + kk * 32, 1024, 2), smem_desc(b_addr + kk * 32, 1024, 2), idesc,
-                      (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kBK / 16; ++kk) umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           issued_any = true;
           umma_commit(&empty[stage]);
           if (++stage == S::STAGES) {
@@ -588,6 +588,12 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
     if (lane == 0 && rank == 0) {
       // -------------------------------------------------------- MMA (even CTA)
       constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, BN);
+      // Descriptors of stage 0 and the cluster addresses of the stage-0 empty barriers,
+      // computed once: the descriptor's start-address field holds address / 16 (shared
+      // addresses stay below 256 KB, so adding stage and K-step offsets never carries out
+      // of it), and the barriers of later stages follow at 8-byte steps.
+      const uint64_t a_desc0 = smem_desc(smem_u32(sA), 1024, 2), b_desc0 = smem_desc(smem_u32(sB), 1024, 2);
+      const uint32_t e_lead0 = mapa_shared(smem_u32(&empty[0]), 0), e_peer0 = mapa_shared(smem_u32(&empty[0]), 1);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -605,17 +611,14 @@ __global__ void __launch_bounds__(Epi<RL>::THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * S::A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * S::B_BYTES);
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage * (S::A_BYTES >> 4));
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage * (S::B_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            umma_bf16_pair(d_tmem, smem_desc(a_addr + kk * 32, 1024, 2), smem_desc(b_addr + kk * 32, 1024, 2),
-                           idesc, (kb > kb0 || kk != 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk != 0) ? 1u : 0u);
           issued_any = true;
-          const uint32_t e_local = smem_u32(&empty[stage]);
-          umma_commit_pair(mapa_shared(e_local, 0));
-          umma_commit_pair(mapa_shared(e_local, 1));
+          umma_commit_pair(e_lead0 + 8u * stage);
+          umma_commit_pair(e_peer0 + 8u * stage);
           if (++stage == S::STAGES) {
             stage = 0;
             phase ^= 1u;
