@@ -229,14 +229,16 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, int row, int 
               v[8 * g + 2 * i] *= th ? gelu_tanh_grad(z.x) : gelu_erf_grad(z.x);
               v[8 * g + 2 * i + 1] *= th ? gelu_tanh_grad(z.y) : gelu_erf_grad(z.y);
             }
-          } else {
+          } else if (p.act == ACT_GELU_TANH) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float x = v[8 * g + i];
-              if (p.act == ACT_GELU_TANH) x = gelu_tanh(x);
-              else if (p.act == ACT_GELU_ERF) x = gelu_erf(x);
-              v[8 * g + i] = x;
+            for (int i = 0; i < 4; ++i) {
+              const float2 y = gelu_tanh2(make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]));
+              v[8 * g + 2 * i] = y.x;
+              v[8 * g + 2 * i + 1] = y.y;
             }
+          } else if (p.act == ACT_GELU_ERF) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[8 * g + i] = gelu_erf(v[8 * g + i]);
           }
           if (resid && p.act < ACT_DGELU_TANH) add_bf16x8(v + 8 * g, rq[g]);
         }
@@ -735,10 +737,16 @@ __global__ void __launch_bounds__(256) gemm_split_sum(const GemmParams p) {
     v[3] += b.y;
   };
   if (p.bias) add4(__ldg(reinterpret_cast<const uint2*>(static_cast<const bf16*>(p.bias) + col)));
+  if (p.act == ACT_GELU_TANH) {  // the tile epilogue's packed form, so that split and whole tiles agree
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    if (p.act == ACT_GELU_TANH) v[c] = gelu_tanh(v[c]);
-    else if (p.act == ACT_GELU_ERF) v[c] = gelu_erf(v[c]);
+    for (int c = 0; c < 4; c += 2) {
+      const float2 y = gelu_tanh2(make_float2(v[c], v[c + 1]));
+      v[c] = y.x;
+      v[c + 1] = y.y;
+    }
+  } else if (p.act == ACT_GELU_ERF) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) v[c] = gelu_erf(v[c]);
   }
   if (p.resid)
     add4(*reinterpret_cast<const uint2*>(static_cast<const bf16*>(p.resid) + static_cast<size_t>(row) * p.ldr + col));

@@ -356,6 +356,14 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return d;
 }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0,%1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   float2 d;
   asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
@@ -377,12 +385,15 @@ __device__ __forceinline__ float fast_tanh(float x) {
   return y;
 }
 
-// GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
-__device__ __forceinline__ float gelu_tanh(float x) {
-  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-  const float k1 = 0.044715f;
-  float u = k0 * fmaf(k1 * x * x, x, x);
-  return 0.5f * x * (1.0f + fast_tanh(u));
+// GELU, tanh form, 0.5 x (1 + tanh(k0 (x + k1 x^3))) with k0 = sqrt(2/pi), k1 = 0.044715,
+// for two elements on the packed fp32 pipe: u = x (k0 + k0 k1 x^2), result h + h tanh(u)
+// with h = x / 2.
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) {
+  const float k0 = 0.7978845608028654f, k0k1 = 0.7978845608028654f * 0.044715f;
+  const float2 x2 = fmul2(x, x);
+  const float2 u = fmul2(x, ffma2(x2, make_float2(k0k1, k0k1), make_float2(k0, k0)));
+  const float2 h = fmul2(x, make_float2(0.5f, 0.5f));
+  return ffma2(h, make_float2(fast_tanh(u.x), fast_tanh(u.y)), h);
 }
 
 // GELU, exact form: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)).
@@ -439,9 +450,9 @@ __device__ __forceinline__ void add_bf16x8(float* v, uint4 u) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 f = unpack_bf16x2(w[i]);
-    v[2 * i] += f.x;
-    v[2 * i + 1] += f.y;
+    const float2 r = fadd2(make_float2(v[2 * i], v[2 * i + 1]), unpack_bf16x2(w[i]));
+    v[2 * i] = r.x;
+    v[2 * i + 1] = r.y;
   }
 }
 
